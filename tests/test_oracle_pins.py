@@ -1,0 +1,234 @@
+"""Pins of the CPU oracle against things other than itself.
+
+* brute force on tiny inputs (tests/brute.py: numpy + lexsort, written apart);
+* hand-worked fixtures (tests/golden/*.txt, each with its derivation);
+* closed forms (ramps, constant keys) whose answer is known without a program;
+* invariants that the method's definition implies (g=1, Kc >= prefix,
+  causality, Reuse sharing, row sizes);
+* the pages' demo shape (seq_len, num_heads, top_k) = (1024, 8, 64).
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from tests import brute
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def int_inputs(rng, L, H, d, lo=-3, hi=3):
+    """Small-integer inputs: every dot product and proxy sum is exact, ties are frequent."""
+    q = rng.integers(lo, hi + 1, size=(L, H, d)).astype(np.float32)
+    k = rng.integers(lo, hi + 1, size=(L, H, d)).astype(np.float32)
+    return synthetic.bf16_from_f32(q), synthetic.bf16_from_f32(k)
+
+
+def bits(vals):
+    return synthetic.bf16_from_f32(np.asarray(vals, dtype=np.float32))
+
+
+# ---------------------------------------------------------------- brute force
+@pytest.mark.parametrize("seed", range(24))
+def test_prefill_matches_brute_force_exact_inputs(seed):
+    rng = np.random.default_rng(1000 + seed)
+    L = int(rng.integers(1, 60))
+    H = int(rng.integers(1, 3))
+    d = int(rng.choice([2, 4, 8]))
+    g = int(rng.choice([1, 2, 3, 5, 8]))
+    top_k = int(rng.integers(1, 9))
+    Kc = int(rng.integers(top_k, 3 * top_k + 1))
+    q, k = int_inputs(rng, L, H, d, -2, 2)
+    for mode in (oracle.REFINE, oracle.REUSE):
+        got = oracle.prefill(q, k, g, top_k, Kc, mode)["out"]
+        want = brute.prefill(q, k, g, top_k, Kc, mode)
+        np.testing.assert_array_equal(got, want, err_msg=f"mode={mode} L={L} g={g} k={top_k} Kc={Kc}")
+    got = oracle.dense(q, k, top_k)["out"]
+    np.testing.assert_array_equal(got, brute.dense(q, k, top_k))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_prefill_matches_brute_force_gaussian(seed):
+    rng = np.random.default_rng(2000 + seed)
+    L = int(rng.integers(20, 120))
+    g = int(rng.choice([2, 4, 8]))
+    q, k = synthetic.gen_prefill(L, 2, 16, seed=seed, rho=0.9)
+    for mode in (oracle.REFINE, oracle.REUSE):
+        got = oracle.prefill(q, k, g, 6, 12, mode)["out"]
+        np.testing.assert_array_equal(got, brute.prefill(q, k, g, 6, 12, mode))
+    np.testing.assert_array_equal(oracle.dense(q, k, 6)["out"], brute.dense(q, k, 6))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_decode_matches_brute_force(seed):
+    rng = np.random.default_rng(3000 + seed)
+    g = int(rng.choice([1, 2, 3]))
+    B = int(rng.integers(1, 4))
+    lens = rng.integers(0, 40, size=B) + g
+    cu = np.zeros(B + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    H, d = 2, 4
+    q = synthetic.bf16_from_f32(rng.integers(-2, 3, size=(B, g, H, d)).astype(np.float32))
+    kc = synthetic.bf16_from_f32(rng.integers(-2, 3, size=(int(cu[-1]), H, d)).astype(np.float32))
+    bi, hi = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+    for mode in (oracle.REFINE, oracle.REUSE):
+        r = oracle.decode_units(q, kc, cu, g, 4, 9, mode, bi.ravel(), hi.ravel())
+        got = r["out"].reshape(B, H, g, 4).transpose(0, 2, 1, 3)
+        np.testing.assert_array_equal(got, brute.decode(q, kc, cu, g, 4, 9, mode))
+
+
+# ------------------------------------------------------------ golden fixtures
+def _load_worked():
+    rows = {}
+    vals = {}
+    with open(os.path.join(GOLD, "worked_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, *rest = line.split()
+            if head in ("keys", "queries", "proxies"):
+                vals[head] = [[float(x) for x in v.split(",")] for v in rest]
+            else:
+                top_k, Kc = int(rest[0]), int(rest[1])
+                body = " ".join(rest[2:]).split("|")
+                rows[(head, top_k, Kc)] = [[int(x) for x in r.split(",")] for r in body]
+    return vals, rows
+
+
+def test_worked_example():
+    vals, rows = _load_worked()
+    k = bits(vals["keys"])[:, None, :]
+    q = bits(vals["queries"])[:, None, :]
+    for (mode, top_k, Kc), want in rows.items():
+        if mode == "dense":
+            got = oracle.dense(q, k, top_k)["out"][:, 0]
+        else:
+            m = oracle.REFINE if mode == "refine" else oracle.REUSE
+            r = oracle.prefill(q, k, 2, top_k, Kc, m)
+            got = r["out"][:, 0]
+            proxies = synthetic.bf16_to_f32(r["proxy"][:, 0])
+            np.testing.assert_array_equal(proxies, np.asarray(vals["proxies"], np.float32))
+        np.testing.assert_array_equal(got, np.asarray(want), err_msg=f"{mode} k={top_k} Kc={Kc}")
+
+
+def test_proxy_rounding_fixture():
+    with open(os.path.join(GOLD, "proxy_rounding.txt")) as f:
+        cases = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    for members, want in cases:
+        m = [float(x) for x in members.split(",")]
+        n = len(m)
+        q = bits(m)[:, None, None]                       # [n, 1, 1]: one group of n members
+        k = bits([1.0] * n)[:, None, None]
+        r = oracle.prefill_units(q, k, n, 1, 1, oracle.REFINE, [0], [0])
+        assert synthetic.bf16_to_f32(r["proxy"][0])[0] == np.float32(float(want)), members
+
+
+# --------------------------------------------------------------- closed forms
+def ramp_keys(L, d, sign=1.0):
+    """k_j = sign*(j+1)*e_0 (exact in bf16 for j < 256)."""
+    k = np.zeros((L, 1, d), np.float32)
+    k[:, 0, 0] = sign * (np.arange(L) + 1)
+    return synthetic.bf16_from_f32(k)
+
+
+@pytest.mark.parametrize("top_k", [1, 3, 8])
+def test_dense_ramp_picks_latest_keys(top_k):
+    L, d = 40, 4
+    q = np.zeros((L, 1, d), np.float32)
+    q[:, 0, 0] = 1.0
+    out = oracle.dense(synthetic.bf16_from_f32(q), ramp_keys(L, d), top_k)["out"][:, 0]
+    for pos in range(L):
+        want = list(range(max(0, pos - top_k), pos)) + [-1] * max(0, top_k - pos)
+        assert list(out[pos]) == want, pos
+
+
+def test_constant_keys_ties_go_to_lowest_index():
+    L, d, top_k = 30, 4, 5
+    rng = np.random.default_rng(7)
+    q = synthetic.bf16_from_f32(rng.standard_normal((L, 1, d)).astype(np.float32))
+    k = synthetic.bf16_from_f32(np.ones((L, 1, d), np.float32))
+    want = np.array([[j if j < min(top_k, pos) else -1 for j in range(top_k)] for pos in range(L)])
+    np.testing.assert_array_equal(oracle.dense(q, k, top_k)["out"][:, 0], want)
+    for g in (2, 4):
+        r = oracle.prefill(q, k, g, top_k, 2 * top_k, oracle.REFINE)["out"][:, 0]
+        np.testing.assert_array_equal(r, want)
+        r = oracle.prefill(q, k, g, top_k, 2 * top_k, oracle.REUSE)["out"][:, 0]
+        for pos in range(L):
+            s = (pos // g) * g
+            assert list(r[pos]) == [j if j < min(top_k, s) else -1 for j in range(top_k)]
+
+
+def test_refine_rescoring_uses_member_queries():
+    """Proxy points up the ramp, the second member points down: its picks are the oldest candidates."""
+    L, d, g, top_k, Kc = 48, 4, 2, 3, 6
+    q = np.zeros((L, 1, d), np.float32)
+    q[0::2, 0, 0] = 3.0     # first member of each group
+    q[1::2, 0, 0] = -1.0    # second member; proxy = +1 e_0
+    r = oracle.prefill(synthetic.bf16_from_f32(q), ramp_keys(L, d), g, top_k, Kc, oracle.REFINE)
+    out = r["out"][:, 0]
+    for s in range(0, L, g):
+        last = s + 1
+        C = list(range(max(0, last - Kc), last))            # the Kc largest j < last
+        V0 = [j for j in C if j < s]
+        assert list(out[s]) == (V0[-top_k:] + [-1] * (top_k - len(V0[-top_k:]))), s
+        V1 = [j for j in C if j < s + 1]
+        sel = V1[:top_k]
+        assert list(out[s + 1]) == sel + [-1] * (top_k - len(sel)), s + 1
+
+
+# ------------------------------------------------------------------ invariants
+@pytest.mark.parametrize("seed", range(4))
+def test_invariants(seed):
+    rng = np.random.default_rng(4000 + seed)
+    L, H, d = int(rng.integers(30, 90)), 2, 8
+    q, k = synthetic.gen_prefill(L, H, d, seed=seed)
+    top_k = int(rng.integers(2, 9))
+    dense = oracle.dense(q, k, top_k)["out"]
+    # g = 1: the proxy of one query is that query, so Refine and Reuse are dense.
+    np.testing.assert_array_equal(oracle.prefill(q, k, 1, top_k, 2 * top_k, oracle.REFINE)["out"], dense)
+    np.testing.assert_array_equal(oracle.prefill(q, k, 1, top_k, top_k, oracle.REUSE)["out"], dense)
+    for g in (3, 8):
+        # Kc >= every scan prefix: Refine sees every key and equals dense.
+        np.testing.assert_array_equal(oracle.prefill(q, k, g, top_k, L, oracle.REFINE)["out"], dense)
+        ref = oracle.prefill(q, k, g, top_k, 2 * top_k, oracle.REFINE)["out"]
+        reu = oracle.prefill(q, k, g, top_k, 2 * top_k, oracle.REUSE)["out"]
+        pos = np.arange(L)[:, None, None]
+        for out in (ref, reu, dense):
+            valid = out >= 0
+            assert np.all(out[valid] < np.broadcast_to(pos, out.shape)[valid])       # causal
+            # valid entries first, strictly ascending, unique
+            assert np.all(np.diff(valid.astype(int), axis=-1) <= 0)
+            o = np.where(valid, out, 10**9)
+            assert np.all(np.diff(o, axis=-1)[valid[..., 1:]] > 0)
+        for s in range(0, L, g):                                   # Reuse shared in a group
+            e = min(s + g, L)
+            assert np.all(reu[s:e] == reu[s])
+        n_valid = (ref >= 0).sum(-1)
+        want = np.minimum(top_k, np.arange(L))[:, None]
+        if 2 * top_k >= top_k + g - 1:
+            np.testing.assert_array_equal(n_valid, np.broadcast_to(want, n_valid.shape))
+        np.testing.assert_array_equal((dense >= 0).sum(-1), np.broadcast_to(want, n_valid.shape))
+
+
+def test_edges_and_scores_consistent():
+    q, k = synthetic.gen_prefill(64, 1, 8, seed=11)
+    r = oracle.dense(q, k, 4)
+    qf, kf = brute.decode_bf16(q), brute.decode_bf16(k)
+    for pos in range(5, 64):
+        sel = r["out"][pos, 0]
+        np.testing.assert_allclose(r["score"][pos, 0], kf[sel, 0] @ qf[pos, 0], rtol=1e-12)
+        allsc = np.sort(kf[:pos, 0] @ qf[pos, 0])[::-1]
+        np.testing.assert_allclose(r["edge"][pos, 0], allsc[3:5], rtol=1e-12)
+
+
+def test_demo_shape_c0():
+    """The pages' demo: S=1024, H=8, D=64, top_k=64, g=8 -> index shape (1024, 8, 64)."""
+    q, k = synthetic.make_prefill("C0")
+    c = synthetic.CONFIGS["C0"]
+    r = oracle.prefill(q, k, c["g"], c["top_k"], c["Kc"], oracle.REFINE)
+    assert r["out"].shape == (1024, 8, 64)
+    assert np.all(r["out"][0] == -1)
+    assert np.all((r["out"] >= 0).sum(-1)[1:] == np.minimum(64, np.arange(1, 1024))[:, None])
