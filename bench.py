@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of the PIVOT-Refine indexer at L=131072 on B200.
+
+One step = one PIVOT-Refine call (proxy build, tcgen05 prefix scan with fused
+filter, exact candidate select, per-member refine) over the long-context
+prefill workload: L=131072, H=16, d=128, g=16, top_k=2048, Kc=4096, bf16,
+seeded synthetic inputs (heavy-tailed keys, AR(1) queries).  The metric is
+indexed query-heads per second (L*H per step), aggregated over all GPUs; each
+GPU indexes its own independent layer (weak scaling, no collective on the
+data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  `--impl reference` times the CPU oracle
+(the plain fp64 restatement of the method) on a bounded sample of the same
+workload on the host cores.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "PIVOT-Refine indexed queries/s at L=131072; fraction of tensor/HBM roofline"
+UNIT = "query-heads/s"
+WORKLOAD = "C3"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sust=float(p["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+def workload_config(c):
+    return {"workload": f"{WORKLOAD} long-context prefill L={c['L']} H={c['H']} d={c['d']} g={c['g']} "
+                        f"top_k={c['top_k']} Kc={c['Kc']} PIVOT-Refine",
+            "generator": f"keys N(0,1) with {c['heavy_frac']*100:g}% positions x{c['heavy_scale']:g}; "
+                         f"queries AR(1) rho={c['rho']}; seed {c['seed']} (+rank)",
+            "l2": "inputs 1.07 GB and outputs 17.2 GB per step exceed the 126 MB L2; no flush needed",
+            "parallelism": "one independent layer per GPU (weak scaling), no collective"}
+
+
+def algorithmic(c):
+    """Method's own work per step, by kernel (flops or bytes)."""
+    L, H, d, g, k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
+    G = (L + g - 1) // g
+    i = np.arange(G, dtype=np.int64)
+    last = np.minimum(i * g + g, L) - 1
+    scan_flops = 2.0 * d * H * float(last.sum())
+    nC = np.minimum(Kc, last)
+    return {
+        "scan_filter": ("tensor", scan_flops),
+        # a select must at least read Kc (key, index) pairs and write Kc indices per row
+        "finalize": ("hbm", float(H * nC.sum() * (8 + 4))),
+        # output rows + candidate rows + member queries + every key once
+        "refine": ("hbm", float(L * H * k * 4 + H * nC.sum() * 4 + 2 * L * H * d * 2)),
+        "proxy": ("hbm", float(L * H * d * 2 + G * H * d * 2)),
+        "fallback": ("hbm", 0.0),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def cpu_baseline(c, q, k, budget_s=12.0, seed=0):
+    """The oracle, as it stands, on a seeded sample of (group, head) units."""
+    import oracle
+    L, H, g = c["L"], c["H"], c["g"]
+    G = (L + g - 1) // g
+    rng = np.random.default_rng(seed)
+    t0 = time.perf_counter()
+    n_q = 0
+    n_units = 0
+    while time.perf_counter() - t0 < budget_s:
+        gi = rng.integers(0, G, size=4).astype(np.int32)
+        hi = rng.integers(0, H, size=4).astype(np.int32)
+        oracle.prefill_units(q, k, g, c["top_k"], c["Kc"], oracle.REFINE, gi, hi)
+        n_q += int(sum(min(i * g + g, L) - i * g for i in gi))
+        n_units += 4
+    dt = time.perf_counter() - t0
+    return {"value": n_q / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n_units} random (group, head) units of {WORKLOAD} ({n_q} query-heads), "
+                      f"single-threaded C, {dt:.1f} s"}
+
+
+def run_reference(args, rank):
+    """CPU oracle timed per step on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    c = synthetic.CONFIGS[WORKLOAD]
+    q, k = synthetic.make_prefill(WORKLOAD)
+    L, H, g = c["L"], c["H"], c["g"]
+    G = (L + g - 1) // g
+    rng = np.random.default_rng(1234)
+    units = 48
+
+    def step():
+        gi = rng.integers(0, G, size=units).astype(np.int32)
+        hi = rng.integers(0, H, size=units).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.prefill_units(q, k, g, c["top_k"], c["Kc"], oracle.REFINE, gi, hi)
+        return time.perf_counter() - t0, int(sum(min(i * g + g, L) - i * g for i in gi))
+
+    for _ in range(args.warmup):
+        step()
+    tot_t, tot_q = 0.0, 0
+    for _ in range(args.steps):
+        t, n = step()
+        tot_t += t
+        tot_q += n
+    value = tot_q / tot_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(c),
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": 1,
+                             "sample": f"{units} random (group, head) units of {WORKLOAD} per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip the Reuse/dense comparison runs")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import query_group_top_b200 as qg
+    qg.load_library()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    c = dict(synthetic.CONFIGS[WORKLOAD])
+    L, H, d, g, top_k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
+    q_np, k_np = synthetic.gen_prefill(L, H, d, c["seed"] + rank, c["rho"], c["heavy_frac"], c["heavy_scale"])
+    q = torch.from_numpy(q_np.view(np.int16)).cuda().view(torch.bfloat16)
+    k = torch.from_numpy(k_np.view(np.int16)).cuda().view(torch.bfloat16)
+    out = torch.empty((L, H, top_k), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        qg.pivot_index(q, k, g, top_k, Kc, qg.REFINE, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    qg.sync_status()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    barrier()
+    torch.cuda.synchronize()
+    qg.trace_enable(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    qg.trace_enable(False)
+    trace = qg.trace_collect()
+    ms = e0.elapsed_time(e1) / args.steps
+    clk = clocks.stop()
+    flags = qg.sync_status()
+    ms_max = max_over_ranks(ms)
+    value = world * L * H / (ms_max / 1000.0)
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    alg = algorithmic(c)
+    kern = {name: {"ms_per_launch": tot / max(n, 1), "launches": n, "share": tot / (ms * args.steps)}
+            for name, (tot, n) in trace.items()}
+    dom = max(trace, key=lambda n: trace[n][0])
+    bound, work = alg.get(dom, ("hbm", 0.0))
+    t_launch = trace[dom][0] / trace[dom][1] / 1000.0
+    if bound == "tensor":
+        achieved = work / t_launch / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sust"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_sust"], "traffic": None, "kernel": dom,
+                "peak_note": f"{pk['src']} sustained bf16 dense (kernel timed inside a multi-ms step)"}
+    else:
+        achieved = work / t_launch / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "traffic": None, "kernel": dom,
+                "peak_note": f"{pk['src']} HBM copy bandwidth"}
+    scan_t = trace.get("scan_filter", (0, 1))
+    scan_tf = alg["scan_filter"][1] / (scan_t[0] / scan_t[1] / 1000.0) / 1e12 if scan_t[0] else None
+    gpu_launches = sum(n for _, n in trace.values())
+
+    # end to end through the public API: pinned host inputs -> device -> indexer -> host result
+    e2e = None
+    try:
+        q_h = torch.from_numpy(q_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+        k_h = torch.from_numpy(k_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+        try:
+            out_h = torch.empty((L, H, top_k), dtype=torch.int32, pin_memory=True)
+            pinned = True
+        except Exception:
+            out_h = torch.empty((L, H, top_k), dtype=torch.int32)
+            pinned = False
+        q_d = torch.empty_like(q)
+        k_d = torch.empty_like(k)
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            k_d.copy_(k_h, non_blocking=True)
+            qg.pivot_index(q_d, k_d, g, top_k, Kc, qg.REFINE, out=out)
+            out_h.copy_(out, non_blocking=pinned)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps)
+        e2e = {"value": world * L * H / (e2e_ms / 1000.0), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(q.numel() * 2 + k.numel() * 2),
+               "d2h_bytes_per_step": int(out.numel() * 4), "pinned_output": pinned}
+        del q_h, k_h, out_h, q_d, k_d
+    except Exception as ex:  # pragma: no cover - host memory limits
+        e2e = {"value": None, "unit": UNIT, "error": str(ex)[:200]}
+
+    extras = {}
+    if not args.no_extras:
+        def timed(fn, n):
+            fn()
+            torch.cuda.synchronize()
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(n):
+                fn()
+            t1.record(stream)
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1) / n
+        out_reuse = torch.empty_like(out)
+        reuse_ms = timed(lambda: qg.pivot_index(q, k, g, top_k, Kc, qg.REUSE, out=out_reuse), args.steps)
+        out_dense = torch.empty_like(out)
+        dense_ms = timed(lambda: qg.dense_index(q, k, top_k, out=out_dense), 1)
+        qg.sync_status()
+        # Recall@k against the dense indexer on a seeded 1% of rows
+        rng = np.random.default_rng(7)
+        rows = torch.from_numpy(rng.integers(1, L, size=L * H // 100)).cuda()
+        heads = torch.from_numpy(rng.integers(0, H, size=rows.numel())).cuda()
+        dn = out_dense[rows, heads].cpu().numpy()
+        rec = {}
+        for name, o in (("refine", out), ("reuse", out_reuse)):
+            pv = o[rows, heads].cpu().numpy()
+            hit = [np.intersect1d(a[a >= 0], b[b >= 0]).size / max(1, (b >= 0).sum()) for a, b in zip(pv, dn)]
+            rec[name] = float(np.mean(hit))
+        extras = {"refine_ms": ms, "reuse_ms": reuse_ms, "dense_ms": dense_ms,
+                  "speedup_refine_vs_dense": dense_ms / ms, "speedup_reuse_vs_dense": dense_ms / reuse_ms,
+                  "recall_at_k_vs_dense": rec, "recall_rows": int(rows.numel())}
+        del out_reuse, out_dense
+
+    if rank == 0:
+        import oracle
+        oracle.build()
+        cpu = cpu_baseline(c, q_np, k_np) if world == 1 else None
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(c),
+                "roofline": roof, "scan_tflops": scan_tf, "kernels": kern, "gpu_launches": gpu_launches,
+                "status_flags": flags, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "extras": extras}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

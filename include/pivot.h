@@ -1,0 +1,151 @@
+/*
+ * pivot.h -- C ABI of the B200 (sm_100a) PIVOT query-group indexer.
+ *
+ * The operation is the indexer of token-level sparse attention and its PIVOT
+ * replacement, as described in "PIVOT: Efficient Query-Group Indexing for
+ * Token-Level Sparse Attention" (arXiv 2607.24593): the pages "PIVOT explained
+ * -- from paper to working code in 10 minutes" (sections "The Problem", "How It
+ * Works", "Show Me The Code") and the paper's abstract.
+ *
+ * Common conventions (all entry points):
+ *  - Tensors are row-major, bfloat16 for q and k ("const void*" pointing to
+ *    2-byte bf16 values), int32 for indices.  All tensor pointers are DEVICE
+ *    pointers, 16-byte aligned.  The caller owns every buffer; the library keeps
+ *    no pointer after the call returns.
+ *  - Calls are asynchronous: work is enqueued on `stream` (a cudaStream_t passed
+ *    as void*; NULL = the legacy default stream) and the call returns without
+ *    synchronising.  Outputs are valid once the stream has reached that point.
+ *  - Scores are unscaled dot products q . k.  A query at position pos may only
+ *    select keys j < pos.  Ties in score go to the lower key index.  Every
+ *    output row holds its selected key indices in ascending order, followed by
+ *    -1 padding up to top_k.
+ *  - head_dim d must be 64 or 128; 1 <= top_k <= Kc <= 4096.
+ *  - Return value: PIVOT_OK, or an error code with a message available from
+ *    pivot_last_error() (thread-local).  Argument errors are detected on the
+ *    host before anything is enqueued.  Errors raised by the kernels (a bounded
+ *    wait that gave up, an over-long decode sequence) are reported by
+ *    pivot_sync_status().
+ *  - There is no CPU fallback: on a machine without an sm_100 device every
+ *    call returns PIVOT_ERR_UNSUPPORTED.
+ */
+#ifndef PIVOT_H_
+#define PIVOT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PIVOT_REFINE = 0, PIVOT_REUSE = 1 } pivot_mode_t;
+
+typedef enum {
+  PIVOT_OK = 0,
+  PIVOT_ERR_INVALID_ARG = 1,
+  PIVOT_ERR_UNSUPPORTED = 2,
+  PIVOT_ERR_CUDA = 3,
+  PIVOT_ERR_TIMEOUT = 4,
+  PIVOT_ERR_WORKSPACE = 5
+} pivot_status_t;
+
+/*
+ * PIVOT prefill indexer for one layer, all heads.
+ * Paper abstract and "How It Works": consecutive queries form groups of g
+ * (starting at 0, g, 2g, ...; the last may be partial); each group's proxy is
+ * the mean of its queries (fp64 sum, rounded to fp32 then bf16); one scan of
+ * the proxy over the group's causal prefix gives a candidate set.
+ *   mode = PIVOT_REFINE ("How It Works" per-query refine; listing pivot_refine):
+ *     scan keys j < last (the group's largest position), C = top-min(Kc,last);
+ *     member pos re-scores {j in C : j < pos} with its own query and keeps
+ *     top-min(top_k, that count).
+ *   mode = PIVOT_REUSE (listing pivot_reuse): scan keys j < s (group start);
+ *     every member gets the proxy's top-min(top_k, s).  Kc is not used.
+ * q, k:     bf16 [L][H][d].
+ * out_idx:  int32 [L][H][top_k].
+ * Temporary device memory is taken with cudaMallocAsync on `stream` and freed
+ * on it before return (see pivot_index_ws to supply it instead).
+ */
+int pivot_index(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
+                int32_t* out_idx, void* stream);
+
+/*
+ * Dense indexer -- the per-query scan that PIVOT replaces ("The Problem": every
+ * query scores every preceding token and keeps the top-k).
+ * out_idx[pos][h] = top-min(top_k, pos) of q[pos,h] . k[j,h] over j < pos.
+ * q, k bf16 [L][H][d]; out_idx int32 [L][H][top_k].
+ */
+int dense_index(const void* q, const void* k, int L, int H, int d, int top_k, int32_t* out_idx,
+                void* stream);
+
+/*
+ * PIVOT decode indexer for one multi-token-prediction step over a batch of
+ * sequences (paper abstract: in decode a group is the queries decoded together
+ * in one MTP step).  Sequence b holds n_b context keys plus the g keys of this
+ * step in the packed cache rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ * (n_b = cu_seqlens[b+1] - cu_seqlens[b] - g >= 0); its g queries sit at
+ * positions n_b .. n_b+g-1.  Refine scans j < n_b+g-1 and keeps top-min(Kc, .)
+ * candidates; Reuse scans j < n_b.  Indices are positions within the sequence.
+ * q:          bf16 [B][g][H][d].
+ * kcache:     bf16 [cu_seqlens[B]][H][d].
+ * cu_seqlens: int32 [B+1], device memory, non-decreasing.
+ * max_seqlen: an upper bound on cu_seqlens[b+1]-cu_seqlens[b] for every b; a
+ *             longer sequence is skipped on the device and reported by
+ *             pivot_sync_status() as PIVOT_ERR_INVALID_ARG.
+ * out_idx:    int32 [B][g][H][top_k].
+ */
+int pivot_decode_index(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
+                       int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx, void* stream);
+
+/*
+ * Workspace-taking variants: identical results; `workspace` (device, 256-byte
+ * aligned, owned by the caller, contents ignored) must hold at least the
+ * number of bytes reported by the matching *_workspace_size call, otherwise
+ * PIVOT_ERR_WORKSPACE is returned and nothing runs.  out_scores (nullable,
+ * float32, same shape as out_idx) receives the score that decided each output
+ * index -- the member query's score for Refine and dense, the proxy's score
+ * for Reuse -- and NaN in the padding.
+ */
+size_t pivot_workspace_size(int L, int H, int d, int g, int top_k, int Kc, int mode);
+int pivot_index_ws(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
+                   int32_t* out_idx, float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
+
+size_t dense_workspace_size(int L, int H, int d, int top_k);
+int dense_index_ws(const void* q, const void* k, int L, int H, int d, int top_k, int32_t* out_idx,
+                   float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
+
+size_t pivot_decode_workspace_size(int B, int H, int d, int g, int top_k, int Kc, int mode, int max_seqlen);
+int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
+                          int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
+                          float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's kernel status
+ * word.  Returns PIVOT_OK, PIVOT_ERR_TIMEOUT (a bounded wait inside a kernel
+ * gave up; that call's outputs are not valid), PIVOT_ERR_INVALID_ARG (a decode
+ * sequence exceeded max_seqlen) or PIVOT_ERR_CUDA.  *flags (nullable) receives
+ * the raw status bits; bit 4 means some rows took the exact fallback path
+ * (results remain exact).
+ */
+int pivot_sync_status(void* stream, int* flags);
+
+/*
+ * Launch trace (profiling aid, off by default; per calling thread).  While
+ * enabled, every kernel launch of this library is bracketed by two CUDA events
+ * recorded on the launch stream.  pivot_trace_collect() waits for the recorded
+ * events, aggregates them by kernel name and clears the trace: names receives a
+ * comma-separated list, ms[i] the summed device time of kernel i, count[i] its
+ * launches (up to max_items kernels).  Returns the number of kernels, or a
+ * negated error code.
+ */
+int pivot_trace_enable(int on);
+int pivot_trace_collect(char* names, size_t names_len, float* ms, int* count, int max_items);
+
+/* Message of the last error on the calling thread ("" if none). */
+const char* pivot_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PIVOT_H_ */

@@ -1,0 +1,211 @@
+"""B200 (sm_100a) PIVOT query-group indexer -- Python binding.
+
+Argument marshalling only: every step runs in the CUDA kernels of the in-tree
+``libpivot.so`` (C ABI declared in ``include/pivot.h``).  PyTorch supplies
+device memory and streams.  There is no CPU fallback: without the built
+library or an sm_100 device every call raises.
+
+    idx = pivot_index(q, k, g=16, top_k=2048, Kc=4096, mode=REFINE)   # [L, H, top_k] int32
+    idx = dense_index(q, k, top_k=2048)
+    idx = pivot_decode_index(q, kcache, cu_seqlens, g=2, top_k=2048, Kc=4096, max_seqlen=...)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["REFINE", "REUSE", "PivotError", "pivot_index", "dense_index", "pivot_decode_index",
+           "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED"]
+
+REFINE, REUSE = 0, 1
+FLAG_TIMEOUT, FLAG_BADLEN, FLAG_FALLBACK = 1, 2, 4
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libpivot.so")
+_lib = None
+
+# Every symbol declared in include/pivot.h.
+EXPORTED = (
+    "pivot_index", "dense_index", "pivot_decode_index",
+    "pivot_workspace_size", "pivot_index_ws", "dense_workspace_size", "dense_index_ws",
+    "pivot_decode_workspace_size", "pivot_decode_index_ws", "pivot_sync_status", "pivot_last_error",
+    "pivot_trace_enable", "pivot_trace_collect",
+)
+
+
+class PivotError(RuntimeError):
+    pass
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libpivot.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise PivotError(f"{_LIB_PATH} is missing: build it with `python -m query_group_top_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "pivot_index": ([P, P, I, I, I, I, I, I, I, P, P], I),
+        "dense_index": ([P, P, I, I, I, I, P, P], I),
+        "pivot_decode_index": ([P, P, P, I, I, I, I, I, I, I, I, P, P], I),
+        "pivot_workspace_size": ([I, I, I, I, I, I, I], Z),
+        "pivot_index_ws": ([P, P, I, I, I, I, I, I, I, P, P, P, Z, P], I),
+        "dense_workspace_size": ([I, I, I, I], Z),
+        "dense_index_ws": ([P, P, I, I, I, I, P, P, P, Z, P], I),
+        "pivot_decode_workspace_size": ([I, I, I, I, I, I, I, I], Z),
+        "pivot_decode_index_ws": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, Z, P], I),
+        "pivot_sync_status": ([P, ctypes.POINTER(I)], I),
+        "pivot_last_error": ([], ctypes.c_char_p),
+        "pivot_trace_enable": ([I], I),
+        "pivot_trace_collect": ([ctypes.c_char_p, Z, P, P, I], I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _err(lib, rc: int):
+    if rc != 0:
+        raise PivotError(f"pivot error {rc}: {lib.pivot_last_error().decode(errors='replace')}")
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _check_bf16(name, t, ndim):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise PivotError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise PivotError(f"{name} must be bfloat16 (got {t.dtype})")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise PivotError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+_ws = {}
+
+
+def _workspace(nbytes: int, device, stream_ptr: int) -> torch.Tensor:
+    """Per (device, stream) cached workspace, grown on demand."""
+    key = (device, stream_ptr)
+    t = _ws.get(key)
+    if t is None or t.numel() < nbytes:
+        _ws.pop(key, None)
+        t = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        _ws[key] = t
+    return t
+
+
+def _out(out, shape, dtype, device, name):
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    if tuple(out.shape) != tuple(shape) or out.dtype != dtype or not out.is_contiguous() or out.device != device:
+        raise PivotError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}")
+    return out
+
+
+def pivot_index(q, k, g, top_k, Kc, mode=REFINE, out=None, out_scores=None, stream=None):
+    """PIVOT prefill indexer: q, k bf16 [L, H, d] -> int32 [L, H, top_k] (ascending, -1 padded)."""
+    lib = load_library()
+    _check_bf16("q", q, 3)
+    _check_bf16("k", k, 3)
+    if q.shape != k.shape:
+        raise PivotError("q and k must have the same shape [L, H, d]")
+    L, H, d = q.shape
+    out = _out(out, (L, H, top_k), torch.int32, q.device, "out")
+    if out_scores is not None:
+        out_scores = _out(out_scores, (L, H, top_k), torch.float32, q.device, "out_scores")
+    sp = _stream_ptr(stream)
+    n = lib.pivot_workspace_size(L, H, d, g, top_k, Kc, mode)
+    ws = _workspace(n, q.device, sp)
+    rc = lib.pivot_index_ws(q.data_ptr(), k.data_ptr(), L, H, d, g, top_k, Kc, mode, out.data_ptr(),
+                            None if out_scores is None else out_scores.data_ptr(), ws.data_ptr(), ws.numel(), sp)
+    _err(lib, rc)
+    return out
+
+
+def dense_index(q, k, top_k, out=None, out_scores=None, stream=None):
+    """Dense per-query indexer: q, k bf16 [L, H, d] -> int32 [L, H, top_k]."""
+    lib = load_library()
+    _check_bf16("q", q, 3)
+    _check_bf16("k", k, 3)
+    if q.shape != k.shape:
+        raise PivotError("q and k must have the same shape [L, H, d]")
+    L, H, d = q.shape
+    out = _out(out, (L, H, top_k), torch.int32, q.device, "out")
+    if out_scores is not None:
+        out_scores = _out(out_scores, (L, H, top_k), torch.float32, q.device, "out_scores")
+    sp = _stream_ptr(stream)
+    n = lib.dense_workspace_size(L, H, d, top_k)
+    ws = _workspace(n, q.device, sp)
+    rc = lib.dense_index_ws(q.data_ptr(), k.data_ptr(), L, H, d, top_k, out.data_ptr(),
+                            None if out_scores is None else out_scores.data_ptr(), ws.data_ptr(), ws.numel(), sp)
+    _err(lib, rc)
+    return out
+
+
+def pivot_decode_index(q, kcache, cu_seqlens, g, top_k, Kc, mode=REFINE, max_seqlen=None, out=None,
+                       out_scores=None, stream=None):
+    """PIVOT decode indexer: q bf16 [B, g, H, d], kcache bf16 [rows, H, d], cu_seqlens int32 [B+1]
+    (device) -> int32 [B, g, H, top_k].  max_seqlen bounds every sequence's cache rows."""
+    lib = load_library()
+    _check_bf16("q", q, 4)
+    _check_bf16("kcache", kcache, 3)
+    B, gq, H, d = q.shape
+    if gq != g:
+        raise PivotError("q's second axis must equal g")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.numel() != B + 1:
+        raise PivotError("cu_seqlens must be an int32 CUDA tensor of B+1 offsets")
+    if max_seqlen is None:
+        raise PivotError("max_seqlen (an upper bound on cache rows per sequence) is required")
+    out = _out(out, (B, g, H, top_k), torch.int32, q.device, "out")
+    if out_scores is not None:
+        out_scores = _out(out_scores, (B, g, H, top_k), torch.float32, q.device, "out_scores")
+    sp = _stream_ptr(stream)
+    n = lib.pivot_decode_workspace_size(B, H, d, g, top_k, Kc, mode, int(max_seqlen))
+    ws = _workspace(n, q.device, sp)
+    rc = lib.pivot_decode_index_ws(q.data_ptr(), kcache.data_ptr(), cu_seqlens.data_ptr(), B, H, d, g, top_k, Kc,
+                                   mode, int(max_seqlen), out.data_ptr(),
+                                   None if out_scores is None else out_scores.data_ptr(), ws.data_ptr(),
+                                   ws.numel(), sp)
+    _err(lib, rc)
+    return out
+
+
+def trace_enable(on: bool = True) -> None:
+    """Turns the library's per-launch CUDA-event trace on or off (calling thread)."""
+    _err(load_library(), load_library().pivot_trace_enable(1 if on else 0))
+
+
+def trace_collect() -> dict:
+    """Waits for the traced launches and returns {kernel: (total_ms, launches)}; clears the trace."""
+    lib = load_library()
+    names = ctypes.create_string_buffer(4096)
+    ms = (ctypes.c_float * 64)()
+    cnt = (ctypes.c_int * 64)()
+    n = lib.pivot_trace_collect(names, 4096, ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), 64)
+    if n < 0:
+        _err(lib, -n)
+    keys = names.value.decode().split(",") if n > 0 else []
+    return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(keys)}
+
+
+def sync_status(stream=None) -> int:
+    """Synchronises the stream and returns the kernels' status bits; raises on a kernel error."""
+    lib = load_library()
+    flags = ctypes.c_int(0)
+    rc = lib.pivot_sync_status(_stream_ptr(stream), ctypes.byref(flags))
+    _err(lib, rc)
+    return flags.value

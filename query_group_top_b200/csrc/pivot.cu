@@ -1,0 +1,622 @@
+// Host side of the C ABI declared in include/pivot.h: argument checks,
+// workspace layout, TMA descriptors and the launch sequence of each call.
+//
+// Prefill (pivot_index / dense_index), per head pass:
+//   proxy_kernel        group means -> bf16 proxies          (skipped for dense)
+//   scan_filter_kernel  tcgen05 prefix scan + threshold filter -> spill lists
+//   finalize_kernel     exact top-K per row from the spill list
+//   fallback_kernel     exact recompute for rows the filter could not settle
+// then refine_kernel (Refine only): per-member re-score of the candidate set.
+// Decode (pivot_decode_index): proxy_kernel -> decode_scan_kernel ->
+// decode_select_kernel -> refine_kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/pivot.h"
+#include "finalize.cuh"
+#include "proxy_decode.cuh"
+#include "ptx.cuh"
+#include "refine.cuh"
+#include "scan.cuh"
+
+namespace {
+
+using namespace pivot;
+
+__device__ int g_status_word;  // per-device kernel status bits
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+// ---------------------------------------------------------------- launch trace
+// Optional: every kernel launch of the calling thread is bracketed by two CUDA
+// events on its stream; pivot_trace_collect() turns them into per-kernel times.
+struct TraceRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+thread_local bool g_trace_on = false;
+thread_local std::vector<TraceRec> g_trace;
+thread_local std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct TraceScope {
+  TraceRec rec{nullptr, nullptr, nullptr};
+  cudaStream_t st;
+  TraceScope(const char* name, cudaStream_t s) : st(s) {
+    if (!g_trace_on) return;
+    rec.name = name;
+    rec.a = pool_event();
+    rec.b = pool_event();
+    cudaEventRecord(rec.a, st);
+  }
+  ~TraceScope() {
+    if (!rec.name) return;
+    cudaEventRecord(rec.b, st);
+    g_trace.push_back(rec);
+  }
+};
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sms = 0;
+  int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(PIVOT_ERR_UNSUPPORTED, "no CUDA device available");
+  if (dev < 0 || dev >= kMaxDevices) return fail(PIVOT_ERR_UNSUPPORTED, "device index out of range");
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    d.supported = (major == 10 && minor == 0);
+    d.sms = sms;
+    if (d.supported) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess)
+        return fail(PIVOT_ERR_CUDA, "cudaGetSymbolAddress(status): %s", cudaGetErrorString(cudaGetLastError()));
+      d.status = static_cast<int*>(p);
+    }
+    d.ready = true;
+  }
+  if (!d.supported) return fail(PIVOT_ERR_UNSUPPORTED, "this library needs an sm_100 (B200) device");
+  *out = &d;
+  return PIVOT_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// View of a [rows][H][d] bf16 tensor starting at `base` (which may point at a
+// later head), covering `heads` heads; box = 64 channels x 1 head x box_rows
+// rows, 128-byte swizzle.
+int make_rows_map(CUtensorMap* m, const void* base, int rows, int heads, int H, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(PIVOT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PIVOT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return PIVOT_OK;
+}
+
+// ---------------------------------------------------------------- workspace layout
+constexpr size_t kAlign = 256;
+constexpr size_t kSpillBudget = size_t(8) << 30;  // spill bytes per head pass
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+  // sizes
+  int G, cap, S, K_sel, heads_per_pass, nfb;
+  // offsets
+  size_t off_proxy, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, total;
+};
+
+// Sample stride and spill capacity for a select of K_sel keys per row over
+// prefixes up to L keys.
+void filter_shape(int K_sel, int L, int* cap, int* S) {
+  const int BN = 256;
+  int c = std::max(2 * K_sel, 2 * BN);
+  int s = std::max(1, std::min(16, c / BN));
+  const int min_s = (L + BN * 255 - 1) / (BN * 255);  // at most 255 sampled tiles per row
+  s = std::max(s, min_s);
+  c = std::max(c, s * BN);
+  *cap = (c + 7) / 8 * 8;
+  *S = s;
+}
+
+Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool dense, int sms) {
+  Plan p{};
+  p.G = dense ? L : (L + g - 1) / g;
+  p.K_sel = (dense || mode == PIVOT_REUSE) ? top_k : Kc;
+  filter_shape(p.K_sel, L, &p.cap, &p.S);
+  const size_t per_head_spill = static_cast<size_t>(p.G) * p.cap * sizeof(uint2);
+  p.heads_per_pass = static_cast<int>(std::max<size_t>(1, std::min<size_t>(H, kSpillBudget / per_head_spill)));
+  p.nfb = 2 * std::max(1, sms);
+  const size_t rows_pass = static_cast<size_t>(p.heads_per_pass) * p.G;
+  size_t o = 0;
+  p.off_proxy = o;
+  o += dense ? 0 : up(static_cast<size_t>(p.G) * H * d * 2);
+  p.off_spill = o;
+  o += up(rows_pass * p.cap * sizeof(uint2));
+  p.off_cnt = o;
+  o += up(rows_pass * sizeof(int));
+  p.off_fb = o;
+  o += up(sizeof(int));
+  p.off_fblist = o;
+  o += up(rows_pass * sizeof(int));
+  p.off_fbscratch = o;
+  o += up(static_cast<size_t>(p.nfb) * L * sizeof(uint32_t));
+  p.off_cand = o;
+  o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(H) * p.G * Kc * sizeof(int32_t)) : 0;
+  p.total = o;
+  return p;
+}
+
+uint32_t tmem_cols_for(int Kc) {
+  const int need = 16 * ((Kc + 127) / 128);
+  uint32_t c = 32;
+  while (static_cast<int>(c) < need) c <<= 1;
+  return c;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(const void* q, const void* k, int H, int d, int top_k, int Kc, int mode, const void* out) {
+  if (!q || !k || !out) return fail(PIVOT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(out))
+    return fail(PIVOT_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (H < 1) return fail(PIVOT_ERR_INVALID_ARG, "H must be >= 1");
+  if (d != 64 && d != 128) return fail(PIVOT_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", d);
+  if (top_k < 1 || Kc < top_k || Kc > 4096)
+    return fail(PIVOT_ERR_INVALID_ARG, "need 1 <= top_k <= Kc <= 4096 (top_k=%d, Kc=%d)", top_k, Kc);
+  if (mode != PIVOT_REFINE && mode != PIVOT_REUSE) return fail(PIVOT_ERR_INVALID_ARG, "mode must be 0 or 1");
+  return PIVOT_OK;
+}
+
+#define CUDA_TRY(expr)                                                                       \
+  do {                                                                                       \
+    cudaError_t e_ = (expr);                                                                 \
+    if (e_ != cudaSuccess) return fail(PIVOT_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+template <int D>
+int launch_scan(const CUtensorMap& tmP, const CUtensorMap& tmK, const ScanParams& sp, int heads, cudaStream_t st) {
+  using C = ScanCfg<D>;
+  CUDA_TRY(cudaFuncSetAttribute(scan_filter_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  TraceScope tr("scan_filter", st);
+  scan_filter_kernel<D><<<heads * sp.tiles_per_head, C::THREADS, C::SMEM, st>>>(tmP, tmK, sp);
+  CUDA_TRY(cudaGetLastError());
+  return PIVOT_OK;
+}
+
+template <int D>
+int launch_refine(const RefineParams& rp, int units, cudaStream_t st) {
+  const int smem = RefineCfg<D>::smem_bytes(rp.Kc);
+  CUDA_TRY(cudaFuncSetAttribute(refine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  TraceScope tr("refine", st);
+  refine_kernel<D><<<units, RefineCfg<D>::NT, smem, st>>>(rp);
+  CUDA_TRY(cudaGetLastError());
+  return PIVOT_OK;
+}
+
+// Shared prefill driver (PIVOT Refine/Reuse, and dense when `dense`).
+int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode, bool dense,
+                int32_t* out, float* out_scores, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (L < 1) return fail(PIVOT_ERR_INVALID_ARG, "L must be >= 1");
+  if (!dense && g < 1) return fail(PIVOT_ERR_INVALID_ARG, "g must be >= 1");
+  if (static_cast<long long>(L) * H * d >= (1ll << 40)) return fail(PIVOT_ERR_INVALID_ARG, "tensor too large");
+  if (L >= (1 << 30)) return fail(PIVOT_ERR_INVALID_ARG, "L too large");
+  if (out_scores && !aligned16(out_scores)) return fail(PIVOT_ERR_INVALID_ARG, "out_scores must be 16-byte aligned");
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  const Plan pl = plan_prefill(L, H, d, dense ? 1 : g, top_k, Kc, mode, dense, dev->sms);
+  if (!ws || ws_bytes < pl.total)
+    return fail(PIVOT_ERR_WORKSPACE, "workspace too small: need %zu bytes, got %zu", pl.total, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
+    return fail(PIVOT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const uint16_t* P = dense ? static_cast<const uint16_t*>(q) : reinterpret_cast<const uint16_t*>(w + pl.off_proxy);
+  const int gg = dense ? 1 : g;
+  const bool refine = !dense && mode == PIVOT_REFINE;
+
+  if (!dense) {
+    const long long n = static_cast<long long>(pl.G) * H * (d / 8);
+    TraceScope tr("proxy", st);
+    proxy_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        static_cast<const uint16_t*>(q), reinterpret_cast<uint16_t*>(w + pl.off_proxy), pl.G, H, d, gg, L, 0);
+    CUDA_TRY(cudaGetLastError());
+  }
+
+  for (int h0 = 0; h0 < H; h0 += pl.heads_per_pass) {
+    const int nh = std::min(pl.heads_per_pass, H - h0);
+    // TMA views start at head h0 so that the kernels' head index is pass-local.
+    const uint16_t* Ph = P + static_cast<size_t>(h0) * d;
+    const uint16_t* Kh = static_cast<const uint16_t*>(k) + static_cast<size_t>(h0) * d;
+    CUtensorMap tmP, tmK;
+    if (int rc = make_rows_map(&tmP, Ph, pl.G, nh, H, d, 128)) return rc;
+    if (int rc = make_rows_map(&tmK, Kh, L, nh, H, d, 256)) return rc;
+    ScanParams sp{};
+    sp.G = pl.G;
+    sp.L = L;
+    sp.H = H;
+    sp.g = gg;
+    sp.bound_kind = refine ? 0 : 1;
+    sp.K_sel = pl.K_sel;
+    sp.cap = pl.cap;
+    sp.S = pl.S;
+    sp.tiles_per_head = (pl.G + 127) / 128;
+    sp.spill = reinterpret_cast<uint2*>(w + pl.off_spill);
+    sp.cnt = reinterpret_cast<int*>(w + pl.off_cnt);
+    sp.status = dev->status;
+    int rc = (d == 128) ? launch_scan<128>(tmP, tmK, sp, nh, st) : launch_scan<64>(tmP, tmK, sp, nh, st);
+    if (rc) return rc;
+
+    FinalizeParams fp{};
+    fp.G = pl.G;
+    fp.L = L;
+    fp.H = H;
+    fp.g = gg;
+    fp.bound_kind = sp.bound_kind;
+    fp.K_sel = pl.K_sel;
+    fp.cap = pl.cap;
+    fp.width = refine ? Kc : top_k;
+    fp.broadcast = refine ? 0 : 1;
+    fp.spill = sp.spill;
+    fp.cnt = sp.cnt;
+    // Head-local row ids: shift the output bases by h0 heads.
+    fp.cand = refine ? reinterpret_cast<int32_t*>(w + pl.off_cand) + static_cast<size_t>(h0) * pl.G * Kc : nullptr;
+    fp.out = refine ? nullptr : out + static_cast<size_t>(h0) * top_k;
+    fp.out_scores = (refine || !out_scores) ? nullptr : out_scores + static_cast<size_t>(h0) * top_k;
+    fp.fb_list = reinterpret_cast<int*>(w + pl.off_fblist);
+    fp.fb_count = reinterpret_cast<int*>(w + pl.off_fb);
+    fp.status = dev->status;
+    fp.proxy = Ph;
+    fp.keys = Kh;
+    fp.d = d;
+    fp.fb_scratch = reinterpret_cast<uint32_t*>(w + pl.off_fbscratch);
+    CUDA_TRY(cudaMemsetAsync(fp.fb_count, 0, sizeof(int), st));
+    const int fin_smem = pl.cap * 8 + pl.K_sel * 8;
+    CUDA_TRY(cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fin_smem));
+    {
+      TraceScope tr("finalize", st);
+      finalize_kernel<<<static_cast<unsigned>(nh * pl.G), kFinNT, fin_smem, st>>>(fp);
+    }
+    CUDA_TRY(cudaGetLastError());
+    const int fb_smem = pl.K_sel * 8;
+    CUDA_TRY(cudaFuncSetAttribute(fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fb_smem));
+    {
+      TraceScope tr("fallback", st);
+      fallback_kernel<<<pl.nfb, kFbNT, fb_smem, st>>>(fp);
+    }
+    CUDA_TRY(cudaGetLastError());
+  }
+
+  if (refine) {
+    RefineParams rp{};
+    rp.q = static_cast<const uint16_t*>(q);
+    rp.keys = static_cast<const uint16_t*>(k);
+    rp.cand = reinterpret_cast<const int32_t*>(w + pl.off_cand);
+    rp.out = out;
+    rp.out_scores = out_scores;
+    rp.cu = nullptr;
+    rp.G = pl.G;
+    rp.L = L;
+    rp.H = H;
+    rp.g = g;
+    rp.top_k = top_k;
+    rp.Kc = Kc;
+    rp.d = d;
+    rp.tmem_cols = tmem_cols_for(Kc);
+    rp.status = dev->status;
+    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, st) : launch_refine<64>(rp, H * pl.G, st);
+    if (rc) return rc;
+  }
+  return PIVOT_OK;
+}
+
+size_t decode_ws_size(int B, int H, int d, int Kc, int mode, int max_seqlen) {
+  size_t o = up(static_cast<size_t>(B) * H * d * 2);                        // proxies
+  o += up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t));       // order keys
+  if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(H) * B * Kc * sizeof(int32_t));
+  return o;
+}
+
+int check_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, int d, int g, int top_k, int Kc,
+                 int mode, int max_seqlen, const void* out, const void* out_scores) {
+  if (int rc = check_common(q, kc, H, d, top_k, Kc, mode, out)) return rc;
+  if (!cu) return fail(PIVOT_ERR_INVALID_ARG, "null cu_seqlens");
+  if (B < 1 || g < 1 || max_seqlen < g) return fail(PIVOT_ERR_INVALID_ARG, "need B >= 1, g >= 1, max_seqlen >= g");
+  if (max_seqlen >= (1 << 30)) return fail(PIVOT_ERR_INVALID_ARG, "max_seqlen too large");
+  if (out_scores && !aligned16(out_scores)) return fail(PIVOT_ERR_INVALID_ARG, "out_scores must be 16-byte aligned");
+  return PIVOT_OK;
+}
+
+int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, int d, int g, int top_k, int Kc,
+               int mode, int max_seqlen, int32_t* out, float* out_scores, void* ws, size_t ws_bytes,
+               cudaStream_t st) {
+  if (int rc = check_decode(q, kc, cu, B, H, d, g, top_k, Kc, mode, max_seqlen, out, out_scores)) return rc;
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  const size_t need = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  if (!ws || ws_bytes < need) return fail(PIVOT_ERR_WORKSPACE, "workspace too small: need %zu bytes", need);
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
+    return fail(PIVOT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* P = reinterpret_cast<uint16_t*>(w);
+  uint32_t* scores = reinterpret_cast<uint32_t*>(w + up(static_cast<size_t>(B) * H * d * 2));
+  int32_t* cand = reinterpret_cast<int32_t*>(w + up(static_cast<size_t>(B) * H * d * 2) +
+                                             up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t)));
+  const long long n = static_cast<long long>(B) * H * (d / 8);
+  {
+    TraceScope tr("proxy", st);
+    proxy_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(static_cast<const uint16_t*>(q), P, B, H,
+                                                                          d, g, 0, 1);
+  }
+  CUDA_TRY(cudaGetLastError());
+  DecodeParams dp{};
+  dp.kcache = static_cast<const uint16_t*>(kc);
+  dp.P = P;
+  dp.cu = cu;
+  dp.scores = scores;
+  dp.cand = mode == PIVOT_REFINE ? cand : nullptr;
+  dp.out = out;
+  dp.out_scores = mode == PIVOT_REUSE ? out_scores : nullptr;
+  dp.B = B;
+  dp.H = H;
+  dp.d = d;
+  dp.g = g;
+  dp.mode = mode;
+  dp.K_sel = mode == PIVOT_REFINE ? Kc : top_k;
+  dp.width = mode == PIVOT_REFINE ? Kc : top_k;
+  dp.max_seqlen = max_seqlen;
+  dp.status = dev->status;
+  dim3 grid((max_seqlen + kDecChunk - 1) / kDecChunk, H, B);
+  {
+  TraceScope tr("decode_scan", st);
+  if (d == 128)
+    decode_scan_kernel<128><<<grid, kDecNT, 0, st>>>(dp);
+  else
+    decode_scan_kernel<64><<<grid, kDecNT, 0, st>>>(dp);
+  }
+  CUDA_TRY(cudaGetLastError());
+  const int sel_smem = dp.K_sel * 8;
+  CUDA_TRY(cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem));
+  {
+    TraceScope tr("decode_select", st);
+    decode_select_kernel<<<B * H, kDecSelNT, sel_smem, st>>>(dp);
+  }
+  CUDA_TRY(cudaGetLastError());
+  if (mode == PIVOT_REFINE) {
+    RefineParams rp{};
+    rp.q = static_cast<const uint16_t*>(q);
+    rp.keys = static_cast<const uint16_t*>(kc);
+    rp.cand = cand;
+    rp.out = out;
+    rp.out_scores = out_scores;
+    rp.cu = cu;
+    rp.G = B;
+    rp.L = 0;
+    rp.H = H;
+    rp.g = g;
+    rp.top_k = top_k;
+    rp.Kc = Kc;
+    rp.d = d;
+    rp.tmem_cols = tmem_cols_for(Kc);
+    rp.status = dev->status;
+    int rc = (d == 128) ? launch_refine<128>(rp, H * B, st) : launch_refine<64>(rp, H * B, st);
+    if (rc) return rc;
+  }
+  return PIVOT_OK;
+}
+
+// Runs `body(ws, bytes)` with a stream-ordered temporary allocation.
+template <class F>
+int with_temp_workspace(size_t bytes, cudaStream_t st, F body) {
+  void* ws = nullptr;
+  CUDA_TRY(cudaMallocAsync(&ws, std::max<size_t>(bytes, kAlign), st));
+  const int rc = body(ws, bytes);
+  const cudaError_t e = cudaFreeAsync(ws, st);
+  if (rc) return rc;
+  if (e != cudaSuccess) return fail(PIVOT_ERR_CUDA, "cudaFreeAsync: %s", cudaGetErrorString(e));
+  return PIVOT_OK;
+}
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pivot_workspace_size(int L, int H, int d, int g, int top_k, int Kc, int mode) {
+  if (L < 1 || H < 1 || g < 1 || top_k < 1 || Kc < top_k) return 0;
+  return plan_prefill(L, H, d, g, top_k, Kc, mode, false, device_sms()).total;
+}
+
+size_t dense_workspace_size(int L, int H, int d, int top_k) {
+  if (L < 1 || H < 1 || top_k < 1) return 0;
+  return plan_prefill(L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, device_sms()).total;
+}
+
+size_t pivot_decode_workspace_size(int B, int H, int d, int g, int top_k, int Kc, int mode, int max_seqlen) {
+  (void)g;
+  (void)top_k;
+  if (B < 1 || H < 1 || max_seqlen < 1) return 0;
+  return decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+}
+
+int pivot_index_ws(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
+                   int32_t* out_idx, float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_common(q, k, H, d, top_k, Kc, mode, out_idx)) return rc;
+  return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, out_scores, workspace, workspace_bytes,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int pivot_index(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
+                int32_t* out_idx, void* stream) {
+  if (int rc = check_common(q, k, H, d, top_k, Kc, mode, out_idx)) return rc;
+  if (L < 1 || g < 1) return fail(PIVOT_ERR_INVALID_ARG, "need L >= 1 and g >= 1");
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = plan_prefill(L, H, d, g, top_k, Kc, mode, false, dev->sms).total;
+  return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
+    return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, nullptr, ws, n, st);
+  });
+}
+
+int dense_index_ws(const void* q, const void* k, int L, int H, int d, int top_k, int32_t* out_idx,
+                   float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_common(q, k, H, d, top_k, top_k, PIVOT_REUSE, out_idx)) return rc;
+  return run_prefill(q, k, L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, out_idx, out_scores, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int dense_index(const void* q, const void* k, int L, int H, int d, int top_k, int32_t* out_idx, void* stream) {
+  if (int rc = check_common(q, k, H, d, top_k, top_k, PIVOT_REUSE, out_idx)) return rc;
+  if (L < 1) return fail(PIVOT_ERR_INVALID_ARG, "L must be >= 1");
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = plan_prefill(L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, dev->sms).total;
+  return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
+    return run_prefill(q, k, L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, out_idx, nullptr, ws, n, st);
+  });
+}
+
+int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
+                          int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
+                          float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
+  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, workspace,
+                    workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pivot_decode_index(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d, int g,
+                       int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx, void* stream) {
+  if (int rc = check_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr))
+    return rc;
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
+    return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr, ws, n, st);
+  });
+}
+
+int pivot_sync_status(void* stream, int* flags) {
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  CUDA_TRY(cudaMemcpy(&v, dev->status, sizeof v, cudaMemcpyDeviceToHost));
+  const int zero = 0;
+  CUDA_TRY(cudaMemcpy(dev->status, &zero, sizeof zero, cudaMemcpyHostToDevice));
+  if (flags) *flags = v;
+  if (v & kStTimeout) return fail(PIVOT_ERR_TIMEOUT, "a kernel wait timed out; outputs of that call are invalid");
+  if (v & kStBadLen) return fail(PIVOT_ERR_INVALID_ARG, "a decode sequence was longer than max_seqlen");
+  return PIVOT_OK;
+}
+
+const char* pivot_last_error(void) { return g_err; }
+
+int pivot_trace_enable(int on) {
+  g_trace_on = on != 0;
+  return PIVOT_OK;
+}
+
+int pivot_trace_collect(char* names, size_t names_len, float* ms, int* count, int max_items) {
+  // Aggregate by kernel name: ms[i] = total time, count[i] = launches.
+  std::vector<const char*> keys;
+  std::vector<double> tot;
+  std::vector<int> cnt;
+  int rc = PIVOT_OK;
+  for (TraceRec& r : g_trace) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      rc = fail(PIVOT_ERR_CUDA, "trace event query failed");
+    size_t i = 0;
+    while (i < keys.size() && strcmp(keys[i], r.name) != 0) ++i;
+    if (i == keys.size()) {
+      keys.push_back(r.name);
+      tot.push_back(0.0);
+      cnt.push_back(0);
+    }
+    tot[i] += t;
+    cnt[i] += 1;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_trace.clear();
+  size_t off = 0;
+  if (names && names_len) names[0] = 0;
+  const int n = static_cast<int>(std::min<size_t>(keys.size(), max_items > 0 ? max_items : 0));
+  for (int i = 0; i < n; ++i) {
+    if (ms) ms[i] = static_cast<float>(tot[i]);
+    if (count) count[i] = cnt[i];
+    if (names) {
+      const int w = snprintf(names + off, off < names_len ? names_len - off : 0, "%s%s", i ? "," : "", keys[i]);
+      off += w > 0 ? static_cast<size_t>(w) : 0;
+    }
+  }
+  return rc == PIVOT_OK ? n : -rc;
+}
+
+}  // extern "C"

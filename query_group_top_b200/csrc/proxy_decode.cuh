@@ -1,0 +1,175 @@
+// Proxy build (prefill and decode) and the decode-side scan and select.
+//
+// Proxy: "PIVOT explained", "How It Works": proxy_q = mean(group); the mean is
+// accumulated in fp64 in member order, divided by the member count, rounded
+// to fp32 and then to bf16 (the scan's tensor-core operand).  A partial last
+// group averages over its actual members.
+//
+// Decode (paper abstract: in decode a group is "the queries decoded together
+// in one multi-token prediction step"): one group per sequence, members at
+// positions n_b .. n_b+g-1 of a packed key cache.  With a single proxy row per
+// (sequence, head) the scan is a matrix-vector product bound by HBM: each warp
+// streams 16-byte slices of consecutive key rows, reduces each row's dot
+// product with shuffles and writes one 32-bit order key per key (4 bytes per
+// 256 key bytes read).  An exact block select then keeps the top-K per
+// (sequence, head).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace pivot {
+
+// P[u][h][:] for units u < G.  Prefill: members are positions u*g .. min(u*g+g, L)-1
+// of q [L][H][d].  Decode (decode != 0): members are rows u*g .. u*g+g-1 of q [B*g][H][d].
+__global__ void proxy_kernel(const uint16_t* __restrict__ q, uint16_t* __restrict__ P, int G, int H, int d,
+                             int g, int L, int decode) {
+  const long long total = static_cast<long long>(G) * H * (d / 8);
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  const int c8 = static_cast<int>(t % (d / 8));
+  const long long uh = t / (d / 8);
+  const int h = static_cast<int>(uh % H);
+  const int u = static_cast<int>(uh / H);
+  const long long row0 = static_cast<long long>(u) * g;
+  const int n = decode ? g : min(u * g + g, L) - u * g;
+  double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int m = 0; m < n; ++m) {
+    const uint4 v = *reinterpret_cast<const uint4*>(q + ((row0 + m) * H + h) * d + c8 * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[2 * k] += static_cast<double>(__uint_as_float(w[k] << 16));
+      acc[2 * k + 1] += static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u));
+    }
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float lo = __double2float_rn(__ddiv_rn(acc[2 * k], static_cast<double>(n)));
+    const float hi = __double2float_rn(__ddiv_rn(acc[2 * k + 1], static_cast<double>(n)));
+    const uint32_t blo = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t bhi = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    o[k] = blo | (bhi << 16);
+  }
+  *reinterpret_cast<uint4*>(P + (static_cast<long long>(u) * H + h) * d + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+struct DecodeParams {
+  const uint16_t* kcache;   // [rows][H][d]
+  const uint16_t* P;        // [B][H][d] proxies
+  const int32_t* cu;        // [B+1]
+  uint32_t* scores;         // [H*B][max_seqlen] order keys
+  int32_t* cand;            // [H][B][width] (Refine)
+  int32_t* out;             // [B][g][H][width] (Reuse)
+  float* out_scores;        // [B][g][H][width] or null (Reuse)
+  int B, H, d, g;
+  int mode;                 // 0 Refine (scan j < n_b+g-1, keep Kc), 1 Reuse (scan j < n_b, keep top_k)
+  int K_sel, width, max_seqlen;
+  int* status;
+};
+
+constexpr int kDecChunk = 2048;   // keys per scan CTA
+constexpr int kDecNT = 256;
+
+__device__ __forceinline__ bool decode_unit(const DecodeParams& p, int b, int& n_b, int& bound) {
+  const int len = p.cu[b + 1] - p.cu[b];
+  n_b = len - p.g;
+  bound = p.mode == 0 ? n_b + p.g - 1 : n_b;
+  return len <= p.max_seqlen && n_b >= 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecNT) decode_scan_kernel(DecodeParams p) {
+  constexpr int LPK = D / 8;          // lanes per key row (16 bytes each)
+  constexpr int KPW = 32 / LPK;       // key rows per warp step
+  constexpr int NW = kDecNT / 32;
+  const int b = blockIdx.z, h = blockIdx.y;
+  int n_b, bound;
+  if (!decode_unit(p, b, n_b, bound)) {
+    if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) atomicOr(p.status, kStBadLen);
+    return;
+  }
+  const int j_begin = blockIdx.x * kDecChunk;
+  if (j_begin >= bound) return;
+  const int j_end = min(bound, j_begin + kDecChunk);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / LPK, part = lane % LPK;
+  float pf[8];
+  {
+    const uint4 v = *reinterpret_cast<const uint4*>(p.P + (static_cast<long long>(b) * p.H + h) * D + part * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      pf[2 * k] = __uint_as_float(w[k] << 16);
+      pf[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+  const uint16_t* kb = p.kcache + (static_cast<long long>(p.cu[b]) * p.H + h) * D + part * 8;
+  const long long kstride = static_cast<long long>(p.H) * D;
+  uint32_t* srow = p.scores + (static_cast<long long>(h) * p.B + b) * p.max_seqlen;
+  constexpr int UNROLL = 4;
+  for (int base = j_begin + warp * KPW; base < j_end; base += NW * KPW * UNROLL) {
+    uint4 kv[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int j = base + u * NW * KPW + sub;
+      kv[u] = (j < j_end) ? __ldg(reinterpret_cast<const uint4*>(kb + j * kstride)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const uint32_t w[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc = fmaf(pf[2 * k], __uint_as_float(w[k] << 16), acc);
+        acc = fmaf(pf[2 * k + 1], __uint_as_float(w[k] & 0xFFFF0000u), acc);
+      }
+#pragma unroll
+      for (int o = LPK / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      const int j = base + u * NW * KPW + sub;
+      if (part == 0 && j < j_end) srow[j] = score_key(acc);
+    }
+  }
+}
+
+constexpr int kDecSelNT = 1024;
+
+// Exact top-K per (sequence, head) over the materialised order keys.
+__global__ void __launch_bounds__(kDecSelNT) decode_select_kernel(DecodeParams p) {
+  __shared__ SelectSmem<kDecSelNT> sm;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  int32_t* sel = reinterpret_cast<int32_t*>(smem_raw);
+  uint32_t* selk = reinterpret_cast<uint32_t*>(sel + p.K_sel);
+  const int h = blockIdx.x / p.B, b = blockIdx.x % p.B;
+  int n_b, bound;
+  if (!decode_unit(p, b, n_b, bound)) return;
+  const int K = min(p.K_sel, bound);
+  const uint32_t* srow = p.scores + (static_cast<long long>(h) * p.B + b) * p.max_seqlen;
+  block_select_emit<kDecSelNT>(
+      bound, K, [&](int e) { return srow[e]; },
+      [&](int slot, int e) {
+        sel[slot] = e;
+        selk[slot] = srow[e];
+      },
+      sm);
+  __syncthreads();
+  if (p.mode == 0) {
+    int32_t* dst = p.cand + (static_cast<long long>(h) * p.B + b) * p.width;
+    for (int t = threadIdx.x; t < p.width; t += kDecSelNT) dst[t] = t < K ? sel[t] : -1;
+  } else {
+    for (int m = 0; m < p.g; ++m) {
+      int32_t* dst = p.out + ((static_cast<long long>(b) * p.g + m) * p.H + h) * p.width;
+      for (int t = threadIdx.x; t < p.width; t += kDecSelNT) dst[t] = t < K ? sel[t] : -1;
+      if (p.out_scores) {
+        float* ds = p.out_scores + ((static_cast<long long>(b) * p.g + m) * p.H + h) * p.width;
+        for (int t = threadIdx.x; t < p.width; t += kDecSelNT)
+          ds[t] = t < K ? key_score(selk[t]) : __int_as_float(0x7fc00000);
+      }
+    }
+  }
+}
+
+}  // namespace pivot

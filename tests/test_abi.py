@@ -1,0 +1,66 @@
+"""The C ABI library loads and exports every entry point of include/pivot.h;
+host-side argument checks answer before any device work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import query_group_top_b200 as qg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pivot.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_]+)\s*\(", text)) - {"if", "sizeof"})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from query_group_top_b200 import build
+    build.build()
+    return qg.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert set(names) == set(qg.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_workspace_sizes_are_host_arithmetic(lib):
+    a = lib.pivot_workspace_size(131072, 16, 128, 16, 2048, 4096, qg.REFINE)
+    b = lib.pivot_workspace_size(131072, 16, 128, 16, 2048, 4096, qg.REUSE)
+    c = lib.dense_workspace_size(8192, 16, 128, 256)
+    d = lib.pivot_decode_workspace_size(64, 16, 128, 2, 2048, 4096, qg.REFINE, 131074)
+    assert a > b > 0 and c > 0 and d > 0
+    # the Refine candidate set alone: H * G * Kc int32
+    assert a - b >= 16 * 8192 * 4096 * 4
+    assert lib.pivot_workspace_size(0, 16, 128, 16, 2048, 4096, 0) == 0
+
+
+def test_argument_errors_before_device_work(lib):
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16
+    rc = lib.pivot_index(None, p, 16, 1, 64, 4, 2, 4, 0, p, None)
+    assert rc == 1 and b"null" in lib.pivot_last_error()
+    assert lib.pivot_index(p, p, 16, 1, 96, 4, 2, 4, 0, p, None) == 2          # d not 64/128
+    assert lib.pivot_index(p, p, 16, 1, 64, 4, 5, 4, 0, p, None) == 1          # top_k > Kc
+    assert lib.pivot_index(p, p, 16, 1, 64, 4, 2, 8192, 0, p, None) == 1       # Kc > 4096
+    assert lib.pivot_index(p, p, 16, 1, 64, 4, 2, 4, 7, p, None) == 1          # bad mode
+    assert lib.pivot_index(p + 2, p, 16, 1, 64, 4, 2, 4, 0, p, None) == 1      # misaligned
+    assert lib.dense_index(p, p, 16, 1, 64, 0, p, None) == 1
+    assert lib.pivot_decode_index(p, p, None, 1, 1, 64, 2, 2, 4, 0, 16, p, None) == 1
+
+
+def test_no_device_means_unsupported(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16
+    assert lib.pivot_index(p, p, 16, 1, 64, 4, 2, 4, 0, p, None) == 2
+    assert b"sm_100" in lib.pivot_last_error() or b"device" in lib.pivot_last_error()

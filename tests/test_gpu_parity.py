@@ -1,0 +1,217 @@
+"""GPU path vs the CPU oracle, element by element, through the C ABI.
+
+Small shapes are checked in full (several 128-row tiles, ragged tails, partial
+groups, d = 64 and 128, g up to 24); the workload sizes are checked on a
+seeded sample of (group, head) units that the oracle computes one by one, plus
+properties that hold on every row (ascending, unique, causal, row sizes).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import query_group_top_b200 as qg
+import synthetic
+from tests.parity import assert_parity, compare, valid_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def run_prefill(q, k, g, top_k, Kc, mode, dense=False):
+    qd, kd = to_dev(q), to_dev(k)
+    L, H, _ = q.shape
+    sc = torch.empty((L, H, top_k), dtype=torch.float32, device="cuda")
+    if dense:
+        out = qg.dense_index(qd, kd, top_k, out_scores=sc)
+    else:
+        out = qg.pivot_index(qd, kd, g, top_k, Kc, mode, out_scores=sc)
+    flags = qg.sync_status()
+    return out.cpu().numpy(), sc.cpu().numpy(), flags
+
+
+def check_full(q, k, g, top_k, Kc, mode, dense=False):
+    got, gs, flags = run_prefill(q, k, g, top_k, Kc, mode, dense)
+    L, H, _ = q.shape
+    pos = np.broadcast_to(np.arange(L)[:, None], (L, H))
+    if dense:
+        ref = oracle.dense(q, k, top_k)
+        cedge = None
+    else:
+        ref = oracle.prefill(q, k, g, top_k, Kc, mode)
+        cedge = ref["cand_edge"][np.arange(L) // g] if mode == oracle.REFINE else None
+    res = compare(got, ref["out"], ref["edge"], pos, cedge, gs, ref["score"])
+    assert_parity(res, f"L={L} H={H} d={q.shape[2]} g={g} k={top_k} Kc={Kc} mode={mode} dense={dense}")
+    return res, flags
+
+
+@pytest.mark.parametrize("mode", ["refine", "reuse", "dense"])
+def test_c0_full(mode):
+    c = synthetic.CONFIGS["C0"]
+    q, k = synthetic.make_prefill("C0")
+    m = oracle.REFINE if mode == "refine" else oracle.REUSE
+    res, _ = check_full(q, k, c["g"], c["top_k"], c["Kc"], m, dense=(mode == "dense"))
+    assert res["exact"] + res["exempt"] == 1024 * 8
+
+
+SMALL = [
+    # L, H, d, g, top_k, Kc
+    (1, 1, 64, 1, 1, 1),
+    (2, 1, 128, 2, 1, 2),
+    (5, 2, 64, 3, 4, 9),
+    (64, 1, 128, 8, 8, 16),
+    (129, 2, 64, 5, 10, 20),
+    (300, 3, 128, 16, 24, 48),
+    (511, 1, 64, 17, 7, 33),
+    (1000, 2, 128, 8, 37, 80),
+    (1500, 1, 64, 24, 64, 128),
+    (2049, 2, 128, 2, 100, 300),
+    (700, 1, 128, 1, 50, 50),
+    (3000, 1, 64, 8, 300, 600),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_small_shapes_all_modes(shape):
+    L, H, d, g, top_k, Kc = shape
+    q, k = synthetic.gen_prefill(L, H, d, seed=L + 7 * g, rho=0.9)
+    check_full(q, k, g, top_k, Kc, oracle.REFINE)
+    check_full(q, k, g, top_k, Kc, oracle.REUSE)
+    check_full(q, k, g, top_k, Kc, oracle.REUSE, dense=True)
+
+
+def test_exact_ties_and_fallback_rows():
+    """Constant keys: every score of a row ties, the lowest indices win; the
+    sampled threshold cannot separate them, so long rows go to the exact
+    fallback path (flag bit 4) and must still be exact."""
+    L, H, d, top_k = 3000, 2, 64, 8
+    rng = np.random.default_rng(5)
+    q = synthetic.bf16_from_f32(rng.standard_normal((L, H, d)).astype(np.float32))
+    k = synthetic.bf16_from_f32(np.ones((L, H, d), np.float32))
+    res, flags = check_full(q, k, 1, top_k, top_k, oracle.REUSE, dense=True)
+    assert flags & qg.FLAG_FALLBACK
+    assert res["exempt"] == 0
+    res, flags = check_full(q, k, 4, top_k, 2 * top_k, oracle.REFINE)
+    assert res["exempt"] == 0
+
+
+def test_g1_pivot_equals_dense_on_gpu():
+    """g = 1: the proxy is the query itself, so Reuse runs the dense computation
+    (bit-identical) and Refine must agree with the dense oracle."""
+    q, k = synthetic.gen_prefill(1200, 2, 128, seed=9)
+    b, _, _ = run_prefill(q, k, 1, 40, 40, oracle.REUSE, dense=True)
+    c, _, _ = run_prefill(q, k, 1, 40, 40, oracle.REUSE)
+    np.testing.assert_array_equal(b, c)
+    a, sa, _ = run_prefill(q, k, 1, 40, 80, oracle.REFINE)
+    ref = oracle.dense(q, k, 40)
+    pos = np.broadcast_to(np.arange(1200)[:, None], (1200, 2))
+    assert_parity(compare(a, ref["out"], ref["edge"], pos, None, sa, ref["score"]), "g=1 refine vs dense")
+
+
+# ------------------------------------------------------------ workload sizes
+def sampled_units(G, H, n, seed):
+    rng = np.random.default_rng(seed)
+    gi = rng.integers(0, G, size=n)
+    gi[:2] = [G - 1, max(0, G // 2)]           # the longest prefix and a ragged middle
+    hi = rng.integers(0, H, size=n)
+    return gi.astype(np.int32), hi.astype(np.int32)
+
+
+def check_sampled(name, modes, n_units):
+    c = synthetic.CONFIGS[name]
+    q, k = synthetic.make_prefill(name)
+    L, H, _ = q.shape
+    g, top_k, Kc = c["g"], c["top_k"], c["Kc"]
+    G = (L + g - 1) // g
+    qd, kd = to_dev(q), to_dev(k)
+    for mode in modes:
+        sc = torch.empty((L, H, top_k), dtype=torch.float32, device="cuda")
+        out = qg.pivot_index(qd, kd, g, top_k, Kc, mode, out_scores=sc)
+        qg.sync_status()
+        # properties of every row
+        o = out.cpu().numpy()
+        pos = np.broadcast_to(np.arange(L)[:, None], (L, H))
+        assert valid_rows(o, pos).all()
+        if mode == oracle.REFINE:
+            want_n = np.minimum(top_k, np.arange(L))[:, None]
+            assert np.all((o >= 0).sum(-1) == want_n)
+        gi, hi = sampled_units(G, H, n_units, seed=L + mode)
+        r = oracle.prefill_units(q, k, g, top_k, Kc, mode, gi, hi)
+        s = sc.cpu().numpy()
+        for u, (i, h) in enumerate(zip(gi, hi)):
+            rows = np.arange(i * g, min(i * g + g, L))
+            nm = len(rows)
+            res = compare(o[rows, h], r["out"][u, :nm], r["edge"][u, :nm], rows,
+                          np.broadcast_to(r["cand_edge"][u], (nm, 2)) if mode == oracle.REFINE else None,
+                          s[rows, h], r["score"][u, :nm])
+            assert_parity(res, f"{name} mode={mode} group={i} head={h}")
+        del out, sc
+    torch.cuda.empty_cache()
+
+
+def test_c1_sampled():
+    check_sampled("C1", (oracle.REFINE, oracle.REUSE), 96)
+
+
+def test_c2_sampled():
+    check_sampled("C2", (oracle.REFINE, oracle.REUSE), 24)
+
+
+def test_c3_sampled():
+    check_sampled("C3", (oracle.REFINE, oracle.REUSE), 12)
+
+
+def test_c1_dense_sampled():
+    c = synthetic.CONFIGS["C1"]
+    q, k = synthetic.make_prefill("C1")
+    L, H, _ = q.shape
+    got, gs, _ = run_prefill(q, k, 1, c["top_k"], c["top_k"], oracle.REUSE, dense=True)
+    rng = np.random.default_rng(17)
+    pi = rng.integers(0, L, size=64).astype(np.int32)
+    pi[0] = L - 1
+    hi = rng.integers(0, H, size=64).astype(np.int32)
+    r = oracle.dense_units(q, k, c["top_k"], pi, hi)
+    res = compare(got[pi, hi], r["out"], r["edge"], pi, None, gs[pi, hi], r["score"])
+    assert_parity(res, "C1 dense")
+
+
+# ------------------------------------------------------------------- decode
+def run_decode(dec, g, top_k, Kc, mode, max_seqlen):
+    qd = to_dev(dec.q)
+    kd = to_dev(dec.kcache)
+    cu = torch.from_numpy(dec.cu_seqlens).cuda()
+    B, _, H, _ = dec.q.shape
+    sc = torch.empty((B, g, H, top_k), dtype=torch.float32, device="cuda")
+    out = qg.pivot_decode_index(qd, kd, cu, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sc)
+    qg.sync_status()
+    return out.cpu().numpy(), sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("case", [
+    # B, H, d, g, lo, hi, top_k, Kc
+    (1, 1, 128, 1, 0, 0, 4, 8),
+    (3, 2, 64, 2, 0, 300, 16, 32),
+    (4, 2, 128, 2, 1000, 5000, 64, 128),
+    (2, 1, 128, 3, 200, 9000, 300, 700),
+    (5, 2, 64, 4, 50, 2500, 100, 200),
+])
+def test_decode_small(case):
+    B, H, d, g, lo, hi, top_k, Kc = case
+    dec = synthetic.gen_decode(B, H, d, g, seed=B * 31 + g, lo=lo, hi=hi)
+    max_seqlen = int(np.diff(dec.cu_seqlens).max())
+    bi, hh = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+    for mode in (oracle.REFINE, oracle.REUSE):
+        got, gs = run_decode(dec, g, top_k, Kc, mode, max_seqlen)
+        r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, g, top_k, Kc, mode, bi.ravel(), hh.ravel())
+        want = r["out"].reshape(B, H, g, top_k).transpose(0, 2, 1, 3)
+        edge = r["edge"].reshape(B, H, g, 2).transpose(0, 2, 1, 3)
+        wsc = r["score"].reshape(B, H, g, top_k).transpose(0, 2, 1, 3)
+        cedge = None
+        if mode == oracle.REFINE:
+            cedge = np.broadcast_to(r["cand_edge"].reshape(B, H, 1, 2).transpose(0, 2, 1, 3), (B, g, H, 2))
+        pos = np.broadcast_to((dec.n_ctx[:, None] + np.arange(g)[None, :])[:, :, None], (B, g, H))
+        res = compare(got, want, edge, pos, cedge, gs, wsc)
+        assert_parity(res, f"decode {case} mode={mode}")
