@@ -194,7 +194,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip the Reuse/dense comparison runs")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=2, help="0 skips the end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling aid: index only this many heads of the workload (0 = all)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -229,6 +232,8 @@ def main():
         return float(t.item())
 
     c = dict(synthetic.CONFIGS[WORKLOAD])
+    if args.heads > 0:
+        c["H"] = min(args.heads, c["H"])
     L, H, d, g, top_k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
     q_np, k_np = synthetic.gen_prefill(L, H, d, c["seed"] + rank, c["rho"], c["heavy_frac"], c["heavy_scale"])
     q = torch.from_numpy(q_np.view(np.int16)).cuda().view(torch.bfloat16)
@@ -290,6 +295,8 @@ def main():
     # end to end through the public API: pinned host inputs -> device -> indexer -> host result
     e2e = None
     try:
+        if args.e2e_steps <= 0:
+            raise RuntimeError("skipped (--e2e-steps 0)")
         q_h = torch.from_numpy(q_np.view(np.int16)).view(torch.bfloat16).pin_memory()
         k_h = torch.from_numpy(k_np.view(np.int16)).view(torch.bfloat16).pin_memory()
         try:
@@ -362,7 +369,7 @@ def main():
     if rank == 0:
         import oracle
         oracle.build()
-        cpu = cpu_baseline(c, q_np, k_np) if world == 1 else None
+        cpu = cpu_baseline(c, q_np, k_np) if (world == 1 and not args.no_cpu_baseline) else None
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(c),

@@ -50,8 +50,10 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;
   static constexpr int OFF_C = OFF_B + KATOMS * ATOM_B + 1024 - (KATOMS * ATOM_B) % 1024;
+  // candidate indices are staged for whole 128-row chunks (-1 past the set)
+  __host__ __device__ static int cidx_bytes(int Kc) { return ((Kc + 127) / 128) * 128 * 4; }
   static int smem_bytes(int Kc) {
-    return OFF_C + ((Kc * 4 + 15) & ~15) + 2 * static_cast<int>(sizeof(HalfSel)) + 64 + 1024;
+    return OFF_C + cidx_bytes(Kc) + 2 * static_cast<int>(sizeof(HalfSel)) + 64 + 1024;
   }
 };
 
@@ -66,7 +68,7 @@ __global__ void __launch_bounds__(256, 1) refine_kernel(RefineParams p) {
   const uint32_t sA = sbase + C::OFF_A;
   const uint32_t sB = sbase + C::OFF_B;
   int32_t* cidx = reinterpret_cast<int32_t*>(smem + C::OFF_C);
-  const int off_hs = C::OFF_C + ((p.Kc * 4 + 15) & ~15);
+  const int off_hs = C::OFF_C + C::cidx_bytes(p.Kc);
   HalfSel* hs = reinterpret_cast<HalfSel*>(smem + off_hs);
   uint8_t* tail = smem + off_hs + 2 * sizeof(HalfSel);
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);            // NS mma-done barriers
