@@ -120,6 +120,28 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode without any device allocation (the paper has no counterpart; this is
+ * a deployment variant of pivot_decode_index, same arguments and results).
+ * For callers that cannot allocate device memory during a decode step: an
+ * inference engine that has already handed all free HBM to its KV-cache pool,
+ * so a cudaMalloc there would fail or fragment it, or host code that has no
+ * allocator of its own and must not own device buffers.  Its scratch is a
+ * 32 MiB array built into the library (held by every GPU that loads it until
+ * the process exits); a call whose scratch need -- proxies B*H*d*2 + order keys
+ * H*B*max_seqlen*4 + (Refine) candidates H*B*Kc*4 bytes, each rounded up to
+ * 256 -- exceeds 32 MiB is rejected with PIVOT_ERR_WORKSPACE and a message.
+ * The first call on each device looks the array's address up (once, with that
+ * device current); make that first call before any stream capture.  All calls
+ * share the one array and it keeps the previous call's contents (nothing in it
+ * needs to start at zero): calls that may overlap on the GPU -- concurrent
+ * streams, or several host threads -- race on it and must be serialised by the
+ * caller.
+ */
+int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
+                               int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
+                               float* out_scores, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's kernel status
  * word.  Returns PIVOT_OK, PIVOT_ERR_TIMEOUT (a bounded wait inside a kernel
  * gave up; that call's outputs are not valid), PIVOT_ERR_INVALID_ARG (a decode

@@ -31,7 +31,7 @@ EXPORTED = (
     "pivot_index", "dense_index", "pivot_decode_index",
     "pivot_workspace_size", "pivot_index_ws", "dense_workspace_size", "dense_index_ws",
     "pivot_decode_workspace_size", "pivot_decode_index_ws", "pivot_sync_status", "pivot_last_error",
-    "pivot_trace_enable", "pivot_trace_collect",
+    "pivot_trace_enable", "pivot_trace_collect", "pivot_decode_index_noalloc",
 )
 
 
@@ -66,6 +66,7 @@ def load_library():
         "pivot_last_error": ([], ctypes.c_char_p),
         "pivot_trace_enable": ([I], I),
         "pivot_trace_collect": ([ctypes.c_char_p, Z, P, P, I], I),
+        "pivot_decode_index_noalloc": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)

@@ -483,7 +483,60 @@ int device_sms() {
 
 }  // namespace
 
+// ---------------------------------------------------------------- no-allocation decode
+// Scratch for pivot_decode_index_noalloc: a fixed device array that every GPU
+// loading this library holds until the process exits.  Host code must not pass
+// the symbol itself to a kernel (on the host it is only a stand-in); its device
+// address is looked up once per device below.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+void* g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call per device, with that device current).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(PIVOT_ERR_UNSUPPORTED, "no usable CUDA device");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(PIVOT_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return PIVOT_OK;
+}
+}  // namespace
+
 extern "C" {
+
+int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
+                               int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
+                               float* out_scores, void* stream) {
+  if (int rc = check_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores))
+    return rc;
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  const size_t need = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  if (need > kNoAllocScratchBytes)
+    return fail(PIVOT_ERR_WORKSPACE,
+                "pivot_decode_index_noalloc: this call needs %zu bytes of scratch, more than the %zu-byte static "
+                "maximum (use pivot_decode_index_ws with a caller workspace)",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  // Nothing in the decode scratch has to start at zero: every word is written
+  // before it is read within the call.
+  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, scratch,
+                    kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
+}
+
 
 size_t pivot_workspace_size(int L, int H, int d, int g, int top_k, int Kc, int mode) {
   if (L < 1 || H < 1 || g < 1 || top_k < 1 || Kc < top_k) return 0;
