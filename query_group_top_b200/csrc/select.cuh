@@ -2,10 +2,12 @@
 //
 // The K entries with the largest keys are kept; among equal keys the earlier
 // entry wins (entries are always presented in ascending key-index order, so
-// "earlier" is "lower index", the tie rule of the method).  The threshold key
-// T (the K-th largest) is found by a 4-pass MSB-first radix select with
-// 256-bin shared histograms; the selected entries are then emitted in entry
-// order with their output slot, so every output row comes out ascending.
+// "earlier" is "lower index", the tie rule of the method).  The rule is found
+// by an MSB-first radix select that starts at the highest key bit that varies
+// among the entries (bits above it are a common prefix) and consumes up to 11
+// bits per pass with a 2048-bin shared histogram, stopping as soon as the
+// boundary bin is taken whole.  The selected entries are emitted in entry order
+// with their output slot, so every output row comes out ascending.
 #pragma once
 
 #include "ptx.cuh"
@@ -14,10 +16,10 @@ namespace pivot {
 
 template <int NT>
 struct SelectSmem {
-  int hist[256];
+  int hist[2048];
   int warp_tot[NT / 32];
-  int bstar;
-  int above;
+  unsigned red[NT / 32];
+  int bstar, above, cntb;
 };
 
 // Exclusive block-wide prefix sum of one int per thread (all NT threads call).
@@ -49,67 +51,19 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_tot, int* t
   return warp_tot[warp] + incl - x;
 }
 
-// Finds, among entries e < n whose key matches (key & mask) == prefix, the
-// digit b at `shift` such that the number of matching entries with digit > b
-// is < rank <= that number plus the count of digit b.  Returns b; *above
-// receives the count with digit > b.
-template <int NT, class Fetch>
-__device__ __forceinline__ int radix_digit(int n, Fetch fetch, uint32_t prefix, uint32_t mask, int shift,
-                                           int rank, SelectSmem<NT>& sm, int* above) {
-  const int lane = threadIdx.x & 31;
-  for (int b = threadIdx.x; b < 256; b += NT) sm.hist[b] = 0;
-  if (threadIdx.x == 0) {
-    sm.bstar = 0;
-    sm.above = 0;
-  }
-  __syncthreads();
-  for (int base = 0; base < n; base += NT) {
-    const int e = base + threadIdx.x;
-    int digit = 256 + lane;  // unique sentinel: matches nobody
-    if (e < n) {
-      const uint32_t key = fetch(e);
-      if ((key & mask) == prefix) digit = (key >> shift) & 255;
-    }
-    const unsigned same = __match_any_sync(0xffffffffu, digit);
-    if (digit < 256 && lane == __ffs(same) - 1) atomicAdd(&sm.hist[digit], __popc(same));
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    // lane l owns bins [8*(31-l), 8*(31-l)+8): lane 0 holds the top bins.
-    const int hi_bin = 255 - 8 * lane;
-    int c[8];
-    int s = 0;
+// Block-wide OR of one value per thread.
+template <int NT>
+__device__ __forceinline__ unsigned block_or(unsigned x, unsigned* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      c[t] = sm.hist[hi_bin - t];
-      s += c[t];
-    }
-    int incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int excl = incl - s;
-    const unsigned hit = __ballot_sync(0xffffffffu, excl < rank && rank <= incl);
-    if (hit && lane == __ffs(hit) - 1) {
-      int cum = excl;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (cum + c[t] >= rank) {
-          sm.bstar = hi_bin - t;
-          sm.above = cum;
-          break;
-        }
-        cum += c[t];
-      }
-    }
-  }
+  for (int o = 16; o > 0; o >>= 1) x |= __shfl_xor_sync(0xffffffffu, x, o);
   __syncthreads();
-  const int b = sm.bstar;
-  *above = sm.above;
+  if (lane == 0) red[warp] = x;
   __syncthreads();
-  return b;
+  unsigned r = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) r |= red[w];
+  return r;
 }
 
 // Selects the top K of n entries (K <= n) and calls emit(slot, e) for each
@@ -121,50 +75,86 @@ __device__ void block_select_emit(int n, int K, Fetch fetch, Emit emit, SelectSm
     for (int e = threadIdx.x; e < n; e += NT) emit(e, e);
     return;
   }
-  uint32_t prefix = 0, mask = 0;
-  int rank = K;
+  // bits that vary among the keys
+  const uint32_t key0 = fetch(0);
+  unsigned diff = 0;
+  for (int e = threadIdx.x; e < n; e += NT) diff |= fetch(e) ^ key0;
+  diff = block_or<NT>(diff, sm.red);
+  int sh = 32 - __clz(diff);                     // bits [sh, 32) are common to all keys
+  uint32_t tmask = sh >= 32 ? 0u : (0xFFFFFFFFu << sh);
+  uint32_t thr = key0 & tmask;
+  int rank = K;                                  // how many keys at or above thr to take
+  bool whole = false;
+  bool ties = (sh == 0);                         // all keys equal: first K in order
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    int above;
-    const int b = radix_digit<NT>(n, fetch, prefix, mask, shift, rank, sm, &above);
-    prefix |= static_cast<uint32_t>(b) << shift;
-    mask |= 0xFFu << shift;
-    rank -= above;
+  while (sh > 0) {
+    const int width = sh >= 11 ? 11 : sh;
+    sh -= width;
+    const int nbn = 1 << width;
+    for (int b = threadIdx.x; b < nbn; b += NT) sm.hist[b] = 0;
+    if (threadIdx.x == 0) {
+      sm.bstar = 0;
+      sm.above = 0;
+      sm.cntb = 0;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += NT) {
+      const uint32_t key = fetch(e);
+      if ((key & tmask) == thr) atomicAdd(&sm.hist[(key >> sh) & (nbn - 1)], 1);
+    }
+    __syncthreads();
+    // thread t owns bins [top - per + 1, top], scanned from the top
+    const int per = (nbn + NT - 1) / NT;
+    const int top = nbn - 1 - per * static_cast<int>(threadIdx.x);
+    int s = 0;
+    for (int t = 0; t < per; ++t)
+      if (top - t >= 0) s += sm.hist[top - t];
+    const int excl = block_exclusive_scan<NT>(s, sm.warp_tot, nullptr);
+    if (excl < rank && rank <= excl + s) {
+      int cum = excl;
+      for (int t = 0; t < per; ++t) {
+        const int cb = sm.hist[top - t];
+        if (cum + cb >= rank) {
+          sm.bstar = top - t;
+          sm.above = cum;
+          sm.cntb = cb;
+          break;
+        }
+        cum += cb;
+      }
+    }
+    __syncthreads();
+    thr |= static_cast<uint32_t>(sm.bstar) << sh;
+    tmask |= static_cast<uint32_t>(nbn - 1) << sh;
+    rank -= sm.above;
+    whole = (sm.cntb == rank);
+    __syncthreads();
+    if (whole) break;          // every key of the boundary bin is taken
+    if (sh == 0) ties = true;  // equal keys, only `rank` of them are taken
   }
-  const uint32_t T = prefix;   // K-th largest key
-  const int need_eq = rank;    // how many entries equal to T are taken (earliest first)
 
   // Each thread owns a contiguous run of entries so that entry order is kept.
   const int per = (n + NT - 1) / NT;
   const int e0 = min(n, static_cast<int>(threadIdx.x) * per);
   const int e1 = min(n, e0 + per);
-  int n_eq = 0;
-  for (int e = e0; e < e1; ++e) n_eq += (fetch(e) == T);
-  const int eq_before = block_exclusive_scan<NT>(n_eq, sm.warp_tot, nullptr);
+  int eq_before = 0;
+  if (ties) {
+    int n_eq = 0;
+    for (int e = e0; e < e1; ++e) n_eq += (fetch(e) == thr);
+    eq_before = block_exclusive_scan<NT>(n_eq, sm.warp_tot, nullptr);
+  }
+  auto take = [&](uint32_t key, int& seen) -> bool {
+    if (!ties) return (key & tmask) >= thr;
+    if (key > thr) return true;
+    if (key == thr) return (eq_before + seen++) < rank;
+    return false;
+  };
   int n_sel = 0, seen = 0;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t key = fetch(e);
-    if (key > T) {
-      ++n_sel;
-    } else if (key == T) {
-      n_sel += (eq_before + seen < need_eq);
-      ++seen;
-    }
-  }
-  const int sel_before = block_exclusive_scan<NT>(n_sel, sm.warp_tot, nullptr);
-  int slot = sel_before;
+  for (int e = e0; e < e1; ++e) n_sel += take(fetch(e), seen);
+  int slot = block_exclusive_scan<NT>(n_sel, sm.warp_tot, nullptr);
   seen = 0;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t key = fetch(e);
-    bool take = false;
-    if (key > T) {
-      take = true;
-    } else if (key == T) {
-      take = (eq_before + seen < need_eq);
-      ++seen;
-    }
-    if (take) emit(slot++, e);
-  }
+  for (int e = e0; e < e1; ++e)
+    if (take(fetch(e), seen)) emit(slot++, e);
 }
 
 }  // namespace pivot
