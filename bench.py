@@ -361,10 +361,40 @@ def main():
             pv = o[rows, heads].cpu().numpy()
             hit = [np.intersect1d(a[a >= 0], b[b >= 0]).size / max(1, (b >= 0).sum()) for a, b in zip(pv, dn)]
             rec[name] = float(np.mean(hit))
-        extras = {"refine_ms": ms, "reuse_ms": reuse_ms, "dense_ms": dense_ms,
+        del out_dense
+        # MTP decode workload: one step over 64 sequences (keys drawn on the device)
+        dc = synthetic.CONFIGS["C4"]
+        dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], dc["seed"] + rank,
+                                                         dc["lo"], dc["hi"], dc["rho"], dc["heavy_frac"],
+                                                         dc["heavy_scale"])
+        max_seqlen = int((n_ctx + dc["g"]).max())
+        dout = torch.empty((dc["B"], dc["g"], dc["H"], dc["top_k"]), dtype=torch.int32, device="cuda")
+        dstep = lambda: qg.pivot_decode_index(dq, dk, dcu, dc["g"], dc["top_k"], dc["Kc"], qg.REFINE,
+                                              max_seqlen=max_seqlen, out=dout)
+        for _ in range(2):
+            dstep()
+        torch.cuda.synchronize()
+        qg.trace_enable(True)
+        dec_ms = timed(dstep, args.steps)
+        qg.trace_enable(False)
+        dtr = qg.trace_collect()
+        qg.sync_status()
+        key_bytes = float(n_ctx.astype(np.int64).sum() + dc["B"] * (dc["g"] - 1)) * dc["H"] * dc["d"] * 2
+        dscan = dtr.get("decode_scan", (0.0, 1))
+        dscan_ms = dscan[0] / max(dscan[1], 1)
+        decode = {"workload": f"C4 MTP decode B={dc['B']} n_b~U[{dc['lo']},{dc['hi']}] H={dc['H']} d={dc['d']} "
+                              f"g={dc['g']} top_k={dc['top_k']} Kc={dc['Kc']} PIVOT-Refine",
+                  "ms_per_step": dec_ms, "query_heads_per_s": dc["B"] * dc["g"] * dc["H"] / (dec_ms / 1000.0),
+                  "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in dtr.items()},
+                  "decode_scan_hbm_gbs": key_bytes / (dscan_ms / 1000.0) / 1e9 if dscan_ms else None,
+                  "decode_scan_hbm_frac": (key_bytes / (dscan_ms / 1000.0) / 1e9 / pk["hbm"]) if dscan_ms else None,
+                  "key_bytes": key_bytes}
+        del dq, dk, dcu, dout
+        torch.cuda.empty_cache()
+        extras = {"refine_ms": ms, "reuse_ms": reuse_ms, "dense_ms": dense_ms, "decode": decode,
                   "speedup_refine_vs_dense": dense_ms / ms, "speedup_reuse_vs_dense": dense_ms / reuse_ms,
                   "recall_at_k_vs_dense": rec, "recall_rows": int(rows.numel())}
-        del out_reuse, out_dense
+        del out_reuse
 
     if rank == 0:
         import oracle

@@ -49,7 +49,8 @@ struct GroupSel {
 template <int D>
 struct RefineCfg {
   static constexpr int NT = 512;
-  static constexpr int NS = 4;                          // gather stages
+  static constexpr int NS = 5;                          // gather stages
+  static constexpr int LA = 3;                          // chunks in flight ahead of the MMA
   static constexpr int KATOMS = D / 64;
   static constexpr int ATOM_A = 128 * 128;              // 128 rows x 128 bytes
   static constexpr int STAGE = KATOMS * ATOM_A;
@@ -187,23 +188,25 @@ __global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
     }
     // ---- gather + MMA pipeline over candidate chunks
     const int seq0 = seq;
-    // always NS-1 groups in the prologue, so that wait_group<NS-1> below
-    // means "chunk c has landed" whatever nch is
-    for (int c = 0; c < C::NS - 1; ++c) {
+    // always LA groups in the prologue, so that wait_group<LA> below means
+    // "chunk c has landed" whatever nch is
+    for (int c = 0; c < C::LA; ++c) {
       if (c < nch) issue_gather(c, (seq0 + c) % C::NS);
       cp_async_commit();
     }
     for (int c = 0; c < nch; ++c) {
-      const int cn = c + C::NS - 1;
+      const int cn = c + C::LA;
       if (cn < nch) {
-        if (c >= 1) {
-          const int prev = seq0 + c - 1;  // chunk whose stage is refilled now
+        // the stage refilled now last held chunk cn - NS = c - 2, whose MMAs
+        // were issued two iterations ago
+        if (cn >= C::NS) {
+          const int prev = seq0 + cn - C::NS;
           if (!mbar_wait(bar0 + 8u * (prev % C::NS), (prev / C::NS) & 1, abort_flag, p.status)) ok = false;
         }
         if (ok) issue_gather(cn, (seq0 + cn) % C::NS);
       }
       cp_async_commit();
-      cp_async_wait<C::NS - 1>();
+      cp_async_wait<C::LA>();
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) {
         ok = false;

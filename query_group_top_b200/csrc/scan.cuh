@@ -203,56 +203,94 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
     if (sampling)
       for (int b = 0; b < 256; ++b) hist[b * C::BM + r] = 0;
 
+    // Main-pass staging for survivor lookups: this thread's 32 values of the
+    // current chunk as 8 float4 at [(i*128 + r)*4]; it reuses the histogram
+    // space, which is dead once tau is set.
+    float* stage = reinterpret_cast<float*>(hist);
+    // One chunk of 32 scores (columns j0 .. j0+31 of this row), by phase.
+    auto process = [&](const uint32_t (&v)[32], int j0, int phase) {
+      if (j0 >= bound) return;
+      const uint32_t live = (j0 + 32 <= bound) ? 0xFFFFFFFFu : ((1u << (bound - j0)) - 1u);
+      if (phase == 2) {
+        uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          if (__uint_as_float(v[x]) >= tau) m0 |= 1u << x;
+          if (__uint_as_float(v[x + 1]) >= tau) m1 |= 2u << x;
+        }
+        uint32_t m = (m0 | m1) & live;
+        if (m == 0) return;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          reinterpret_cast<uint4*>(stage)[q4 * C::BM + r] =
+              make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        while (m) {
+          const int x = __ffs(m) - 1;
+          m &= m - 1;
+          const float sc = stage[((x >> 2) * C::BM + r) * 4 + (x & 3)];
+          if (cnt < p.cap) spill[cnt] = make_uint2(score_key(sc), static_cast<uint32_t>(j0 + x));
+          ++cnt;
+        }
+      } else if (phase == 0) {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          if ((live >> x) & 1u) {
+            const uint32_t key = score_key(__uint_as_float(v[x]));
+            hist[(key >> 24) * C::BM + r] += 1;
+          }
+        }
+        n_sample += __popc(live);
+      } else if (b1 >= 0) {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          if ((live >> x) & 1u) {
+            const uint32_t key = score_key(__uint_as_float(v[x]));
+            if (static_cast<int>(key >> 24) == b1) hist[((key >> 16) & 255) * C::BM + r] += 1;
+          }
+        }
+      }
+    };
+
+    // An aborted warp keeps stepping (without waits or TMEM loads) so that it
+    // still reaches the epilogue-wide barrier at the end of the sample passes.
+    bool alive = true;
     for (int step = 0; step < nsteps; ++step) {
       const int ab = step & 1;
-      // the whole warp leaves together: tcgen05.ld below is warp-collective
-      const bool got = mbar_wait(tfull_bar(ab), (step >> 1) & 1, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, got)) break;
+      // the whole warp decides together: tcgen05.ld below is warp-collective
+      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(ab), (step >> 1) & 1, abort_flag, p.status));
+      if (alive) {
       tc_fence_after();
       const int jt = step_tile(step);
       const int phase = step < ns ? 0 : (step < 2 * ns ? 1 : 2);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::BN;
+      // two register buffers: the TMEM load of chunk c+1 overlaps the work on chunk c
+      uint32_t va[32], vb[32];
+      tmem_ld_32x32b_x32(taddr, va);
+      tmem_ld_wait();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) reg_fence(va[x]);
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
+      for (int c = 0; c < C::BN / 32; c += 2) {
+        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, vb);
+        process(va, jt * C::BN + c * 32, phase);
         tmem_ld_wait();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) reg_fence(v[x]);
-        if (c == C::BN / 32 - 1) {
+        for (int x = 0; x < 32; ++x) reg_fence(vb[x]);
+        if (c + 2 < C::BN / 32) {
+          tmem_ld_32x32b_x32(taddr + (c + 2) * 32, va);
+        } else {
+          // every column of this accumulator buffer is in registers now
           tc_fence_before();
           mbar_arrive(tempty_bar(ab));
         }
-        const int j0 = jt * C::BN + c * 32;
-        if (j0 >= bound) continue;
-        if (phase == 2) {
+        process(vb, jt * C::BN + (c + 1) * 32, phase);
+        if (c + 2 < C::BN / 32) {
+          tmem_ld_wait();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const float s = __uint_as_float(v[x]);
-            if (j0 + x < bound && s >= tau) {
-              if (cnt < p.cap) spill[cnt] = make_uint2(score_key(s), static_cast<uint32_t>(j0 + x));
-              ++cnt;
-            }
-          }
-        } else if (phase == 0) {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            if (j0 + x < bound) {
-              const uint32_t key = score_key(__uint_as_float(v[x]));
-              hist[(key >> 24) * C::BM + r] += 1;
-              ++n_sample;
-            }
-          }
-        } else if (b1 >= 0) {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            if (j0 + x < bound) {
-              const uint32_t key = score_key(__uint_as_float(v[x]));
-              if (static_cast<int>(key >> 24) == b1) hist[((key >> 16) & 255) * C::BM + r] += 1;
-            }
-          }
+          for (int x = 0; x < 32; ++x) reg_fence(va[x]);
         }
       }
+      }  // alive
       if (step == ns - 1) {
         // end of the first sample pass: choose the top digit of tau
         if (row_samples && n_sample > 0) {
@@ -286,6 +324,9 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
           }
           tau = key_lower_edge_value((static_cast<uint32_t>(b1) << 24) | (static_cast<uint32_t>(b2) << 16));
         }
+        // the main pass reuses the histogram space for staging: every
+        // epilogue thread must be done with its histogram column first
+        named_barrier(1, 128);
       }
     }
     if (row_ok) p.cnt[row_id] = cnt;

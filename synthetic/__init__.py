@@ -154,3 +154,51 @@ def make_prefill(name: str):
     if c["kind"] == "iid":
         return gen_iid(c["L"], c["H"], c["d"], c["seed"])
     return gen_prefill(c["L"], c["H"], c["d"], c["seed"], c["rho"], c["heavy_frac"], c["heavy_scale"])
+
+
+def gen_decode_device(B: int, H: int, d: int, g: int, seed: int, lo: int, hi: int,
+                      rho: float = 0.95, heavy_frac: float = 0.01, heavy_scale: float = 4.0,
+                      device="cuda"):
+    """Large decode batches drawn on the GPU (same recipe as ``gen_decode``).
+
+    Context lengths, heavy-key positions and the step queries come from numpy
+    exactly as in ``gen_decode``; the key rows themselves are drawn with
+    torch's device generator seeded per sequence (seed * 1000003 + b), in fp32,
+    then rounded to bf16 (round to nearest even).  Returns torch tensors
+    (q [B,g,H,d] bf16, kcache [rows,H,d] bf16, cu_seqlens [B+1] int32) on the
+    device and the numpy context lengths.  Use ``kcache[cu[b]:cu[b+1]]`` to
+    read a sequence back for a CPU check.
+    """
+    import torch
+    rng = np.random.default_rng(seed)
+    n_ctx = rng.integers(lo, hi, size=B, endpoint=True).astype(np.int32)
+    lens = n_ctx.astype(np.int64) + g
+    cu = np.zeros(B + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(lens)
+    if cu[-1] >= 2**31:
+        raise ValueError("decode cache too large for int32 offsets")
+    kc = torch.empty((int(cu[-1]), H, d), dtype=torch.bfloat16, device=device)
+    q = np.empty((B, g, H, d), dtype=np.uint16)
+    a = np.float32(rho)
+    b_ = np.float32(math.sqrt(1.0 - rho * rho))
+    gen = torch.Generator(device=device)
+    for b in range(B):
+        n = int(lens[b])
+        gen.manual_seed(seed * 1000003 + b)
+        kb = torch.randn((n, H, d), generator=gen, device=device, dtype=torch.float32)
+        n_heavy = int(round(heavy_frac * n))
+        if n_heavy > 0:
+            pos = np.random.default_rng([seed, b]).choice(n, size=n_heavy, replace=False)
+            kb[torch.from_numpy(pos).to(device)] *= heavy_scale
+        kc[int(cu[b]):int(cu[b + 1])] = kb.to(torch.bfloat16)
+        del kb
+        rq = np.random.default_rng([seed, b, 1])
+        eps = rq.standard_normal((g, H, d), dtype=np.float32)
+        qq = np.empty_like(eps)
+        qq[0] = eps[0]
+        for i in range(1, g):
+            qq[i] = a * qq[i - 1] + b_ * eps[i]
+        q[b] = bf16_from_f32(qq)
+    qd = torch.from_numpy(q.view(np.int16)).to(device).view(torch.bfloat16)
+    cud = torch.from_numpy(cu.astype(np.int32)).to(device)
+    return qd, kc, cud, n_ctx

@@ -215,3 +215,40 @@ def test_decode_small(case):
         pos = np.broadcast_to((dec.n_ctx[:, None] + np.arange(g)[None, :])[:, :, None], (B, g, H))
         res = compare(got, want, edge, pos, cedge, gs, wsc)
         assert_parity(res, f"decode {case} mode={mode}")
+
+
+def test_c4_decode_sampled():
+    """The MTP decode workload at full size (64 sequences, contexts up to 131072,
+    19 GB of keys) in the launch configuration the bench times; the oracle
+    checks whole sequences, all heads, the longest included."""
+    c = synthetic.CONFIGS["C4"]
+    g, top_k, Kc, H = c["g"], c["top_k"], c["Kc"], c["H"]
+    q, kc, cu, n_ctx = synthetic.gen_decode_device(c["B"], H, c["d"], g, c["seed"], c["lo"], c["hi"],
+                                                   c["rho"], c["heavy_frac"], c["heavy_scale"])
+    max_seqlen = int((n_ctx + g).max())
+    cu_h = cu.cpu().numpy()
+    rng = np.random.default_rng(44)
+    seqs = [int(np.argmax(n_ctx)), int(np.argmin(n_ctx))] + list(rng.integers(0, c["B"], size=1))
+    for mode in (oracle.REFINE, oracle.REUSE):
+        sc = torch.empty((c["B"], g, H, top_k), dtype=torch.float32, device="cuda")
+        out = qg.pivot_decode_index(q, kc, cu, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sc)
+        qg.sync_status()
+        o = out.cpu().numpy()
+        pos = np.broadcast_to((n_ctx[:, None] + np.arange(g)[None, :])[:, :, None], o.shape[:3])
+        assert valid_rows(o, pos).all()
+        s = sc.cpu().numpy()
+        for b in seqs:
+            kb = kc[int(cu_h[b]):int(cu_h[b + 1])].cpu().view(torch.int16).numpy().view(np.uint16)
+            qb = q[b:b + 1].cpu().view(torch.int16).numpy().view(np.uint16)
+            cub = np.array([0, kb.shape[0]], np.int32)
+            r = oracle.decode_units(qb, kb, cub, g, top_k, Kc, mode, np.zeros(H, np.int32), np.arange(H, dtype=np.int32))
+            want = r["out"].transpose(1, 0, 2)            # [g, H, k]
+            edge = r["edge"].transpose(1, 0, 2)
+            cedge = None
+            if mode == oracle.REFINE:
+                cedge = np.broadcast_to(r["cand_edge"][None], (g, H, 2))
+            res = compare(o[b], want, edge, pos[b], cedge, s[b], r["score"].transpose(1, 0, 2))
+            assert_parity(res, f"C4 mode={mode} seq={b} n_ctx={n_ctx[b]}")
+        del out, sc
+    del kc
+    torch.cuda.empty_cache()
