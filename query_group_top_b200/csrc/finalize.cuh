@@ -21,7 +21,7 @@ struct FinalizeParams {
   int width;       // output row width (Kc for candidate rows, top_k for index rows)
   int broadcast;   // 0: write the candidate row; 1: write the row to every member's output row
   const uint2* spill;
-  const int* cnt;
+  const int2* cnt;   // per row: entries stored upward from slot 0, and downward from slot cap-1
   int32_t* cand;   // [H*G][width] when broadcast == 0
   int32_t* out;    // [L][H][width] when broadcast == 1
   float* out_scores;  // [L][H][width] or null (broadcast == 1 only)
@@ -72,17 +72,20 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
   sp.G = p.G; sp.L = p.L; sp.g = p.g; sp.bound_kind = p.bound_kind;
   const int bound = row_bound(sp, i);
   const int K = min(p.K_sel, bound);
-  const int n = p.cnt[row_id];
-  if (bound > p.cap && (n < K || n > p.cap)) {
+  const int2 c2 = p.cnt[row_id];
+  const int n = c2.x + c2.y;
+  if (n > p.cap || (bound > p.cap && n < K)) {
     if (threadIdx.x == 0) {
       const int slot = atomicAdd(p.fb_count, 1);
       p.fb_list[slot] = static_cast<int>(row_id);
     }
     return;
   }
-  const int nn = min(n, p.cap);
+  // the upward run (lower key indices) first, then the downward run reversed:
+  // entries in ascending key-index order
+  const int nn = n;
   const uint2* src = p.spill + row_id * p.cap;
-  for (int e = threadIdx.x; e < nn; e += kFinNT) ent[e] = src[e];
+  for (int e = threadIdx.x; e < nn; e += kFinNT) ent[e] = e < c2.x ? src[e] : src[p.cap - 1 - (e - c2.x)];
   __syncthreads();
   block_select_emit<kFinNT>(
       nn, K, [&](int e) { return ent[e].x; },

@@ -193,7 +193,7 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   p.off_spill = o;
   o += up(rows_pass * p.cap * sizeof(uint2));
   p.off_cnt = o;
-  o += up(rows_pass * sizeof(int));
+  o += up(rows_pass * sizeof(int2));
   p.off_fb = o;
   o += up(sizeof(int));
   p.off_fblist = o;
@@ -300,7 +300,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     sp.S = pl.S;
     sp.tiles_per_head = (pl.G + 127) / 128;
     sp.spill = reinterpret_cast<uint2*>(w + pl.off_spill);
-    sp.cnt = reinterpret_cast<int*>(w + pl.off_cnt);
+    sp.cnt = reinterpret_cast<int2*>(w + pl.off_cnt);
     sp.status = dev->status;
     int rc = (d == 128) ? launch_scan<128>(tmP, tmK, sp, nh, st) : launch_scan<64>(tmP, tmK, sp, nh, st);
     if (rc) return rc;

@@ -56,11 +56,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits until the phase with the given parity of `bar` has completed.
 // Returns false (and sets *abort, raising kStTimeout) after kWaitNs, or
-// returns false at once when another role has already set *abort.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+// returns false at once when another role has already set *abort.  With
+// max_sleep_ns > 0 the waiting warp backs off between polls (doubling sleeps
+// up to that bound), leaving issue slots to the warps it is waiting for.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                          unsigned max_sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
+  unsigned sleep_ns = 32;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
@@ -68,6 +71,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       *abort = 1;
       atomicOr(status, kStTimeout);
       return false;
+    }
+    if (max_sleep_ns) {
+      __nanosleep(sleep_ns);
+      sleep_ns = min(2 * sleep_ns, max_sleep_ns);
     }
   }
 }
@@ -189,6 +196,19 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Barrier over `nthreads` threads that also returns whether any of them passed pred != 0.
+__device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(res)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return res != 0;
 }
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

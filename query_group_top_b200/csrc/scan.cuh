@@ -12,7 +12,8 @@
 // -> TMEM pipeline:
 //   warp 0      TMA producer (keys, and the proxy tile once)
 //   warp 1      TMEM allocator and MMA issuer (one elected thread)
-//   warps 2..5  epilogue: thread r owns TMEM lane r = proxy row r
+//   warps 2..9  epilogue, two groups of four: thread (e, r) owns TMEM lane r
+//               (proxy row r) of accumulator buffer e
 // The score matrix is never written out.  Each epilogue thread compares its
 // row's scores with a per-row threshold tau and appends the survivors
 // (order key, key index) to that row's spill list in global memory; an exact
@@ -44,8 +45,11 @@ struct ScanParams {
   int cap;         // spill capacity per row (entries)
   int S;           // sample stride in key tiles (every S-th tile is sampled)
   int tiles_per_head;
-  uint2* spill;    // [H*G][cap]: (order key, key index)
-  int* cnt;        // [H*G]: survivors per row (may exceed cap: overflow)
+  uint2* spill;    // [H*G][cap]: (order key, key index); see cnt
+  int2* cnt;       // [H*G]: survivors from the first half of the row's key
+                   // tiles (stored upward from slot 0) and from the second half
+                   // (stored downward from slot cap-1); a sum above cap means
+                   // the list overflowed
   int* status;     // device status word
 };
 
@@ -62,18 +66,19 @@ struct ScanCfg {
   static constexpr int NST = (D == 128) ? 2 : 4;      // key-tile stages in shared memory
   static constexpr int A_BYTES = BM * D * 2;
   static constexpr int B_BYTES = BN * D * 2;
-  static constexpr int HIST_BYTES = 256 * BM * 2;     // u16 [256 bins][128 rows]
+  static constexpr int HIST_BYTES = 128 * BM * 4;     // [128 bin pairs][128 rows], two u16 counts per word
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + A_BYTES;
   static constexpr int OFF_HIST = OFF_B + NST * B_BYTES;
-  static constexpr int OFF_BAR = OFF_HIST + HIST_BYTES;
+  static constexpr int OFF_MISC = OFF_HIST + HIST_BYTES;  // per-row sample counts of the two groups
+  static constexpr int OFF_BAR = OFF_MISC + 2 * BM * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;   // barriers + alignment slack
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 2 * BN;       // double-buffered accumulator
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_constant__ CUtensorMap tm_keys,
                    ScanParams p) {
   using C = ScanCfg<D>;
@@ -82,7 +87,8 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sA = sbase + C::OFF_A;
   const uint32_t sB = sbase + C::OFF_B;
-  uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::OFF_HIST);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
+  int* nsamp = reinterpret_cast<int*>(smem + C::OFF_MISC);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   // barrier slots: [0,NST) full, [NST,2NST) empty, 2NST a_full, 2NST+1..2 tmem_full, 2NST+3..4 tmem_empty
   const uint32_t bar0 = smem_u32(bars);
@@ -102,6 +108,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
   const int i_last = min(i0 + C::BM, p.G) - 1;
   const int max_bound = row_bound(p, i_last);
   const int nkt = (max_bound + C::BN - 1) / C::BN;                // key tiles needed
+  const int nA = (nkt + 1) / 2;                                    // first-half tiles
   const bool sampling = max_bound > p.cap;
   const int ns = sampling ? nkt / p.S : 0;                         // sampled tiles
   const int nsteps = 2 * ns + nkt;
@@ -128,10 +135,14 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Step order: the two sample passes, then the main pass with even steps on
+  // the first half of the key tiles and odd steps on the second half, so that
+  // accumulator buffer b = step & 1 always belongs to epilogue group b.
   auto step_tile = [&](int step) -> int {
     if (step < ns) return (step + 1) * p.S - 1;
     if (step < 2 * ns) return (step - ns + 1) * p.S - 1;
-    return step - 2 * ns;
+    const int m = step - 2 * ns;
+    return (m & 1) ? nA + (m >> 1) : (m >> 1);
   };
 
   if (warp == 0) {
@@ -188,6 +199,10 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Two groups of four warps; group e owns accumulator buffer e (steps of
+    // parity e).  Thread (e, r) handles row r: group 0 the first half of its
+    // key tiles, group 1 the second half.
+    const int e = (warp - 2) >> 2;
     const int quarter = warp & 3;               // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;          // proxy row within the tile
     const int i = i0 + r;
@@ -200,14 +215,71 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
     int n_sample = 0;
     int b1 = -1, rem = 0;
     const bool row_samples = sampling && bound > p.cap;
-    if (sampling)
-      for (int b = 0; b < 256; ++b) hist[b * C::BM + r] = 0;
+
+    auto bin_count = [&](int b) -> int { return (hist[(b >> 1) * C::BM + r] >> ((b & 1) << 4)) & 0xFFFF; };
+    auto bin_add = [&](int b) { atomicAdd(&hist[(b >> 1) * C::BM + r], 1u << ((b & 1) << 4)); };
+    auto zero_half_row = [&]() {
+      for (int w = 0; w < 64; ++w) hist[(e * 64 + w) * C::BM + r] = 0;
+    };
+    // Phase changes (sample pass 1 -> 2 -> main); every epilogue thread of both
+    // groups takes the same barriers, in the same order.
+    int done = sampling ? 0 : 2;
+    if (sampling) {
+      zero_half_row();
+      named_barrier(1, 256);
+    }
+    auto advance = [&](int target) {
+      while (done < target) {
+        if (done == 0) {
+          // end of sample pass 1: choose the top digit of tau
+          nsamp[e * C::BM + r] = n_sample;
+          named_barrier(1, 256);
+          const int total = nsamp[r] + nsamp[C::BM + r];
+          if (row_samples && total > 0) {
+            const float expect = static_cast<float>(p.K_sel) * static_cast<float>(total) / static_cast<float>(bound);
+            const int target_rank = static_cast<int>(ceilf(expect + 4.0f * sqrtf(expect) + 4.0f));
+            if (target_rank <= total) {
+              int cum = 0;
+              for (int b = 255; b >= 0; --b) {
+                const int cb = bin_count(b);
+                if (cum + cb >= target_rank) {
+                  b1 = b;
+                  rem = target_rank - cum;
+                  break;
+                }
+                cum += cb;
+              }
+            }
+          }
+          named_barrier(1, 256);
+          zero_half_row();
+          named_barrier(1, 256);
+        } else {
+          // end of sample pass 2: the second digit, then tau
+          named_barrier(1, 256);
+          if (b1 >= 0) {
+            int cum = 0, b2 = 0;
+            for (int b = 255; b >= 0; --b) {
+              const int cb = bin_count(b);
+              if (cum + cb >= rem) {
+                b2 = b;
+                break;
+              }
+              cum += cb;
+            }
+            tau = key_lower_edge_value((static_cast<uint32_t>(b1) << 24) | (static_cast<uint32_t>(b2) << 16));
+          }
+          // the main pass reuses the histogram space for staging
+          named_barrier(1, 256);
+        }
+        ++done;
+      }
+    };
 
     // Main-pass staging for survivor lookups: this thread's 32 values of the
-    // current chunk as 8 float4 at [(i*128 + r)*4]; it reuses the histogram
-    // space, which is dead once tau is set.
+    // current chunk as 8 float4 at [((e*8 + i)*128 + r)*4].
     float* stage = reinterpret_cast<float*>(hist);
-    // One chunk of 32 scores (columns j0 .. j0+31 of this row), by phase.
+    const int stage_base = e * 8 * C::BM;
     auto process = [&](const uint32_t (&v)[32], int j0, int phase) {
       if (j0 >= bound) return;
       const uint32_t live = (j0 + 32 <= bound) ? 0xFFFFFFFFu : ((1u << (bound - j0)) - 1u);
@@ -222,47 +294,46 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
         if (m == 0) return;
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
-          reinterpret_cast<uint4*>(stage)[q4 * C::BM + r] =
+          reinterpret_cast<uint4*>(stage)[stage_base + q4 * C::BM + r] =
               make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
         while (m) {
           const int x = __ffs(m) - 1;
           m &= m - 1;
-          const float sc = stage[((x >> 2) * C::BM + r) * 4 + (x & 3)];
-          if (cnt < p.cap) spill[cnt] = make_uint2(score_key(sc), static_cast<uint32_t>(j0 + x));
+          const float sc = stage[((stage_base + (x >> 2) * C::BM) + r) * 4 + (x & 3)];
+          if (cnt < p.cap) {
+            const uint2 ent = make_uint2(score_key(sc), static_cast<uint32_t>(j0 + x));
+            spill[e == 0 ? cnt : p.cap - 1 - cnt] = ent;
+          }
           ++cnt;
         }
       } else if (phase == 0) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          if ((live >> x) & 1u) {
-            const uint32_t key = score_key(__uint_as_float(v[x]));
-            hist[(key >> 24) * C::BM + r] += 1;
-          }
-        }
+        for (int x = 0; x < 32; ++x)
+          if ((live >> x) & 1u) bin_add(static_cast<int>(score_key(__uint_as_float(v[x])) >> 24));
         n_sample += __popc(live);
       } else if (b1 >= 0) {
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
           if ((live >> x) & 1u) {
             const uint32_t key = score_key(__uint_as_float(v[x]));
-            if (static_cast<int>(key >> 24) == b1) hist[((key >> 16) & 255) * C::BM + r] += 1;
+            if (static_cast<int>(key >> 24) == b1) bin_add(static_cast<int>((key >> 16) & 255));
           }
         }
       }
     };
 
     // An aborted warp keeps stepping (without waits or TMEM loads) so that it
-    // still reaches the epilogue-wide barrier at the end of the sample passes.
+    // still takes every phase barrier.
     bool alive = true;
-    for (int step = 0; step < nsteps; ++step) {
-      const int ab = step & 1;
+    for (int step = e; step < nsteps; step += 2) {
+      const int phase = step < ns ? 0 : (step < 2 * ns ? 1 : 2);
+      advance(phase);
       // the whole warp decides together: tcgen05.ld below is warp-collective
-      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(ab), (step >> 1) & 1, abort_flag, p.status));
-      if (alive) {
+      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(e), (step >> 1) & 1, abort_flag, p.status, 256));
+      if (!alive) continue;
       tc_fence_after();
       const int jt = step_tile(step);
-      const int phase = step < ns ? 0 : (step < 2 * ns ? 1 : 2);
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::BN;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + e * C::BN;
       // two register buffers: the TMEM load of chunk c+1 overlaps the work on chunk c
       uint32_t va[32], vb[32];
       tmem_ld_32x32b_x32(taddr, va);
@@ -281,7 +352,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
         } else {
           // every column of this accumulator buffer is in registers now
           tc_fence_before();
-          mbar_arrive(tempty_bar(ab));
+          mbar_arrive(tempty_bar(e));
         }
         process(vb, jt * C::BN + (c + 1) * 32, phase);
         if (c + 2 < C::BN / 32) {
@@ -290,46 +361,9 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
           for (int x = 0; x < 32; ++x) reg_fence(va[x]);
         }
       }
-      }  // alive
-      if (step == ns - 1) {
-        // end of the first sample pass: choose the top digit of tau
-        if (row_samples && n_sample > 0) {
-          const float expect = static_cast<float>(p.K_sel) * static_cast<float>(n_sample) / static_cast<float>(bound);
-          const int target = static_cast<int>(ceilf(expect + 4.0f * sqrtf(expect) + 4.0f));
-          if (target <= n_sample) {
-            int cum = 0;
-            for (int b = 255; b >= 0; --b) {
-              const int cb = hist[b * C::BM + r];
-              if (cum + cb >= target) {
-                b1 = b;
-                rem = target - cum;
-                break;
-              }
-              cum += cb;
-            }
-          }
-        }
-        for (int b = 0; b < 256; ++b) hist[b * C::BM + r] = 0;
-      } else if (step == 2 * ns - 1) {
-        // end of the second sample pass: the second digit, then tau
-        if (b1 >= 0) {
-          int cum = 0, b2 = 0;
-          for (int b = 255; b >= 0; --b) {
-            const int cb = hist[b * C::BM + r];
-            if (cum + cb >= rem) {
-              b2 = b;
-              break;
-            }
-            cum += cb;
-          }
-          tau = key_lower_edge_value((static_cast<uint32_t>(b1) << 24) | (static_cast<uint32_t>(b2) << 16));
-        }
-        // the main pass reuses the histogram space for staging: every
-        // epilogue thread must be done with its histogram column first
-        named_barrier(1, 128);
-      }
     }
-    if (row_ok) p.cnt[row_id] = cnt;
+    advance(2);
+    if (row_ok) reinterpret_cast<int*>(p.cnt)[2 * row_id + e] = cnt;
   }
 
   tc_fence_before();
