@@ -17,8 +17,10 @@
 // Selection: the 16 warps form 4 groups of 4 (one warp per TMEM lane quarter,
 // so each group sees all 128 lanes); group q takes members q, q+4, ...  For a
 // member, thread r loads its block's scores, and an exact radix select on the
-// 32-bit order keys (11 + 11 + 10 bit digits, shared-memory histograms, early
-// stop once the boundary bin is taken whole) finds the k-th largest key.
+// 32-bit order keys finds the k-th largest key: it starts at the highest key
+// bit that varies across the member's candidates (a group-wide AND/OR), takes
+// up to 11 bits per pass with a shared histogram and stops as soon as the
+// boundary bin is taken whole.
 // Because every thread owns an ascending run of candidates, one exclusive scan
 // over the 128 threads orders the output, ascending by key index.
 #pragma once
@@ -43,6 +45,8 @@ struct GroupSel {
   int hist[2048];
   int wsum[4];
   int wsum2[4];
+  uint32_t wand[4];
+  uint32_t wor[4];
   int bstar, above, cntb;
 };
 
@@ -169,11 +173,6 @@ __global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
   const int r = quarter * 32 + lane;  // TMEM lane: this thread's candidate block
   GroupSel& S = gsel[grp];
 
-  // this thread's candidates, ascending, -1 past the set
-  int cand[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) cand[c] = (c < nch) ? cidx[r * nch + c] : -1;
-
   for (int mb = 0; mb < nm && ok; mb += 16) {
     const int nb = min(16, nm - mb);
     // ---- member queries -> B operand (16 rows, swizzled), zero rows past nb
@@ -239,6 +238,7 @@ __global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
     tc_fence_after();
 
     // ---- per-member exact top-k, four groups of 128 threads in parallel
+    const int32_t* myc = cidx + r * nch;   // this thread's ascending candidate run
     for (int m = mb + grp; m < mb + nb; m += 4) {
       const int pos = pos0 + m;
       const int col = m - mb;
@@ -248,42 +248,88 @@ __global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
         key[c] = 0;
         if (c < nch) tmem_ld_32x32b_x1(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c * 16 + col, key[c]);
       }
+      // usable candidates of this thread: the ascending prefix with 0 <= j < pos
+      int lo = 0, hi = nch;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int j = myc[mid];
+        if (j >= 0 && j < pos) lo = mid + 1;
+        else hi = mid;
+      }
+      const int nvt = lo;
       tmem_ld_wait();
-      // candidates of this thread usable by the member: an ascending prefix
-      int nvt = 0;
+      uint32_t kand = 0xFFFFFFFFu, kor = 0u;
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         reg_fence(key[c]);
         key[c] = score_key(__uint_as_float(key[c]));
-        nvt += (cand[c] >= 0 && cand[c] < pos) ? 1 : 0;
+        if (c < nvt) {
+          kand &= key[c];
+          kor |= key[c];
+        }
       }
-      int nv;
-      group_exclusive_scan(nvt, S.wsum, grp, quarter, lane, &nv);
+      // group totals: usable count, and which key bits vary across the member
+      {
+        const int wn = __reduce_add_sync(0xffffffffu, nvt);
+        const uint32_t wa = __reduce_and_sync(0xffffffffu, kand);
+        const uint32_t wo = __reduce_or_sync(0xffffffffu, kor);
+        if (lane == 0) {
+          S.wsum[quarter] = wn;
+          S.wand[quarter] = wa;
+          S.wor[quarter] = wo;
+        }
+        group_sync(grp);
+      }
+      const int nv = S.wsum[0] + S.wsum[1] + S.wsum[2] + S.wsum[3];
+      const uint32_t gand = S.wand[0] & S.wand[1] & S.wand[2] & S.wand[3];
+      const uint32_t gor = S.wor[0] | S.wor[1] | S.wor[2] | S.wor[3];
+      group_sync(grp);
       const int K = min(p.top_k, nv);
 
       // selection rule: take keys whose bits under `tmask` exceed `thr`, and
-      // those equal to it -- all of them, or (ties) the first `rank` in order
-      uint32_t thr = 0, tmask = 0;
+      // those equal to it -- all of them, or (ties) the first `rank` in order.
+      // Bits above the highest varying bit are common to every usable key.
+      int sh = 32 - __clz(gor ^ gand);
+      uint32_t tmask = sh >= 32 ? 0u : (0xFFFFFFFFu << sh);
+      uint32_t thr = gand & tmask;
       int rank = K;
-      bool ties = false;
+      bool ties = (sh == 0);
       if (K > 0 && K < nv) {
+        bool first = true;
 #pragma unroll 1
-        for (int ps = 0; ps < 3; ++ps) {
-          const int sh = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
-          const int nbn = ps == 2 ? 1024 : 2048;
+        while (sh > 0) {
+          const int width = sh >= 11 ? 11 : sh;
+          sh -= width;
+          const int nbn = 1 << width;
           for (int b = r; b < nbn; b += 128) S.hist[b] = 0;
           group_sync(grp);
+          if (first) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c < nvt && (key[c] & tmask) == thr) atomicAdd(&S.hist[(key[c] >> sh) & (nbn - 1)], 1);
+            for (int c = 0; c < 32; ++c)
+              if (c < nvt) atomicAdd(&S.hist[(key[c] >> sh) & (nbn - 1)], 1);
+          } else {
+            // only the few keys inside the current boundary bin take part
+            uint32_t mm = 0;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c < nvt && (key[c] & tmask) == thr) mm |= 1u << c;
+            if (mm) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if ((mm >> c) & 1u) atomicAdd(&S.hist[(key[c] >> sh) & (nbn - 1)], 1);
+            }
+          }
+          first = false;
           group_sync(grp);
-          // thread r owns bins [top - per + 1, top], scanned from the top
-          const int per = nbn / 128;
+          // thread r owns bins [top - per + 1, top]; the reads are rotated by r
+          // to keep the 32 lanes on different banks
+          const int per = nbn >= 128 ? nbn / 128 : 1;
           const int top = nbn - 1 - per * r;
           int s = 0;
-          for (int t = 0; t < per; ++t) s += S.hist[top - t];
-          const int excl = group_exclusive_scan(s, S.wsum, grp, quarter, lane, nullptr);
-          if (excl < rank && rank <= excl + s) {
+          if (top >= 0)
+            for (int t = 0; t < per; ++t) s += S.hist[top - ((t + r) & (per - 1))];
+          const int excl = group_exclusive_scan(s, S.wsum2, grp, quarter, lane, nullptr);
+          if (top >= 0 && excl < rank && rank <= excl + s) {
             int cum = excl;
             for (int t = 0; t < per; ++t) {
               const int cb = S.hist[top - t];
@@ -302,22 +348,24 @@ __global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
           rank -= S.above;
           const bool whole = (S.cntb == rank);
           group_sync(grp);
-          if (whole) break;             // every key of the boundary bin is taken
-          if (ps == 2) ties = true;     // equal keys, only `rank` of them are taken
+          if (whole) break;           // every key of the boundary bin is taken
+          if (sh == 0) ties = true;   // equal keys, only `rank` of them are taken
         }
       }
       // ---- selection flags and ordered emission
       uint32_t sel = 0;
       if (K > 0) {
-        if (!ties) {
+        if (K >= nv) {
+          sel = nvt >= 32 ? 0xFFFFFFFFu : ((1u << nvt) - 1u);
+        } else if (!ties) {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (c < nvt && (K >= nv || (key[c] & tmask) >= thr)) sel |= 1u << c;
+            if (c < nvt && (key[c] & tmask) >= thr) sel |= 1u << c;
         } else {
           int neq = 0;
 #pragma unroll
           for (int c = 0; c < 32; ++c) neq += (c < nvt && key[c] == thr) ? 1 : 0;
-          int eq_before = group_exclusive_scan(neq, S.wsum, grp, quarter, lane, nullptr);
+          int eq_before = group_exclusive_scan(neq, S.wsum2, grp, quarter, lane, nullptr);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             if (c < nvt) {
@@ -334,14 +382,13 @@ __global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
       int slot = group_exclusive_scan(__popc(sel), S.wsum2, grp, quarter, lane, nullptr);
       int32_t* orow = p.out + ((qrow0 + m) * p.H + h) * static_cast<long long>(p.top_k);
       float* srow = p.out_scores ? p.out_scores + ((qrow0 + m) * p.H + h) * static_cast<long long>(p.top_k) : nullptr;
+      if (srow) {
+        int sslot = slot;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        if ((sel >> c) & 1u) {
-          orow[slot] = cand[c];
-          if (srow) srow[slot] = key_score(key[c]);
-          ++slot;
-        }
+        for (int c = 0; c < 32; ++c)
+          if ((sel >> c) & 1u) srow[sslot++] = key_score(key[c]);
       }
+      for (uint32_t bits = sel; bits; bits &= bits - 1) orow[slot++] = myc[__ffs(bits) - 1];
       for (int t = K + r; t < p.top_k; t += 128) {
         orow[t] = -1;
         if (srow) srow[t] = __int_as_float(0x7fc00000);
