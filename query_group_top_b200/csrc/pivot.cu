@@ -244,11 +244,15 @@ int launch_scan(const CUtensorMap& tmP, const CUtensorMap& tmK, const ScanParams
 }
 
 template <int D>
-int launch_refine(const RefineParams& rp, int units, cudaStream_t st) {
+int launch_refine(RefineParams rp, int units, int sms, cudaStream_t st) {
   const int smem = RefineCfg<D>::smem_bytes(rp.Kc);
   CUDA_TRY(cudaFuncSetAttribute(refine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  rp.nbatch = (rp.g + 15) / 16;
+  rp.n_items = units * rp.nbatch;
+  // persistent: one CTA per SM walks the items
+  const int grid = std::max(1, std::min(rp.n_items, sms));
   TraceScope tr("refine", st);
-  refine_kernel<D><<<units, RefineCfg<D>::NT, smem, st>>>(rp);
+  refine_kernel<D><<<grid, RefineCfg<D>::NT, smem, st>>>(rp);
   CUDA_TRY(cudaGetLastError());
   return PIVOT_OK;
 }
@@ -362,7 +366,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.d = d;
     rp.tmem_cols = tmem_cols_for(Kc);
     rp.status = dev->status;
-    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, st) : launch_refine<64>(rp, H * pl.G, st);
+    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, dev->sms, st) : launch_refine<64>(rp, H * pl.G, dev->sms, st);
     if (rc) return rc;
   }
   return PIVOT_OK;
@@ -457,7 +461,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     rp.d = d;
     rp.tmem_cols = tmem_cols_for(Kc);
     rp.status = dev->status;
-    int rc = (d == 128) ? launch_refine<128>(rp, H * B, st) : launch_refine<64>(rp, H * B, st);
+    int rc = (d == 128) ? launch_refine<128>(rp, H * B, dev->sms, st) : launch_refine<64>(rp, H * B, dev->sms, st);
     if (rc) return rc;
   }
   return PIVOT_OK;

@@ -5,30 +5,42 @@
 // and then selects an individual top-k").  Member pos only keeps candidates
 // j < pos (causality).
 //
-// One CTA per (group, head), 16 warps.  With nc candidates and
-// nch = ceil(nc/128) chunks, chunk c's MMA row r holds candidate
-// t = r*nch + c, so TMEM lane r ends up with the contiguous, ascending block of
-// candidates [r*nch, r*nch + nch).  The keys are gathered 128 rows per chunk
-// with 16-byte cp.async into the 128-byte-swizzled K-major layout, and one
-// thread issues tcgen05.mma with M = 128 candidate rows, N = 16 member queries,
-// K = d; chunk c's scores land in TMEM columns [16c, 16c+16).  With Kc <= 4096
-// the whole candidates x members block (4096 x 16 fp32 = 256 KB) stays in TMEM.
+// Persistent, warp-specialised kernel: one CTA per SM walks the work items
+// (unit = (group, head), in batches of up to 16 members) with three roles
+// that run concurrently, so that one unit's selection overlaps the next
+// unit's gather and MMAs:
+//  * producers (warps 0-2) stage the unit's candidate list in shared memory
+//    and gather the candidate keys 128 rows per chunk with 16-byte cp.async
+//    into the 128-byte-swizzled K-major layout (plus the member queries as the
+//    B operand); a stage is handed over on an mbarrier once it has landed;
+//  * the MMA warp (warp 3) issues tcgen05.mma with M = 128 candidate rows,
+//    N = 16 member queries, K = d, into TMEM columns [16c, 16c+16) for chunk
+//    c, and signals "chunk c scored" on a per-chunk mbarrier;
+//  * the select warps (4-19, four per TMEM lane quarter; group grp of four
+//    warps owns members 4grp..4grp+3) select every member's exact top-k and
+//    write the rows.
+// Chunk c's MMA row r holds candidate t = r*nch + c, so TMEM lane r owns the
+// contiguous, ascending candidates [r*nch, r*nch + nch).  With Kc <= 4096 a
+// unit's scores (4096 x 16 fp32 = 256 KB) fill TMEM; the select warps give
+// each chunk's columns back as soon as they no longer need them, and the MMA
+// warp writes the next unit into them.
 //
 // Selection (exact, on 32-bit order keys, ties to the lower index):
-//  * Warp group grp (4 warps, one per TMEM lane quarter) owns members
-//    4grp..4grp+3, read with one 4-column TMEM load per chunk.
-//  * Round 0 runs inside the gather/MMA loop, two chunks behind the MMA: chunk
-//    0 is a 128-candidate sample spread over the whole set; its key range sets
-//    a linear 2048-bin histogram (monotone in the key, clamped at both ends),
-//    and every chunk is counted into it as soon as its scores exist.
-//  * After the loop, warp m finds member m's boundary bin with a two-level scan
-//    and inverts the bin function to key thresholds [kl, kh); one TMEM pass
-//    then marks each thread's candidates "above" (key >= kh) or "boundary".
-//  * A boundary of up to kListCap keys is ranked exactly from a shared list;
-//    larger boundaries are narrowed by further histogram rounds over their own
-//    key range, and a boundary of equal keys takes its first keys in order.
-//  * Output: one group scan gives every thread its output slot; each warp
-//    stages its slice of the row in shared memory and writes it coalesced.
+//  * round 0 follows the MMAs chunk by chunk: chunk 0 is a 128-candidate
+//    sample spread over the whole set; its score range sets a 512-bin
+//    histogram linear in the score (monotone, clamped at both ends), and
+//    every chunk is counted into it as soon as it is scored;
+//  * select warp w finds the boundary bin of member w with a two-level scan
+//    and inverts the bin function to key thresholds [kl, kh); one pass over
+//    the scores marks each candidate "above" (key >= kh) or "boundary" and
+//    collects the boundary keys in a shared list, after which the unit's TMEM
+//    columns are given back;
+//  * a list of up to kListCap keys is ranked exactly (the need-th largest key
+//    tk, and how many of its copies are taken) and its decisions go to
+//    per-member bitmaps; larger boundaries are narrowed by further key-linear
+//    rounds, and a boundary of equal keys takes its first keys in order;
+//  * one group scan gives every thread its output slot; each warp stages its
+//    slice of an output row in shared memory and writes it coalesced.
 #pragma once
 
 #include "ptx.cuh"
@@ -43,6 +55,8 @@ struct RefineParams {
   float* out_scores;      // same shape as out, or null
   const int32_t* cu;      // decode: [B+1] cache row offsets; null for prefill
   int G, L, H, g, top_k, Kc, d;
+  int n_items;            // H * G units x member batches
+  int nbatch;             // member batches of up to 16 per unit
   uint32_t tmem_cols;
   int* status;
 };
@@ -53,12 +67,12 @@ enum : int {
   kMAll = 1,     // takes every usable candidate (top_k >= usable count)
   kMSel = 2,     // narrowing: the boundary bin of the current round is open
   kMWhole = 3,   // every key of the boundary bin is taken
-  kMList = 4,    // boundary ranked from the shared list: (tk, need_eq) known
+  kMList = 4,    // boundary ranked from the shared list
   kMNarrow = 5,  // boundary too large for the list: another round
   kMTies = 6,    // boundary keys all equal: the first need_eq in order
 };
 
-constexpr int kRefBins = 2048;
+constexpr int kRefBins = 512;
 constexpr int kListCap = 256;
 
 struct MemberSel {
@@ -68,8 +82,8 @@ struct MemberSel {
   int active;       // takes part in the current round
   int need;         // keys still to take from the current candidate interval
   int cnt;          // keys in the boundary bin
-  uint32_t lo;      // bin function: origin (a key, or a score's bits) and scale
-  float scale;
+  uint32_t lo;      // key-linear bins: origin; both: scale; score-linear: offset
+  float scale, off;
   int vmode;        // bins linear in the score (1) or in the order key (0)
   uint32_t kl, kh;  // boundary bin = keys in [kl, kh); kh_inf: no upper edge
   int kh_inf;
@@ -83,7 +97,8 @@ struct RefineMisc {
   MemberSel ms[16];
   uint32_t pmin[4][16], pmax[4][16];
   int gscan[4][4][8];
-  uint64_t bars[8];
+  uint64_t full[4], empty[4], cready[2], cfree[2], drain;
+  uint64_t tready[32], tfree[32];
   uint32_t tmem_slot;
   int abort_flag;
   int more;
@@ -91,71 +106,94 @@ struct RefineMisc {
 
 template <int D>
 struct RefineCfg {
-  static constexpr int NT = 512;
+  static constexpr int NPROD = 96;                      // producer threads (warps 0-2)
+  static constexpr int MMA_WARP = 3;
+  static constexpr int SEL_WARP0 = 4;                   // select warps 4-19
+  static constexpr int NSEL = 512;
+  static constexpr int NT = 640;
   static constexpr int NS = 4;                          // gather stages
-  static constexpr int LA = 2;                          // chunks in flight ahead of the MMA
-  static_assert(NS == LA + 2, "stage reuse and score reads both trail the MMA by two chunks");
+  static constexpr int LA = 3;                          // chunks in flight before a stage is handed over
+  static_assert(LA <= NS - 1, "a stage is handed over before its producer waits for it again");
   static constexpr int KATOMS = D / 64;
   static constexpr int ATOM_A = 128 * 128;              // 128 rows x 128 bytes
   static constexpr int STAGE = KATOMS * ATOM_A;
   static constexpr int ATOM_B = 16 * 128;               // 16 member rows x 128 bytes
+  static constexpr int B_BYTES = ((KATOMS * ATOM_B + 1023) / 1024) * 1024;
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = NS * STAGE;
-  static constexpr int OFF_C = OFF_B + ((KATOMS * ATOM_B + 1023) / 1024) * 1024;
-  // histograms: 16 members x 2048 bins of 16-bit counts (two per word); the
-  // same bytes later hold the boundary lists and the per-warp output staging
-  static constexpr int HIST_BYTES = 16 * (kRefBins / 2) * 4;
+  static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
+  static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
+  // histograms: 16 members x 512 bins of 32-bit counts; the same bytes later
+  // hold the boundary lists and the per-warp output staging
+  static constexpr int HIST_BYTES = 16 * kRefBins * 4;
   static_assert(16 * 2 * kListCap * 4 <= HIST_BYTES, "lists alias the histograms");
-  static_assert(16 * 1024 * 4 <= HIST_BYTES, "output staging aliases the histograms");
-  // candidate indices are staged for whole 128-row chunks (-1 past the set)
-  __host__ __device__ static int cidx_bytes(int Kc) { return ((Kc + 127) / 128) * 128 * 4; }
+  static constexpr int STG = 512;                       // output staging entries per select warp
+  static_assert(16 * STG * 4 <= HIST_BYTES, "output staging aliases the histograms");
+  __host__ __device__ static int nch_max(int Kc) { return (Kc + 127) / 128; }
+  __host__ __device__ static int cidx_words(int Kc) { return nch_max(Kc) * 128; }
+  // list decisions: per member, "above" and "equal" bitmaps over candidates
+  __host__ __device__ static int bm_words(int Kc) { return nch_max(Kc) * 4; }
   static int smem_bytes(int Kc) {
-    return OFF_C + cidx_bytes(Kc) + HIST_BYTES + static_cast<int>(sizeof(RefineMisc)) + 1024;
+    return OFF_C + 2 * cidx_words(Kc) * 4 + HIST_BYTES + 16 * 2 * bm_words(Kc) * 4 +
+           static_cast<int>(sizeof(RefineMisc)) + 1024;
   }
 };
 
 // Linear bin of an order key over [lo, ...) with `scale` bins per key unit,
-// clamped to [0, 2047].  Every step (difference, conversion, product,
-// truncation, clamp) is non-decreasing in the key, so the bins are ordered
-// like the keys and equal keys share a bin.
+// clamped to [0, 511].  Every step is non-decreasing in the key.
 __device__ __forceinline__ int key_bin(uint32_t key, uint32_t lo, float scale) {
   const uint32_t dl = key > lo ? key - lo : 0u;
   const uint32_t b = __float2uint_rz(__uint2float_rn(dl) * scale);
   return static_cast<int>(min(b, static_cast<uint32_t>(kRefBins - 1)));
 }
 
-// Linear bin of a score over [lo, ...), clamped to [0, 2047]; explicit
-// roundings keep every step non-decreasing in the score, and -0 and +0 share
-// a bin.  Scores of real data spread evenly over such bins, while order keys
-// of scores on both sides of zero crowd into a few of the key-linear ones.
-__device__ __forceinline__ int value_bin(float s, float lo, float scale) {
-  const float x = __fmul_rn(__fsub_rn(s, lo), scale);
-  return min(max(__float2int_rz(x), 0), kRefBins - 1);
+// Linear bin of a score, trunc(s * scale + off) clamped to [0, 511]: one
+// rounding (the fma) of a function increasing in s, so the bins are ordered
+// like the scores, and -0 and +0 share a bin.  Scores of real data spread
+// evenly over such bins, while the order keys of scores on both sides of zero
+// crowd into a few of the key-linear ones.
+__device__ __forceinline__ int value_bin(float s, float scale, float off) {
+  return static_cast<int>(min(__float2uint_rz(__fmaf_rn(s, scale, off)), static_cast<uint32_t>(kRefBins - 1)));
 }
 
 // Bin of an order key under either bin function; key patterns beyond the
 // infinities (no score has them) clamp to the infinities.
-__device__ __forceinline__ int bin_of_key(uint32_t key, uint32_t lo, float scale, bool vmode) {
+__device__ __forceinline__ int bin_of_key(uint32_t key, uint32_t lo, float scale, float off, bool vmode) {
   if (!vmode) return key_bin(key, lo, scale);
   const uint32_t kc = min(max(key, 0x007FFFFFu), 0xFF800000u);
-  return value_bin(key_score(kc), __uint_as_float(lo), scale);
+  return value_bin(key_score(kc), scale, off);
 }
 
-// Smallest key whose bin is >= b (1 <= b <= 2047), searched by the whole warp
-// 32 ways at a time; false when no key reaches bin b.
-__device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float scale, bool vmode, int lane,
-                                                      uint32_t* out) {
-  if (bin_of_key(0xFFFFFFFFu, lo, scale, vmode) < b) return false;
+// Smallest key whose bin is >= b (1 <= b <= 511), found by the whole warp;
+// false when no key reaches bin b.  A 32-key probe around the bin's nominal
+// edge usually brackets it; otherwise a 32-way search over all keys does.
+__device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float scale, float off, bool vmode,
+                                                      int lane, uint32_t* out) {
+  if (bin_of_key(0xFFFFFFFFu, lo, scale, off, vmode) < b) return false;
+  uint32_t guess;
+  if (vmode) {
+    guess = score_key(__fdiv_rn(__fsub_rn(static_cast<float>(b), off), scale));
+  } else {
+    const float dk = __fdiv_rn(static_cast<float>(b), scale);
+    guess = dk >= 4294967040.0f ? 0xFFFFFFFFu : lo + min(__float2uint_rz(dk), 0xFFFFFFFFu - lo);
+  }
+  const long long p0 = static_cast<long long>(guess) - 16;
+  const long long pk = min(max(p0 + lane, 0ll), 4294967295ll);
+  const unsigned ge =
+      __ballot_sync(0xffffffffu, bin_of_key(static_cast<uint32_t>(pk), lo, scale, off, vmode) >= b);
+  if ((ge & 1u) == 0u && (ge >> 31) != 0u && p0 >= 0 && p0 + 31 <= 4294967295ll) {
+    *out = static_cast<uint32_t>(p0 + __ffs(ge) - 1);
+    return true;
+  }
   unsigned long long base = 0, span = 1ull << 32;
   while (span > 1) {
     const unsigned long long stride = (span + 31) / 32;
     const unsigned long long first = base + static_cast<unsigned long long>(lane) * stride;
-    bool ge = true;  // empty sub-ranges count as "beyond"
+    bool g = true;  // empty sub-ranges count as "beyond"
     if (first < base + span) {
       const unsigned long long last = min(first + stride, base + span) - 1;
-      ge = bin_of_key(static_cast<uint32_t>(last), lo, scale, vmode) >= b;
+      g = bin_of_key(static_cast<uint32_t>(last), lo, scale, off, vmode) >= b;
     }
-    const int j = __ffs(__ballot_sync(0xffffffffu, ge)) - 1;
+    const int j = __ffs(__ballot_sync(0xffffffffu, g)) - 1;
     const unsigned long long nb = base + static_cast<unsigned long long>(j) * stride;
     span = min(stride, base + span - nb);
     base = nb;
@@ -164,668 +202,788 @@ __device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float 
   return true;
 }
 
-__device__ __forceinline__ void group_sync(int grp) { named_barrier(1 + grp, 128); }
+// One work item: a unit's batch of up to 16 members.
+struct RefineItem {
+  int h, u, mb, nb, pos0, nc, nch;
+  long long key_row0;   // cache row of key index 0
+  long long qrow0;      // row (before *H) of member 0's query and output
+};
+
+__device__ __forceinline__ RefineItem refine_item(const RefineParams& p, int item) {
+  RefineItem it;
+  const int ui = item / p.nbatch;
+  it.mb = (item - ui * p.nbatch) * 16;
+  it.h = ui / p.G;
+  it.u = ui - it.h * p.G;
+  int nm;
+  if (p.cu == nullptr) {
+    const int s = it.u * p.g;
+    nm = min(s + p.g, p.L) - s;
+    it.pos0 = s;
+    it.key_row0 = 0;
+    it.qrow0 = s;
+  } else {
+    nm = p.g;
+    it.key_row0 = p.cu[it.u];
+    it.pos0 = p.cu[it.u + 1] - p.cu[it.u] - p.g;
+    it.qrow0 = static_cast<long long>(it.u) * p.g;
+  }
+  it.nb = min(16, nm - it.mb);
+  const int last = it.pos0 + nm - 1;
+  it.nc = min(p.Kc, max(last, 0));
+  it.nch = (it.nc + 127) / 128;
+  return it;
+}
+
+// candidate t = r*nch + c of a list lives at word c*128 + ((r + c) & 127):
+// conflict-free both along a chunk (fixed c) and along a thread's block (fixed r)
+__device__ __forceinline__ int cidx_pos(int c, int r) { return c * 128 + ((r + c) & 127); }
 
 template <int D>
-__global__ void __launch_bounds__(512, 1) refine_kernel(RefineParams p) {
+__global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   using C = RefineCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sA = sbase + C::OFF_A;
   const uint32_t sB = sbase + C::OFF_B;
-  int32_t* cidx = reinterpret_cast<int32_t*>(smem + C::OFF_C);
-  const int off_h = C::OFF_C + C::cidx_bytes(p.Kc);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + off_h);
-  RefineMisc* M = reinterpret_cast<RefineMisc*>(smem + off_h + C::HIST_BYTES);
+  const int NCH = C::nch_max(p.Kc);
+  const int CW = C::cidx_words(p.Kc);
+  const int BMW = C::bm_words(p.Kc);
+  int32_t* cidx0 = reinterpret_cast<int32_t*>(smem + C::OFF_C);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::OFF_C + 2 * CW * 4);
+  uint32_t* bmap = hist + C::HIST_BYTES / 4;          // [16][2][BMW]
+  RefineMisc* M = reinterpret_cast<RefineMisc*>(bmap + 16 * 2 * BMW);
   volatile int* abort_flag = &M->abort_flag;
-  const uint32_t bar0 = smem_u32(&M->bars[0]);
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int grp = warp >> 2, quarter = warp & 3;
-  const int r = quarter * 32 + lane;  // TMEM lane: this thread's candidate block
-  const int h = blockIdx.x / p.G, u = blockIdx.x % p.G;
-
-  // ---- the unit: members, their positions, where keys and outputs live
-  int nm, pos0;
-  long long key_row0 = 0;      // cache row of key index 0
-  long long qrow0;             // row (before *H) of member 0's query and output
-  if (p.cu == nullptr) {
-    const int s = u * p.g;
-    nm = min(s + p.g, p.L) - s;
-    pos0 = s;
-    qrow0 = s;
-  } else {
-    nm = p.g;
-    key_row0 = p.cu[u];
-    pos0 = p.cu[u + 1] - p.cu[u] - p.g;
-    qrow0 = static_cast<long long>(u) * p.g;
-  }
-  const int last = pos0 + nm - 1;
-  const int nc = min(p.Kc, max(last, 0));
-  const int nch = (nc + 127) / 128;
 
   if (tid == 0) {
-    for (int s = 0; s < C::NS; ++s) mbar_init(bar0 + 8u * s, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(smem_u32(&M->full[s]), C::NPROD);
+      mbar_init(smem_u32(&M->empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&M->cready[b]), C::NPROD);
+      mbar_init(smem_u32(&M->cfree[b]), C::NSEL / 32);
+    }
+    for (int c = 0; c < 32; ++c) {
+      mbar_init(smem_u32(&M->tready[c]), 1);
+      mbar_init(smem_u32(&M->tfree[c]), C::NSEL / 32);
+    }
+    mbar_init(smem_u32(&M->drain), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(&M->tmem_slot), p.tmem_cols);
     tmem_relinquish();
   }
-  // candidate t = r*nch + c lives at cidx[c*128 + ((r + c) & 127)]: conflict-free
-  // both along a chunk (fixed c) and along a thread's block (fixed r)
-  const int32_t* crow = p.cand + (static_cast<long long>(h) * p.G + u) * p.Kc;
-  for (int t = tid; t < nch * 128; t += C::NT) {
-    const int rr = t / nch, c = t - rr * nch;
-    cidx[c * 128 + ((rr + c) & 127)] = (t < nc) ? crow[t] : -1;
-  }
-  auto cand_at = [&](int c, int rr) -> int { return cidx[c * 128 + ((rr + c) & 127)]; };
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = M->tmem_slot;
-  const uint32_t tlane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 
-  const uint16_t* kbase = p.keys + (key_row0 * p.H + h) * static_cast<long long>(D);
-  // chunk c, MMA row r  <->  candidate r*nch + c
-  auto issue_gather = [&](int c, int stage) {
-    const uint32_t dst0 = sA + stage * C::STAGE;
-#pragma unroll
-    for (int it = 0; it < (128 * D / 8) / C::NT; ++it) {
-      const int id = tid + it * C::NT;
-      const int rr = id / (D / 8), piece = id % (D / 8);
-      const int a = piece >> 3, p8 = piece & 7;
-      const int j = cand_at(c, rr);
-      const uint16_t* src = kbase + (j >= 0 ? static_cast<long long>(j) * p.H * D : 0) + piece * 8;
-      const uint32_t dst = dst0 + a * C::ATOM_A + rr * 128 + ((p8 ^ (rr & 7)) << 4);
-      cp_async_16(dst, src, j >= 0 ? 16u : 0u);
-    }
-  };
-
-  constexpr uint32_t idesc = umma_idesc_bf16(128, 16);
-  int seq = 0;           // chunks issued so far (all member batches), drives stage/parity
-  int last_commit = -1;  // thread 0: last chunk whose MMAs were committed
-  bool ok = true;
-
-  for (int mb = 0; mb < nm && ok; mb += 16) {
-    const int nb = min(16, nm - mb);
-    // ---- member queries -> B operand (16 rows, swizzled), zero rows past nb
-    for (int id = tid; id < 16 * (D / 8); id += C::NT) {
-      const int rr = id / (D / 8), piece = id % (D / 8);
-      const int a = piece >> 3, p8 = piece & 7;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (rr < nb)
-        v = *reinterpret_cast<const uint4*>(p.q + ((qrow0 + mb + rr) * p.H + h) * static_cast<long long>(D) +
-                                            piece * 8);
-      *reinterpret_cast<uint4*>(smem + C::OFF_B + a * C::ATOM_B + rr * 128 + ((p8 ^ (rr & 7)) << 4)) = v;
-    }
-    // ---- per-member usable counts (the candidate set is ascending) and modes
-    if (tid < 16) {
-      MemberSel& S = M->ms[tid];
-      int nv = 0;
-      if (tid < nb) {
-        const int pos = pos0 + mb + tid;
-        int lo = 0, hi = nc;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          const int q8 = mid / max(nch, 1);
-          if (cand_at(mid - q8 * nch, q8) < pos) lo = mid + 1;
-          else hi = mid;
-        }
-        nv = lo;
+  if (warp < C::MMA_WARP) {
+    // ======================================================== producers
+    const int pt = tid;
+    int sseq = 0;     // chunks issued so far (all items)
+    int handed = 0;   // chunks handed over to the MMA warp so far
+    int kk = 0;       // items processed so far
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+      const RefineItem it = refine_item(p, item);
+      if (it.nb <= 0) continue;
+      const int buf = kk & 1;
+      int32_t* cx = cidx0 + buf * CW;
+      // hand over what is still in flight before the next list is read
+      if (handed < sseq) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        for (; handed < sseq; ++handed) mbar_arrive(smem_u32(&M->full[handed % C::NS]));
       }
-      const int K = min(p.top_k, nv);
-      S.nv = nv;
-      S.K = K;
-      S.mode = K == 0 ? kMNone : (K == nv ? kMAll : kMSel);
-      S.active = S.mode == kMSel;
-      S.need = K;
-      S.cnt = nv;
-      S.nlist = 0;
-      S.bmin = 0xFFFFFFFFu;
-      S.bmax = 0u;
-      S.need_eq = 0;
-      S.tk = 0;
-      S.vmode = 0;
-    }
-    for (int i = tid; i < C::HIST_BYTES / 16; i += C::NT) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
-    __syncthreads();
-
-    // this thread's view of its four members (member 4*grp + i of the batch)
-    uint32_t um[4];       // usable chunks of this thread's block
-    uint32_t hm = 0;      // members counted in the round-0 histogram
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const MemberSel& S = M->ms[4 * grp + i];
-      const int nvt = min(max(S.nv - r * nch, 0), nch);
-      um[i] = nvt >= 32 ? 0xFFFFFFFFu : ((1u << nvt) - 1u);
-      hm |= (S.mode == kMSel ? 1u : 0u) << i;
-    }
-    uint32_t lo4[4] = {0, 0, 0, 0};
-    float sc4[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t vm4 = 0;     // members whose round-0 bins are linear in the score
-
-    // round 0, chunk 0: the sample's key range, per lane quarter
-    auto sample_range = [&]() {
-      uint32_t v[4];
-      tmem_ld_32x32b_x4(tlane + 4 * grp, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        reg_fence(v[i]);
-        const bool use = ((hm >> i) & 1u) && (um[i] & 1u);
-        const uint32_t key = score_key(__uint_as_float(v[i]));
-        const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
-        const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
-        if (lane == 0) {
-          M->pmin[quarter][4 * grp + i] = mn;
-          M->pmax[quarter][4 * grp + i] = mx;
-        }
-      }
-    };
-    // bins over the sample's range (every thread of the group computes the same)
-    auto set_range = [&]() {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = 4 * grp + i;
-        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          mn = min(mn, M->pmin[qq][m]);
-          mx = max(mx, M->pmax[qq][m]);
-        }
-        const float vmin = key_score(mn), vmax = key_score(mx);
-        const float vsc = static_cast<float>(kRefBins) / __fsub_rn(vmax, vmin);
-        const bool vm = mn < mx && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f;
-        if (vm) {
-          lo4[i] = __float_as_uint(vmin);
-          sc4[i] = vsc;
-          vm4 |= 1u << i;
-        } else if (mn > mx) {
-          lo4[i] = 0u;
-          sc4[i] = 0.f;
-        } else {
-          lo4[i] = mn;
-          sc4[i] = static_cast<float>(kRefBins) / (__uint2float_rn(mx - mn) + 1.0f);
-        }
-        if (quarter == 0 && lane == 0) {
-          M->ms[m].lo = lo4[i];
-          M->ms[m].scale = sc4[i];
-          M->ms[m].vmode = vm ? 1 : 0;
-        }
-      }
-    };
-    auto hist_chunk = [&](int c) {
-      uint32_t v[4];
-      tmem_ld_32x32b_x4(tlane + c * 16 + 4 * grp, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        reg_fence(v[i]);
-        if (((hm >> i) & 1u) && ((um[i] >> c) & 1u)) {
-          const float f = __uint_as_float(v[i]);
-          const int b = ((vm4 >> i) & 1u) ? value_bin(f, __uint_as_float(lo4[i]), sc4[i])
-                                          : key_bin(score_key(f), lo4[i], sc4[i]);
-          atomicAdd(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)], 1u << ((b & 1) * 16));
-        }
-      }
-    };
-    auto process_chunk = [&](int c) {
-      if (hm == 0) return;
-      if (c == 0) {
-        sample_range();
-      } else {
-        if (c == 1) {
-          set_range();
-          hist_chunk(0);
-        }
-        hist_chunk(c);
-      }
-    };
-
-    // ---- gather + MMA pipeline over candidate chunks, round-0 histogram two
-    //      chunks behind the MMA
-    const int seq0 = seq;
-    // always LA groups in the prologue, so that wait_group<LA> below means
-    // "chunk c has landed" whatever nch is
-    for (int c = 0; c < C::LA; ++c) {
-      if (c < nch) issue_gather(c, (seq0 + c) % C::NS);
-      cp_async_commit();
-    }
-    for (int c = 0; c < nch; ++c) {
-      if (c >= 2) {
-        // chunk c-2's MMAs are done: its stage may be refilled (with chunk
-        // c + LA) and its scores read
-        const int pv = seq0 + c - 2;
-        if (ok && !mbar_wait(bar0 + 8u * (pv % C::NS), (pv / C::NS) & 1, abort_flag, p.status)) ok = false;
-      }
-      const int cn = c + C::LA;
-      if (ok && cn < nch) issue_gather(cn, (seq0 + cn) % C::NS);
-      cp_async_commit();
-      if (c >= 2) {
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-          tc_fence_after();
-          process_chunk(c - 2);
-        }
-      }
-      cp_async_wait<C::LA>();
-      fence_proxy_async_smem();
-      if (__syncthreads_or(!ok)) {
-        ok = false;
-        break;
-      }
-      if (tid == 0) {
-        tc_fence_after();
-        const int st = (seq0 + c) % C::NS;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int a = kk >> 2, k4 = kk & 3;
-          const uint64_t adesc = sw128_kmajor_desc(sA + st * C::STAGE + a * C::ATOM_A + k4 * 32);
-          const uint64_t bdesc = sw128_kmajor_desc(sB + a * C::ATOM_B + k4 * 32);
-          umma_bf16(tmem + c * 16, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar0 + 8u * st);
-        last_commit = seq0 + c;
-      }
-    }
-    cp_async_wait<0>();
-    seq = seq0 + nch;
-    if (!ok) break;
-    for (int pp = max(0, nch - 2); pp < nch; ++pp) {
-      const int pv = seq0 + pp;
-      if (ok && !mbar_wait(bar0 + 8u * (pv % C::NS), (pv / C::NS) & 1, abort_flag, p.status)) ok = false;
-      ok = __all_sync(0xffffffffu, ok);
+      if (kk >= 2 && ok)
+        ok = mbar_wait(smem_u32(&M->cfree[buf]), ((kk >> 1) - 1) & 1, abort_flag, p.status, 256);
       if (ok) {
-        tc_fence_after();
-        process_chunk(pp);
+        // the unit's candidate list, transposed on the fly; all copies in flight at once
+        const int32_t* crow = p.cand + (static_cast<long long>(it.h) * p.G + it.u) * p.Kc;
+        for (int t = pt; t < it.nch * 128; t += C::NPROD) {
+          const int rr = t / it.nch, c = t - rr * it.nch;
+          if (t < it.nc) cp_async_4(smem_u32(cx + cidx_pos(c, rr)), crow + t);
+          else cx[cidx_pos(c, rr)] = -1;
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
       }
-      if (pp == 0 && __syncthreads_or(!ok)) ok = false;  // the sample ranges are visible
-    }
-    if (ok && nch == 1 && hm != 0) {
-      set_range();
-      hist_chunk(0);
-    }
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
-    }
-
-    // ---- selection rounds
-    uint32_t gt[4] = {0, 0, 0, 0};   // taken: above the boundary
-    uint32_t bnd[4] = {0, 0, 0, 0};  // in the current boundary bin
+      named_barrier(1, C::NPROD);
+      mbar_arrive(smem_u32(&M->cready[buf]));
+      // this thread copies the 16-byte pieces p8, p8 + 8, ... (one per K atom,
+      // same swizzle) of rows rr0, rr0 + RSTEP, ...
+      constexpr int RSTEP = C::NPROD / 8;
+      const int p8 = pt & 7, rr0 = pt >> 3;
+      const long long rowstride = static_cast<long long>(p.H) * D;
+      const uint16_t* kbase = p.keys + (it.key_row0 * p.H + it.h) * static_cast<long long>(D) + p8 * 8;
+      const uint32_t bB = sB + buf * C::B_BYTES;
+      for (int c = 0; c < it.nch; ++c) {
+        const int s = sseq % C::NS;
+        // one warp watches the stage; the others sleep on the named barrier
+        if (sseq >= C::NS && ok && warp == 0)
+          ok = mbar_wait(smem_u32(&M->empty[s]), ((sseq / C::NS) - 1) & 1, abort_flag, p.status, 256);
+        ok = !named_barrier_or(1, C::NPROD, !ok);
+        if (ok) {
+          const uint32_t dst0 = sA + s * C::STAGE;
+          const int32_t* cxc = cx + c * 128;
+          for (int rr = rr0; rr < 128; rr += RSTEP) {
+            const int j = cxc[(rr + c) & 127];
+            const uint16_t* src = kbase + max(j, 0) * rowstride;
+            const uint32_t dst = dst0 + rr * 128 + ((p8 ^ (rr & 7)) << 4);
+            const uint32_t nbytes = j >= 0 ? 16u : 0u;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (M->ms[4 * grp + i].mode == kMAll) gt[i] = um[i];
-
-#pragma unroll 1
-    for (int round = 0;; ++round) {
-      // (a) warp m: member m's boundary bin and its key thresholds
-      if (warp < nb && M->ms[warp].active) {
-        MemberSel& S = M->ms[warp];
-        const uint32_t* hw = hist + warp * (kRefBins / 2);
-        const int need = S.need;
-        // lane l owns words [1024 - 32(l+1), 1024 - 32l): bins in descending order
-        const int w0 = kRefBins / 2 - 32 * (lane + 1);
-        int s = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 x = reinterpret_cast<const uint4*>(hw + w0)[(i + lane) & 7];
-          s += (x.x & 0xFFFFu) + (x.x >> 16) + (x.y & 0xFFFFu) + (x.y >> 16) + (x.z & 0xFFFFu) + (x.z >> 16) +
-               (x.w & 0xFFFFu) + (x.w >> 16);
-        }
-        int incl = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const int L = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;
-        const int exclL = __shfl_sync(0xffffffffu, incl - s, L);
-        // lane i: word (1024 - 32L - 1 - i), holding bins 2w+1 (upper half) and 2w
-        const int w = kRefBins / 2 - 32 * L - 1 - lane;
-        const uint32_t wv = hw[w];
-        const int chi = static_cast<int>(wv >> 16), clo = static_cast<int>(wv & 0xFFFFu);
-        const int s2 = chi + clo;
-        int incl2 = s2;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl2, o);
-          if (lane >= o) incl2 += y;
-        }
-        const int i2 = __ffs(__ballot_sync(0xffffffffu, exclL + incl2 >= need)) - 1;
-        int bstar = 0, above = 0, cntb = 0;
-        if (lane == i2) {
-          const int before = exclL + incl2 - s2;
-          if (before + chi >= need) {
-            bstar = 2 * w + 1;
-            above = before;
-            cntb = chi;
-          } else {
-            bstar = 2 * w;
-            above = before + chi;
-            cntb = clo;
+            for (int a = 0; a < C::KATOMS; ++a) cp_async_16(dst + a * C::ATOM_A, src + a * 64, nbytes);
+          }
+          if (c == 0) {
+            // member queries of this batch -> B operand, zero rows past nb
+            for (int id = pt; id < 16 * (D / 8); id += C::NPROD) {
+              const int rr = id / (D / 8), piece = id % (D / 8);
+              const int a = piece >> 3, p8 = piece & 7;
+              const bool real = rr < it.nb;
+              const uint16_t* src =
+                  p.q + (real ? ((it.qrow0 + it.mb + rr) * p.H + it.h) * static_cast<long long>(D) + piece * 8 : 0);
+              cp_async_16(bB + a * C::ATOM_B + rr * 128 + ((p8 ^ (rr & 7)) << 4), src, real ? 16u : 0u);
+            }
           }
         }
-        bstar = __shfl_sync(0xffffffffu, bstar, i2);
-        above = __shfl_sync(0xffffffffu, above, i2);
-        cntb = __shfl_sync(0xffffffffu, cntb, i2);
-        const uint32_t lo = S.lo;
-        const float sc = S.scale;
-        const bool vm = S.vmode != 0;
-        uint32_t kl = 0, kh = 0;
-        bool has_kl = true, has_kh = false;
-        if (bstar > 0) has_kl = warp_first_key_of_bin(bstar, lo, sc, vm, lane, &kl);
-        if (bstar < kRefBins - 1) has_kh = warp_first_key_of_bin(bstar + 1, lo, sc, vm, lane, &kh);
-        if (lane == 0) {
-          const int need2 = need - above;
-          S.need = need2;
-          S.cnt = cntb;
-          S.kl = has_kl ? kl : 0u;
-          S.kh = kh;
-          S.kh_inf = has_kh ? 0 : 1;
-          S.mode = (cntb == need2) ? kMWhole : (cntb <= kListCap ? kMList : kMNarrow);
-          S.nlist = 0;
-          S.bmin = 0xFFFFFFFFu;
-          S.bmax = 0u;
+        cp_async_commit();
+        ++sseq;
+        if (sseq - handed > C::LA) {
+          // the oldest chunk in flight has landed: hand its stage over
+          cp_async_wait<C::LA>();
+          fence_proxy_async_smem();
+          mbar_arrive(smem_u32(&M->full[handed % C::NS]));
+          ++handed;
         }
       }
-      __syncthreads();
+      ++kk;
+      if (named_barrier_or(1, C::NPROD, !ok)) break;
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    for (; handed < sseq; ++handed) mbar_arrive(smem_u32(&M->full[handed % C::NS]));
+  } else if (warp == C::MMA_WARP) {
+    // ======================================================== MMA issuer
+    constexpr uint32_t idesc = umma_idesc_bf16(128, 16);
+    int sseq = 0, kk = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const RefineItem it = refine_item(p, item);
+      if (it.nb <= 0) continue;
+      const uint32_t bB = sB + (kk & 1) * C::B_BYTES;
+      for (int c = 0; c < NCH && ok; ++c) {
+        // the previous item's select warps are done with these columns
+        if (kk >= 1) ok = mbar_wait(smem_u32(&M->tfree[c]), (kk - 1) & 1, abort_flag, p.status, 128);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && c < it.nch) {
+          const int s = sseq % C::NS;
+          ok = mbar_wait(smem_u32(&M->full[s]), (sseq / C::NS) & 1, abort_flag, p.status, 64);
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok && lane == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kq = 0; kq < D / 16; ++kq) {
+              const int a = kq >> 2, k4 = kq & 3;
+              const uint64_t adesc = sw128_kmajor_desc(sA + s * C::STAGE + a * C::ATOM_A + k4 * 32);
+              const uint64_t bdesc = sw128_kmajor_desc(bB + a * C::ATOM_B + k4 * 32);
+              umma_bf16(tmem + c * 16, adesc, bdesc, idesc, kq > 0 ? 1u : 0u);
+            }
+            umma_commit(smem_u32(&M->empty[s]));
+          }
+          ++sseq;
+        }
+        if (ok && lane == 0) umma_commit(smem_u32(&M->tready[c]));
+        __syncwarp();
+      }
+      ++kk;
+    }
+    // every MMA issued has finished before TMEM can be freed
+    if (lane == 0) {
+      umma_commit(smem_u32(&M->drain));
+      mbar_wait_cleanup(smem_u32(&M->drain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ======================================================== select
+    const int sw = warp - C::SEL_WARP0;   // 0..15: also the member whose bins this warp scans
+    const int grp = sw >> 2;              // member group: members 4grp..4grp+3
+    const int quarter = warp & 3;         // TMEM lane quarter
+    const int r = quarter * 32 + lane;    // this thread's candidate block
+    const int stid = sw * 32 + lane;      // 0..511
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 4 * grp;
+    auto sel_sync = [&]() { named_barrier(2, C::NSEL); };
+    int kk = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+      const RefineItem it = refine_item(p, item);
+      if (it.nb <= 0) continue;
+      const int buf = kk & 1;
+      const int nch = it.nch, nb = it.nb;
+      const int32_t* cx = cidx0 + buf * CW;
+      if (ok) ok = mbar_wait(smem_u32(&M->cready[buf]), (kk >> 1) & 1, abort_flag, p.status, 256);
+      // ---- per-member usable counts (the candidate set is ascending) and modes
+      if (stid < 16 && ok) {
+        MemberSel& S = M->ms[stid];
+        int nv = 0;
+        if (stid < nb) {
+          const int pos = it.pos0 + it.mb + stid;
+          int lo = 0, hi = it.nc;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            const int rr = mid / nch;
+            if (cx[cidx_pos(mid - rr * nch, rr)] < pos) lo = mid + 1;
+            else hi = mid;
+          }
+          nv = lo;
+        }
+        const int K = min(p.top_k, nv);
+        S.nv = nv;
+        S.K = K;
+        S.mode = K == 0 ? kMNone : (K == nv ? kMAll : kMSel);
+        S.active = S.mode == kMSel;
+        S.need = K;
+        S.cnt = nv;
+        S.nlist = 0;
+        S.bmin = 0xFFFFFFFFu;
+        S.bmax = 0u;
+        S.need_eq = 0;
+        S.tk = 0;
+        S.vmode = 0;
+        S.off = 0.f;
+      }
+      for (int i = stid; i < C::HIST_BYTES / 16; i += C::NSEL) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+      for (int i = stid; i < 16 * 2 * BMW / 4; i += C::NSEL) reinterpret_cast<uint4*>(bmap)[i] = make_uint4(0, 0, 0, 0);
+      if (named_barrier_or(2, C::NSEL, !ok)) break;
 
-      // (b) one pass over the scores: above / boundary, boundary lists and ranges
-      {
-        uint32_t act = 0, lst = 0, nar = 0;
-        uint32_t kl4[4], kh4[4];
-        bool khinf4[4];
+      // this thread's view of its four members (member 4*grp + i)
+      uint32_t um[4];       // usable chunks of this thread's block (a low-bit prefix)
+      uint32_t hm = 0;      // members counted in the round-0 histogram (uniform in the group)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const MemberSel& S = M->ms[4 * grp + i];
+        const int nvt = min(max(S.nv - r * nch, 0), nch);
+        um[i] = nvt >= 32 ? 0xFFFFFFFFu : ((1u << nvt) - 1u);
+        hm |= (S.mode == kMSel ? 1u : 0u) << i;
+      }
+      uint32_t ob4[4];    // score-linear bins: the offset's bits; key-linear: the origin
+      float sc4[4];
+      uint32_t vm4 = 0;   // members whose round-0 bins are linear in the score
+
+      auto sample_range = [&]() {
+        uint32_t v[4];
+        tmem_ld_32x32b_x4(tl, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          reg_fence(v[i]);
+          const bool use = ((hm >> i) & um[i] & 1u) != 0u;
+          const uint32_t key = score_key(__uint_as_float(v[i]));
+          const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
+          const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
+          if (lane == 0) {
+            M->pmin[quarter][4 * grp + i] = mn;
+            M->pmax[quarter][4 * grp + i] = mx;
+          }
+        }
+      };
+      auto set_range = [&]() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = 4 * grp + i;
+          uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            mn = min(mn, M->pmin[qq][m]);
+            mx = max(mx, M->pmax[qq][m]);
+          }
+          const float vmin = key_score(mn), vmax = key_score(mx);
+          const float vsc = static_cast<float>(kRefBins) / __fsub_rn(vmax, vmin);
+          const float voff = __fmul_rn(-vmin, vsc);
+          const bool vm = mn < mx && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f && isfinite(voff);
+          if (vm) {
+            ob4[i] = __float_as_uint(voff);
+            sc4[i] = vsc;
+            vm4 |= 1u << i;
+          } else if (mn > mx) {
+            ob4[i] = 0u;
+            sc4[i] = 0.f;
+          } else {
+            ob4[i] = mn;
+            sc4[i] = static_cast<float>(kRefBins) / (__uint2float_rn(mx - mn) + 1.0f);
+          }
+          if (quarter == 0 && lane == 0) {
+            M->ms[m].lo = vm ? 0u : ob4[i];
+            M->ms[m].off = vm ? voff : 0.f;
+            M->ms[m].scale = sc4[i];
+            M->ms[m].vmode = vm ? 1 : 0;
+          }
+        }
+      };
+      auto hist_chunk = [&](int c) {
+        uint32_t v[4];
+        tmem_ld_32x32b_x4(tl + c * 16, v);
+        tmem_ld_wait();
+        if (vm4 == hm) {  // every counted member has score-linear bins (the rule)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            reg_fence(v[i]);
+            const bool cnt = ((hm >> i) & (um[i] >> c) & 1u) != 0u;
+            const int b = value_bin(__uint_as_float(v[i]), sc4[i], __uint_as_float(ob4[i]));
+            if (cnt) red_shared_add(smem_u32(&hist[(4 * grp + i) * kRefBins + b]), 1u);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            reg_fence(v[i]);
+            if (((hm >> i) & (um[i] >> c) & 1u) != 0u) {
+              const float f = __uint_as_float(v[i]);
+              const int b = ((vm4 >> i) & 1u) ? value_bin(f, sc4[i], __uint_as_float(ob4[i]))
+                                              : key_bin(score_key(f), ob4[i], sc4[i]);
+              red_shared_add(smem_u32(&hist[(4 * grp + i) * kRefBins + b]), 1u);
+            }
+          }
+        }
+      };
+
+      // ---- round 0, chunk by chunk as the MMAs finish
+      for (int c = 0; c < nch; ++c) {
+        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && hm != 0) {
+          tc_fence_after();
+          if (c == 0) {
+            sample_range();
+          } else {
+            if (c == 1) {
+              set_range();
+              hist_chunk(0);
+            }
+            hist_chunk(c);
+          }
+        }
+        if (c == 0) sel_sync();  // the sample ranges are visible
+      }
+      if (ok && nch == 1 && hm != 0) {
+        set_range();
+        hist_chunk(0);
+      }
+      if (named_barrier_or(2, C::NSEL, !ok)) break;
+
+      // ---- selection rounds
+      uint32_t gt[4], bnd[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        gt[i] = M->ms[4 * grp + i].mode == kMAll ? um[i] : 0u;
+        bnd[i] = 0u;
+      }
+      int released = 0;   // chunks whose TMEM columns this warp has given back
+      auto release_upto = [&](int upto) {
+        if (upto <= released) return;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          for (int c = released; c < upto; ++c) mbar_arrive(smem_u32(&M->tfree[c]));
+        released = upto;
+      };
+#pragma unroll 1
+      for (int round = 0;; ++round) {
+        // (a) warp sw: boundary bin and key thresholds of member sw
+        if (sw < nb && M->ms[sw].active) {
+          MemberSel& S = M->ms[sw];
+          const uint32_t* hw = hist + sw * kRefBins;
+          const int need = S.need;
+          // lane l owns bins [512 - 16(l+1), 512 - 16l): descending order by lane
+          const int w0 = kRefBins - 16 * (lane + 1);
+          int s = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 x = reinterpret_cast<const uint4*>(hw + w0)[(i + lane) & 3];
+            s += static_cast<int>(x.x + x.y + x.z + x.w);
+          }
+          int incl = s;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const int L = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;
+          const int exclL = __shfl_sync(0xffffffffu, incl - s, L);
+          // lane i < 16: bin (512 - 16L - 1 - i)
+          const int w = kRefBins - 16 * L - 1 - lane;
+          const int s2 = lane < 16 ? static_cast<int>(hw[w]) : 0;
+          int incl2 = s2;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl2, o);
+            if (lane >= o) incl2 += y;
+          }
+          const int i2 = __ffs(__ballot_sync(0xffffffffu, exclL + incl2 >= need)) - 1;
+          const int bstar = kRefBins - 16 * L - 1 - i2;
+          const int above = __shfl_sync(0xffffffffu, exclL + incl2 - s2, i2);
+          const int cntb = __shfl_sync(0xffffffffu, s2, i2);
+          const uint32_t lo = S.lo;
+          const float sc = S.scale, off = S.off;
+          const bool vm = S.vmode != 0;
+          uint32_t kl = 0, kh = 0;
+          bool has_kl = true, has_kh = false;
+          if (bstar > 0) has_kl = warp_first_key_of_bin(bstar, lo, sc, off, vm, lane, &kl);
+          if (bstar < kRefBins - 1) has_kh = warp_first_key_of_bin(bstar + 1, lo, sc, off, vm, lane, &kh);
+          if (lane == 0) {
+            const int need2 = need - above;
+            S.need = need2;
+            S.cnt = cntb;
+            S.kl = has_kl ? kl : 0u;
+            S.kh = kh;
+            S.kh_inf = has_kh ? 0 : 1;
+            S.mode = (cntb == need2) ? kMWhole : (cntb <= kListCap ? kMList : kMNarrow);
+            S.nlist = 0;
+            S.bmin = 0xFFFFFFFFu;
+            S.bmax = 0u;
+          }
+          __syncwarp();
+        }
+        sel_sync();
+
+        // (b) one pass over the scores: above / boundary, boundary lists.  In
+        //     round 0 the columns are given back chunk by chunk unless a
+        //     boundary needs more rounds or the scores are written out.
+        //     key >= K  <=>  score >= key_score(K) (the key order is the score
+        //     order, -0 folded onto +0), so the pass compares scores; no upper
+        //     edge compares against NaN (never true), no lower edge against -inf.
+        bool keep_tmem = p.out_scores != nullptr;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) keep_tmem |= M->ms[m].active && M->ms[m].mode == kMNarrow;
+        uint32_t lst = 0, nar = 0;
+        float th4[4], tl4[4];
+        uint32_t cand4[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const MemberSel& S = M->ms[4 * grp + i];
           const bool a = S.active != 0;
-          act |= (a ? 1u : 0u) << i;
           lst |= (a && S.mode == kMList ? 1u : 0u) << i;
           nar |= (a && S.mode == kMNarrow ? 1u : 0u) << i;
-          kl4[i] = S.kl;
-          kh4[i] = S.kh;
-          khinf4[i] = S.kh_inf != 0;
+          th4[i] = S.kh_inf ? __int_as_float(0x7fc00000) : key_score(S.kh);
+          tl4[i] = S.kl == 0u ? -__int_as_float(0x7f800000) : key_score(S.kl);
+          cand4[i] = a ? (round == 0 ? um[i] : bnd[i]) : 0u;
+          if (a) bnd[i] = 0u;
         }
-        uint32_t cand4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          cand4[i] = ((act >> i) & 1u) ? (round == 0 ? um[i] : bnd[i]) : 0u;
-          if ((act >> i) & 1u) bnd[i] = 0u;
-        }
-        uint32_t bmn[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-        uint32_t bmx[4] = {0u, 0u, 0u, 0u};
-        const uint32_t any = __reduce_or_sync(0xffffffffu, cand4[0] | cand4[1] | cand4[2] | cand4[3]);
-        if (act != 0) {
+        const uint32_t anyc = __reduce_or_sync(0xffffffffu, cand4[0] | cand4[1] | cand4[2] | cand4[3]);
 #pragma unroll 1
-          for (int cb = 0; cb < nch; cb += 8) {
-            if (((any >> cb) & 0xFFu) == 0u) continue;
-            uint32_t v[8][4];
+        for (int cb = 0; cb < nch; cb += 4) {
+          if (((anyc >> cb) & 15u) != 0u) {
+            uint32_t v[4][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (cb + j < nch) tmem_ld_32x32b_x4(tlane + (cb + j) * 16 + 4 * grp, v[j]);
+            for (int j = 0; j < 4; ++j)
+              if (cb + j < nch) tmem_ld_32x32b_x4(tl + (cb + j) * 16, v[j]);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {
+              const int c = cb + j;
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 reg_fence(v[j][i]);
-                const int c = cb + j;
-                if (c < nch && ((cand4[i] >> c) & 1u)) {
-                  const uint32_t key = score_key(__uint_as_float(v[j][i]));
-                  if (!khinf4[i] && key >= kh4[i]) {
-                    gt[i] |= 1u << c;
-                  } else if (key >= kl4[i]) {
-                    bnd[i] |= 1u << c;
-                    bmn[i] = min(bmn[i], key);
-                    bmx[i] = max(bmx[i], key);
-                    if ((lst >> i) & 1u) {
-                      const int m = 4 * grp + i;
-                      const int at = atomicAdd(&M->ms[m].nlist, 1);
-                      if (at < kListCap) {
-                        hist[m * 2 * kListCap + at] = key;
-                        hist[m * 2 * kListCap + kListCap + at] = static_cast<uint32_t>(r * nch + c);
-                      }
-                    }
+                const float f = __uint_as_float(v[j][i]);
+                const uint32_t in = c < nch ? (cand4[i] >> c) & 1u : 0u;
+                const uint32_t hi = f >= th4[i] ? in : 0u;
+                const uint32_t lo = f >= tl4[i] ? in : 0u;
+                gt[i] |= hi << c;
+                bnd[i] |= (lo & ~hi) << c;
+              }
+            }
+            // this batch's boundary keys join their member's list, one
+            // shared-memory atomic per warp and member (boundaries are small)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t mine = ((lst >> i) & 1u) ? (bnd[i] >> cb) & 15u : 0u;
+              if (__ballot_sync(0xffffffffu, mine != 0u) == 0u) continue;
+              const int n = __popc(mine);
+              int incl = n;
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+              }
+              const int m = 4 * grp + i;
+              int base = 0;
+              if (lane == 31) base = static_cast<int>(atom_shared_add(smem_u32(&M->ms[m].nlist), static_cast<uint32_t>(incl)));
+              int at = __shfl_sync(0xffffffffu, base, 31) + incl - n;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if ((mine >> j) & 1u) {
+                  if (at < kListCap) {
+                    hist[m * 2 * kListCap + at] = score_key(__uint_as_float(v[j][i]));
+                    hist[m * 2 * kListCap + kListCap + at] = static_cast<uint32_t>(r * nch + cb + j);
                   }
+                  ++at;
                 }
               }
             }
           }
+          if (round == 0 && !keep_tmem) release_upto(min(cb + 4, nch));
+        }
+        // key ranges of the boundaries that need another round (rare)
+        if (nar != 0) {
+#pragma unroll 1
+          for (int c = 0; c < nch; ++c) {
+            uint32_t v[4];
+            tmem_ld_32x32b_x4(tl + c * 16, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if ((nar >> i) & 1u) {
-              const uint32_t mn = __reduce_min_sync(0xffffffffu, bmn[i]);
-              const uint32_t mx = __reduce_max_sync(0xffffffffu, bmx[i]);
-              if (lane == 0) {
-                atomicMin(&M->ms[4 * grp + i].bmin, mn);
-                atomicMax(&M->ms[4 * grp + i].bmax, mx);
+            for (int i = 0; i < 4; ++i) {
+              reg_fence(v[i]);
+              const bool in = ((nar >> i) & (bnd[i] >> c) & 1u) != 0u;
+              const uint32_t key = score_key(__uint_as_float(v[i]));
+              const uint32_t mn = __reduce_min_sync(0xffffffffu, in ? key : 0xFFFFFFFFu);
+              const uint32_t mx = __reduce_max_sync(0xffffffffu, in ? key : 0u);
+              if (lane == 0 && ((nar >> i) & 1u)) {
+                red_shared_min(smem_u32(&M->ms[4 * grp + i].bmin), mn);
+                red_shared_max(smem_u32(&M->ms[4 * grp + i].bmax), mx);
               }
             }
           }
         }
-      }
-      if (tid == 0) M->more = 0;
-      __syncthreads();
+        if (stid == 0) M->more = 0;
+        sel_sync();
 
-      // (c) warp m closes member m's round: rank the list, or detect equal
-      //     keys, or set up the next round over the boundary's own range
-      if (warp < nb && M->ms[warp].active) {
-        MemberSel& S = M->ms[warp];
-        const int mode = S.mode;
-        const int need = S.need;
-        if (mode == kMWhole) {
-          if (lane == 0) {
-            S.need_eq = 0x7FFFFFFF;
-            S.active = 0;
-          }
-        } else if (mode == kMList) {
-          const int n = min(S.nlist, kListCap);
-          const uint32_t* lk = hist + warp * 2 * kListCap;
-          // the need-th largest key (with multiplicity) and how many of its
-          // copies are taken
-          for (int e = lane; e < n; e += 32) {
-            const uint32_t ke = lk[e];
-            int ngt = 0, neq = 0;
-            for (int f = 0; f < n; ++f) {
-              const uint32_t kf = lk[f];
-              ngt += kf > ke ? 1 : 0;
-              neq += kf == ke ? 1 : 0;
+        // (c) warp sw closes member sw's round: rank the list, or detect equal
+        //     keys, or set up the next round over the boundary's key range
+        if (sw < nb && M->ms[sw].active) {
+          MemberSel& S = M->ms[sw];
+          const int m = sw;
+          const int mode = S.mode;
+          const int need = S.need;
+          if (mode == kMWhole) {
+            if (lane == 0) {
+              S.need_eq = 0x7FFFFFFF;
+              S.active = 0;
             }
-            if (ngt < need && need <= ngt + neq) {
-              S.tk = ke;             // every such lane writes the same values
-              S.need_eq = need - ngt;
+          } else if (mode == kMList) {
+            const int n = min(S.nlist, kListCap);
+            const uint32_t* lk = hist + m * 2 * kListCap;
+            // the need-th largest key (with multiplicity) and how many of its
+            // copies are taken
+            for (int e = lane; e < n; e += 32) {
+              const uint32_t ke = lk[e];
+              int ngt = 0, neq = 0;
+              for (int f = 0; f < n; ++f) {
+                const uint32_t kf = lk[f];
+                ngt += kf > ke ? 1 : 0;
+                neq += kf == ke ? 1 : 0;
+              }
+              if (ngt < need && need <= ngt + neq) {
+                S.tk = ke;             // every such lane writes the same values
+                S.need_eq = need - ngt;
+              }
+            }
+            __syncwarp();
+            // the list's decisions, as bitmaps over candidates
+            const uint32_t tk = S.tk;
+            uint32_t* bgt = bmap + (m * 2) * BMW;
+            uint32_t* beq = bgt + BMW;
+            for (int e = lane; e < n; e += 32) {
+              const uint32_t ke = lk[e];
+              const uint32_t te = lk[kListCap + e];
+              if (ke > tk) red_shared_or(smem_u32(&bgt[te >> 5]), 1u << (te & 31));
+              else if (ke == tk) red_shared_or(smem_u32(&beq[te >> 5]), 1u << (te & 31));
+            }
+            if (lane == 0) S.active = 0;
+          } else {  // kMNarrow
+            if (lane == 0) {
+              const uint32_t mn = S.bmin, mx = S.bmax;
+              if (mn == mx) {
+                S.mode = kMTies;
+                S.tk = mn;
+                S.need_eq = need;
+                S.active = 0;
+              } else {
+                S.lo = mn;
+                S.scale = static_cast<float>(kRefBins) / (__uint2float_rn(mx - mn) + 1.0f);
+                S.off = 0.f;
+                S.vmode = 0;
+                S.mode = kMSel;
+                M->more = 1;
+              }
             }
           }
           __syncwarp();
-          if (lane == 0) S.active = 0;
-        } else {  // kMNarrow
-          if (lane == 0) {
-            const uint32_t mn = S.bmin, mx = S.bmax;
-            if (mn == mx) {
-              S.mode = kMTies;
-              S.tk = mn;
-              S.need_eq = need;
-              S.active = 0;
-            } else {
-              S.lo = mn;
-              S.scale = static_cast<float>(kRefBins) / (__uint2float_rn(mx - mn) + 1.0f);
-              S.vmode = 0;
-              S.mode = kMSel;
-              M->more = 1;
-            }
-          }
         }
-      }
-      __syncthreads();
-      if (!M->more) break;
+        sel_sync();
+        if (!M->more) break;
 
-      // (d) another histogram round over the open boundaries (rare: more than
-      //     kListCap keys in one bin with distinct values)
-      for (int i = tid; i < C::HIST_BYTES / 16; i += C::NT) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
-      __syncthreads();
-      {
-        uint32_t act = 0;
-        uint32_t lo_[4];
-        float sc_[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const MemberSel& S = M->ms[4 * grp + i];
-          act |= (S.active ? 1u : 0u) << i;
-          lo_[i] = S.lo;
-          sc_[i] = S.scale;
-        }
-        uint32_t c4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) c4[i] = ((act >> i) & 1u) ? bnd[i] : 0u;
-        const uint32_t any = __reduce_or_sync(0xffffffffu, c4[0] | c4[1] | c4[2] | c4[3]);
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          if (((any >> c) & 1u) == 0u) continue;
-          uint32_t v[4];
-          tmem_ld_32x32b_x4(tlane + c * 16 + 4 * grp, v);
-          tmem_ld_wait();
+        // (d) another histogram round over the open boundaries (rare: more
+        //     than kListCap keys in one bin with distinct values)
+        for (int i = stid; i < C::HIST_BYTES / 16; i += C::NSEL)
+          reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+        sel_sync();
+        {
+          uint32_t c4[4], lo_[4];
+          float sc_[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            reg_fence(v[i]);
-            if ((c4[i] >> c) & 1u) {
-              const int b = key_bin(score_key(__uint_as_float(v[i])), lo_[i], sc_[i]);
-              atomicAdd(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)], 1u << ((b & 1) * 16));
+            const MemberSel& S = M->ms[4 * grp + i];
+            c4[i] = S.active ? bnd[i] : 0u;
+            lo_[i] = S.lo;
+            sc_[i] = S.scale;
+          }
+          const uint32_t anyb = __reduce_or_sync(0xffffffffu, c4[0] | c4[1] | c4[2] | c4[3]);
+#pragma unroll 1
+          for (int c = 0; c < nch; ++c) {
+            if (((anyb >> c) & 1u) == 0u) continue;
+            uint32_t v[4];
+            tmem_ld_32x32b_x4(tl + c * 16, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              reg_fence(v[i]);
+              if ((c4[i] >> c) & 1u) {
+                const int b = key_bin(score_key(__uint_as_float(v[i])), lo_[i], sc_[i]);
+                red_shared_add(smem_u32(&hist[(4 * grp + i) * kRefBins + b]), 1u);
+              }
             }
           }
         }
+        sel_sync();
       }
-      __syncthreads();
-    }
 
-    // ---- final rule per member: gt, plus the first need_eq of eq in order
-    uint32_t eq[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const MemberSel& S = M->ms[4 * grp + i];
-      const int mode = S.mode;
-      if (mode == kMWhole || mode == kMTies) {
-        eq[i] = bnd[i];
-      } else if (mode == kMList) {
-        // re-read the few boundary keys and split them around tk
-        const uint32_t tk = S.tk;
-        uint32_t any = __reduce_or_sync(0xffffffffu, bnd[i]);
-        while (any) {
-          const int c = __ffs(any) - 1;
-          any &= any - 1;
-          uint32_t v;
-          tmem_ld_32x32b_x1(tlane + c * 16 + 4 * grp + i, v);
-          tmem_ld_wait();
-          if ((bnd[i] >> c) & 1u) {
-            const uint32_t key = score_key(__uint_as_float(v));
-            if (key > tk) gt[i] |= 1u << c;
-            else if (key == tk) eq[i] |= 1u << c;
-          }
-        }
-      }
-    }
-    // group scan (thread order = candidate order) of (|gt|, |eq|) for 4 members
-    int ex[8];
-    {
-      int incl[8];
+      // ---- final rule per member: gt, plus the first need_eq of eq in order
+      uint32_t eq[4];
+      const int t0 = r * nch;
+      auto my_bits = [&](const uint32_t* bm) -> uint32_t {
+        if (nch == 0) return 0u;
+        const int w = t0 >> 5, o = t0 & 31;
+        uint32_t x = bm[w] >> o;
+        if (o != 0 && w + 1 < BMW) x |= bm[w + 1] << (32 - o);
+        return nch >= 32 ? x : (x & ((1u << nch) - 1u));
+      };
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        incl[i] = __popc(gt[i]);
-        incl[4 + i] = __popc(eq[i]);
+        const int m = 4 * grp + i;
+        const int mode = M->ms[m].mode;
+        eq[i] = 0u;
+        if (mode == kMWhole || mode == kMTies) {
+          eq[i] = bnd[i];
+        } else if (mode == kMList) {
+          gt[i] |= my_bits(bmap + (m * 2) * BMW);
+          eq[i] = my_bits(bmap + (m * 2 + 1) * BMW);
+        }
       }
-      int own[8];
+      // group scan (thread order = candidate order) of (|gt|, |eq|) for the four members
+      int ex[8];
+      {
+        int incl[8], own[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) own[k] = incl[k];
+        for (int i = 0; i < 4; ++i) {
+          own[i] = __popc(gt[i]);
+          own[4 + i] = __popc(eq[i]);
+        }
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
+        for (int k = 0; k < 8; ++k) incl[k] = own[k];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int y = __shfl_up_sync(0xffffffffu, incl[k], o);
+            if (lane >= o) incl[k] += y;
+          }
+        }
+        if (lane == 31) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) M->gscan[grp][quarter][k] = incl[k];
+        }
+        named_barrier(3 + grp, 128);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const int y = __shfl_up_sync(0xffffffffu, incl[k], o);
-          if (lane >= o) incl[k] += y;
+          int off = 0;
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) off += (qq < quarter) ? M->gscan[grp][qq][k] : 0;
+          ex[k] = off + incl[k] - own[k];
         }
       }
-      if (lane == 31) {
+      // the histogram bytes become per-warp output staging (STG entries a
+      // warp); a warp's slice of a row goes out in STG-entry parts
+      uint32_t* stg = hist + sw * C::STG;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) M->gscan[grp][quarter][k] = incl[k];
-      }
-      group_sync(grp);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        int off = 0;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) off += (qq < quarter) ? M->gscan[grp][qq][k] : 0;
-        ex[k] = off + incl[k] - own[k];
-      }
-    }
-    // the histogram bytes become per-warp output staging (1024 entries a warp)
-    uint32_t* stg = hist + warp * 1024;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = 4 * grp + i;
-      if (m >= nb) continue;
-      const MemberSel& S = M->ms[m];
-      const int K = S.K, need_eq = S.need_eq;
-      const int eqb = ex[4 + i];
-      const int neq = __popc(eq[i]);
-      const int take = min(max(need_eq - eqb, 0), neq);
-      uint32_t sel = gt[i];
-      if (take == neq) {
-        sel |= eq[i];
-      } else {
-        uint32_t e = eq[i];
-        for (int k = 0; k < take; ++k) {
-          sel |= e & (0u - e);  // lowest remaining equal key
-          e &= e - 1;
+      for (int i = 0; i < 4; ++i) {
+        const int m = 4 * grp + i;
+        if (m >= nb) continue;
+        const int K = M->ms[m].K, need_eq = M->ms[m].need_eq;
+        const int eqb = ex[4 + i];
+        const int neq = __popc(eq[i]);
+        const int take = min(max(need_eq - eqb, 0), neq);
+        uint32_t sel = gt[i];
+        if (take == neq) {
+          sel |= eq[i];
+        } else {
+          uint32_t e = eq[i];
+          for (int k = 0; k < take; ++k) {
+            sel |= e & (0u - e);  // lowest remaining equal key
+            e &= e - 1;
+          }
         }
-      }
-      const int slot = ex[i] + min(eqb, need_eq);
-      const int wb = __shfl_sync(0xffffffffu, slot, 0);
-      const int wc = __shfl_sync(0xffffffffu, slot + __popc(sel), 31) - wb;
-      const long long orow_off = ((qrow0 + mb + m) * p.H + h) * static_cast<long long>(p.top_k);
-      int32_t* orow = p.out + orow_off;
-      {
-        int o = slot - wb;
-        for (uint32_t bits = sel; bits; bits &= bits - 1) {
-          const int c = __ffs(bits) - 1;
-          stg[o++] = static_cast<uint32_t>(cand_at(c, r));
+        const int slot = ex[i] + min(eqb, need_eq);
+        const int wb = __shfl_sync(0xffffffffu, slot, 0);
+        // (the selection takes exactly K; the bound only guards the row)
+        const int wc = min(__shfl_sync(0xffffffffu, slot + __popc(sel), 31), K) - wb;
+        const long long orow_off = ((it.qrow0 + it.mb + m) * p.H + it.h) * static_cast<long long>(p.top_k);
+        int32_t* orow = p.out + orow_off;
+        for (int part = 0; part * C::STG < wc; ++part) {
+          const int plo = part * C::STG;
+          int o = slot - wb - plo;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const uint32_t bit = (sel >> c) & 1u;
+            if (bit && o >= 0 && o < C::STG) stg[o] = static_cast<uint32_t>(cx[cidx_pos(c, r)]);
+            o += static_cast<int>(bit);
+          }
+          __syncwarp();
+          const int n = min(wc - plo, C::STG);
+#pragma unroll 4
+          for (int x = lane; x < n; x += 32) orow[wb + plo + x] = static_cast<int32_t>(stg[x]);
+          __syncwarp();
         }
+        if (p.out_scores) {
+          float* srow = p.out_scores + orow_off;
+          const uint32_t any = __reduce_or_sync(0xffffffffu, sel);
+          for (int part = 0; part * C::STG < wc; ++part) {
+            const int plo = part * C::STG;
+            int o = slot - wb - plo;
+            for (uint32_t a = any; a; a &= a - 1) {
+              const int c = __ffs(a) - 1;
+              uint32_t v;
+              tmem_ld_32x32b_x1(tl + c * 16 + i, v);
+              tmem_ld_wait();
+              if ((sel >> c) & 1u) {
+                if (o >= 0 && o < C::STG) stg[o] = v;
+                ++o;
+              }
+            }
+            __syncwarp();
+            const int n = min(wc - plo, C::STG);
+            for (int x = lane; x < n; x += 32) srow[wb + plo + x] = __uint_as_float(stg[x]);
+            __syncwarp();
+          }
+          for (int x = K + r; x < p.top_k; x += 128) srow[x] = __int_as_float(0x7fc00000);
+        }
+        for (int x = K + r; x < p.top_k; x += 128) orow[x] = -1;
       }
+      // this item's TMEM columns and candidate list are free
+      release_upto(NCH);
       __syncwarp();
-      for (int x = lane; x < wc; x += 32) orow[wb + x] = static_cast<int32_t>(stg[x]);
-      __syncwarp();
-      if (p.out_scores) {
-        float* srow = p.out_scores + orow_off;
-        uint32_t any = __reduce_or_sync(0xffffffffu, sel);
-        int o = slot - wb;
-        while (any) {
-          const int c = __ffs(any) - 1;
-          any &= any - 1;
-          uint32_t v;
-          tmem_ld_32x32b_x1(tlane + c * 16 + 4 * grp + i, v);
-          tmem_ld_wait();
-          if ((sel >> c) & 1u) stg[o++] = v;
-        }
-        __syncwarp();
-        for (int x = lane; x < wc; x += 32) srow[wb + x] = __uint_as_float(stg[x]);
-        __syncwarp();
-        for (int x = K + r; x < p.top_k; x += 128) srow[x] = __int_as_float(0x7fc00000);
-      }
-      for (int x = K + r; x < p.top_k; x += 128) orow[x] = -1;
+      if (lane == 0) mbar_arrive(smem_u32(&M->cfree[buf]));
+      ++kk;
+      if (named_barrier_or(2, C::NSEL, !ok)) break;
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
   }
 
-  // On an aborted run, let the MMAs already issued finish before TMEM is freed.
-  if (tid == 0 && !ok && last_commit >= 0)
-    mbar_wait_cleanup(bar0 + 8u * (last_commit % C::NS), (last_commit / C::NS) & 1);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
   }

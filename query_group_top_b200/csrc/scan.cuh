@@ -217,7 +217,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
     const bool row_samples = sampling && bound > p.cap;
 
     auto bin_count = [&](int b) -> int { return (hist[(b >> 1) * C::BM + r] >> ((b & 1) << 4)) & 0xFFFF; };
-    auto bin_add = [&](int b) { atomicAdd(&hist[(b >> 1) * C::BM + r], 1u << ((b & 1) << 4)); };
+    auto bin_add = [&](int b) { red_shared_add(smem_u32(&hist[(b >> 1) * C::BM + r]), 1u << ((b & 1) << 4)); };
     auto zero_half_row = [&]() {
       for (int w = 0; w < 64; ++w) hist[(e * 64 + w) * C::BM + r] = 0;
     };

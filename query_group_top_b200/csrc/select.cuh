@@ -100,7 +100,7 @@ __device__ void block_select_emit(int n, int K, Fetch fetch, Emit emit, SelectSm
     __syncthreads();
     for (int e = threadIdx.x; e < n; e += NT) {
       const uint32_t key = fetch(e);
-      if ((key & tmask) == thr) atomicAdd(&sm.hist[(key >> sh) & (nbn - 1)], 1);
+      if ((key & tmask) == thr) red_shared_add(smem_u32(&sm.hist[(key >> sh) & (nbn - 1)]), 1u);
     }
     __syncthreads();
     // thread t owns bins [top - per + 1, top], scanned from the top
