@@ -701,26 +701,18 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const uint32_t mine = ((lst >> i) & 1u) ? (bnd[i] >> cb) & 15u : 0u;
-              if (__ballot_sync(0xffffffffu, mine != 0u) == 0u) continue;
-              const int n = __popc(mine);
-              int incl = n;
+              if (mine != 0u) {
+                const int m = 4 * grp + i;
+                int at = static_cast<int>(atom_shared_add(smem_u32(&M->ms[m].nlist), static_cast<uint32_t>(__popc(mine))));
 #pragma unroll
-              for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-              }
-              const int m = 4 * grp + i;
-              int base = 0;
-              if (lane == 31) base = static_cast<int>(atom_shared_add(smem_u32(&M->ms[m].nlist), static_cast<uint32_t>(incl)));
-              int at = __shfl_sync(0xffffffffu, base, 31) + incl - n;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                if ((mine >> j) & 1u) {
-                  if (at < kListCap) {
-                    hist[m * 2 * kListCap + at] = score_key(__uint_as_float(v[j][i]));
-                    hist[m * 2 * kListCap + kListCap + at] = static_cast<uint32_t>(r * nch + cb + j);
+                for (int j = 0; j < 4; ++j) {
+                  if ((mine >> j) & 1u) {
+                    if (at < kListCap) {
+                      hist[m * 2 * kListCap + at] = score_key(__uint_as_float(v[j][i]));
+                      hist[m * 2 * kListCap + kListCap + at] = static_cast<uint32_t>(r * nch + cb + j);
+                    }
+                    ++at;
                   }
-                  ++at;
                 }
               }
             }
@@ -934,12 +926,15 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         int32_t* orow = p.out + orow_off;
         for (int part = 0; part * C::STG < wc; ++part) {
           const int plo = part * C::STG;
-          int o = slot - wb - plo;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const uint32_t bit = (sel >> c) & 1u;
-            if (bit && o >= 0 && o < C::STG) stg[o] = static_cast<uint32_t>(cx[cidx_pos(c, r)]);
-            o += static_cast<int>(bit);
+          // this lane's selected candidates that fall in the part [plo, plo + STG)
+          const int o0 = slot - wb - plo;
+          uint32_t bits = sel;
+          if (o0 < 0) {  // skip the ones staged by an earlier part
+            for (int k = 0; k < -o0 && bits; ++k) bits &= bits - 1;
+          }
+          for (int o = max(o0, 0); bits && o < C::STG; ++o, bits &= bits - 1) {
+            const int c = __ffs(bits) - 1;
+            stg[o] = static_cast<uint32_t>(cx[cidx_pos(c, r)]);
           }
           __syncwarp();
           const int n = min(wc - plo, C::STG);
