@@ -145,9 +145,11 @@ int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t*
  * Synchronises `stream`, then reads and clears this device's kernel status
  * word.  Returns PIVOT_OK, PIVOT_ERR_TIMEOUT (a bounded wait inside a kernel
  * gave up; that call's outputs are not valid), PIVOT_ERR_INVALID_ARG (a decode
- * sequence exceeded max_seqlen) or PIVOT_ERR_CUDA.  *flags (nullable) receives
- * the raw status bits; bit 4 means some rows took the exact fallback path
- * (results remain exact).
+ * sequence exceeded max_seqlen) or PIVOT_ERR_CUDA (a CUDA error, or status bit
+ * 8: a refine selection exceeded its round limit, which finite scores never
+ * do; that call's outputs are not valid).  *flags (nullable) receives the raw
+ * status bits; bit 4 means some rows took the exact fallback path (results
+ * remain exact).
  */
 int pivot_sync_status(void* stream, int* flags);
 

@@ -20,7 +20,7 @@ __all__ = ["REFINE", "REUSE", "PivotError", "pivot_index", "dense_index", "pivot
            "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED"]
 
 REFINE, REUSE = 0, 1
-FLAG_TIMEOUT, FLAG_BADLEN, FLAG_FALLBACK = 1, 2, 4
+FLAG_TIMEOUT, FLAG_BADLEN, FLAG_FALLBACK, FLAG_NOCONVERGE = 1, 2, 4, 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpivot.so")

@@ -629,6 +629,7 @@ int pivot_sync_status(void* stream, int* flags) {
   if (flags) *flags = v;
   if (v & kStTimeout) return fail(PIVOT_ERR_TIMEOUT, "a kernel wait timed out; outputs of that call are invalid");
   if (v & kStBadLen) return fail(PIVOT_ERR_INVALID_ARG, "a decode sequence was longer than max_seqlen");
+  if (v & kStNoConverge) return fail(PIVOT_ERR_CUDA, "a refine selection did not converge; outputs of that call are invalid");
   return PIVOT_OK;
 }
 

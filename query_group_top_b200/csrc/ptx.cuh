@@ -15,6 +15,7 @@ enum : int {
   kStTimeout = 1,   // a bounded wait on a barrier gave up
   kStBadLen = 2,    // a decode sequence was longer than the declared maximum
   kStFallback = 4,  // informational: some rows took the exact fallback path
+  kStNoConverge = 8,  // a selection exceeded its round limit (cannot happen on finite scores)
 };
 
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s

@@ -72,8 +72,11 @@ enum : int {
   kMTies = 6,    // boundary keys all equal: the first need_eq in order
 };
 
-constexpr int kRefBins = 512;
+constexpr int kRefBins = 1024;
 constexpr int kListCap = 256;
+// Each key-linear round shrinks a boundary's key range by a factor of about
+// 256, so 32-bit keys need at most five rounds after round 0.
+constexpr int kMaxRounds = 8;
 
 struct MemberSel {
   int nv;           // usable candidates: the ascending prefix with j < pos
@@ -122,12 +125,13 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
   static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
-  // histograms: 16 members x 512 bins of 32-bit counts; the same bytes later
-  // hold the boundary lists and the per-warp output staging
-  static constexpr int HIST_BYTES = 16 * kRefBins * 4;
+  // histograms: 16 members x 1024 bins of 16-bit counts (two per word); the
+  // same bytes later hold the boundary lists, and together with the decision
+  // bitmaps that follow them, the per-warp output staging
+  static constexpr int HIST_BYTES = 16 * (kRefBins / 2) * 4;
   static_assert(16 * 2 * kListCap * 4 <= HIST_BYTES, "lists alias the histograms");
-  static constexpr int STG = 512;                       // output staging entries per select warp
-  static_assert(16 * STG * 4 <= HIST_BYTES, "output staging aliases the histograms");
+  // output staging entries per select warp: the histogram and bitmap bytes
+  __host__ __device__ static int stg_entries(int Kc) { return (HIST_BYTES / 4 + 16 * 2 * bm_words(Kc)) / 16; }
   __host__ __device__ static int nch_max(int Kc) { return (Kc + 127) / 128; }
   __host__ __device__ static int cidx_words(int Kc) { return nch_max(Kc) * 128; }
   // list decisions: per member, "above" and "equal" bitmaps over candidates
@@ -535,7 +539,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             reg_fence(v[i]);
             const bool cnt = ((hm >> i) & (um[i] >> c) & 1u) != 0u;
             const int b = value_bin(__uint_as_float(v[i]), sc4[i], __uint_as_float(ob4[i]));
-            if (cnt) red_shared_add(smem_u32(&hist[(4 * grp + i) * kRefBins + b]), 1u);
+            if (cnt) red_shared_add(smem_u32(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)]), 1u << ((b & 1) << 4));
           }
         } else {
 #pragma unroll
@@ -545,7 +549,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               const float f = __uint_as_float(v[i]);
               const int b = ((vm4 >> i) & 1u) ? value_bin(f, sc4[i], __uint_as_float(ob4[i]))
                                               : key_bin(score_key(f), ob4[i], sc4[i]);
-              red_shared_add(smem_u32(&hist[(4 * grp + i) * kRefBins + b]), 1u);
+              red_shared_add(smem_u32(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)]), 1u << ((b & 1) << 4));
             }
           }
         }
@@ -593,18 +597,24 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       };
 #pragma unroll 1
       for (int round = 0;; ++round) {
+        if (round == kMaxRounds) {
+          if (stid == 0) atomicOr(p.status, kStNoConverge);
+          break;
+        }
         // (a) warp sw: boundary bin and key thresholds of member sw
         if (sw < nb && M->ms[sw].active) {
           MemberSel& S = M->ms[sw];
-          const uint32_t* hw = hist + sw * kRefBins;
+          const uint32_t* hw = hist + sw * (kRefBins / 2);
           const int need = S.need;
-          // lane l owns bins [512 - 16(l+1), 512 - 16l): descending order by lane
-          const int w0 = kRefBins - 16 * (lane + 1);
+          // lane l owns words [512 - 16(l+1), 512 - 16l), i.e. 32 bins, in
+          // descending order by lane; a word holds bins 2w (low half) and 2w+1
+          const int w0 = kRefBins / 2 - 16 * (lane + 1);
           int s = 0;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint4 x = reinterpret_cast<const uint4*>(hw + w0)[(i + lane) & 3];
-            s += static_cast<int>(x.x + x.y + x.z + x.w);
+            s += static_cast<int>((x.x & 0xFFFFu) + (x.x >> 16) + (x.y & 0xFFFFu) + (x.y >> 16) + (x.z & 0xFFFFu) +
+                                  (x.z >> 16) + (x.w & 0xFFFFu) + (x.w >> 16));
           }
           int incl = s;
 #pragma unroll
@@ -612,21 +622,30 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
           }
-          const int L = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;
+          // (the counts always reach need; the clamps only keep indices in range)
+          const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+          const int L = hit ? __ffs(hit) - 1 : 31;
           const int exclL = __shfl_sync(0xffffffffu, incl - s, L);
-          // lane i < 16: bin (512 - 16L - 1 - i)
-          const int w = kRefBins - 16 * L - 1 - lane;
-          const int s2 = lane < 16 ? static_cast<int>(hw[w]) : 0;
+          // lane i < 16: word (512 - 16L - 1 - i), bins 2w+1 then 2w
+          const int w = kRefBins / 2 - 16 * L - 1 - lane;
+          const uint32_t wv = lane < 16 ? hw[w] : 0u;
+          const int chi = static_cast<int>(wv >> 16), clo = static_cast<int>(wv & 0xFFFFu);
+          const int s2 = chi + clo;
           int incl2 = s2;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl2, o);
             if (lane >= o) incl2 += y;
           }
-          const int i2 = __ffs(__ballot_sync(0xffffffffu, exclL + incl2 >= need)) - 1;
-          const int bstar = kRefBins - 16 * L - 1 - i2;
-          const int above = __shfl_sync(0xffffffffu, exclL + incl2 - s2, i2);
-          const int cntb = __shfl_sync(0xffffffffu, s2, i2);
+          const unsigned hit2 = __ballot_sync(0xffffffffu, exclL + incl2 >= need);
+          const int i2 = hit2 ? __ffs(hit2) - 1 : 15;
+          const int before = __shfl_sync(0xffffffffu, exclL + incl2 - s2, i2);
+          const int hi2 = __shfl_sync(0xffffffffu, chi, i2), lo2 = __shfl_sync(0xffffffffu, clo, i2);
+          const int w2 = kRefBins / 2 - 16 * L - 1 - i2;
+          const bool upper = before + hi2 >= need;
+          const int bstar = upper ? 2 * w2 + 1 : 2 * w2;
+          const int above = upper ? before : before + hi2;
+          const int cntb = upper ? hi2 : lo2;
           const uint32_t lo = S.lo;
           const float sc = S.scale, off = S.off;
           const bool vm = S.vmode != 0;
@@ -835,7 +854,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               reg_fence(v[i]);
               if ((c4[i] >> c) & 1u) {
                 const int b = key_bin(score_key(__uint_as_float(v[i])), lo_[i], sc_[i]);
-                red_shared_add(smem_u32(&hist[(4 * grp + i) * kRefBins + b]), 1u);
+                red_shared_add(smem_u32(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)]), 1u << ((b & 1) << 4));
               }
             }
           }
@@ -865,6 +884,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           eq[i] = my_bits(bmap + (m * 2 + 1) * BMW);
         }
       }
+      sel_sync();  // every warp has read its bitmaps: their bytes become staging
       // group scan (thread order = candidate order) of (|gt|, |eq|) for the four members
       int ex[8];
       {
@@ -897,9 +917,10 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           ex[k] = off + incl[k] - own[k];
         }
       }
-      // the histogram bytes become per-warp output staging (STG entries a
-      // warp); a warp's slice of a row goes out in STG-entry parts
-      uint32_t* stg = hist + sw * C::STG;
+      // the histogram and bitmap bytes become per-warp output staging (STGE
+      // entries a warp); a warp's slice of a row goes out in STGE-entry parts
+      const int STGE = C::stg_entries(p.Kc);
+      uint32_t* stg = hist + sw * STGE;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = 4 * grp + i;
@@ -924,20 +945,20 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         const int wc = min(__shfl_sync(0xffffffffu, slot + __popc(sel), 31), K) - wb;
         const long long orow_off = ((it.qrow0 + it.mb + m) * p.H + it.h) * static_cast<long long>(p.top_k);
         int32_t* orow = p.out + orow_off;
-        for (int part = 0; part * C::STG < wc; ++part) {
-          const int plo = part * C::STG;
-          // this lane's selected candidates that fall in the part [plo, plo + STG)
+        for (int part = 0; part * STGE < wc; ++part) {
+          const int plo = part * STGE;
+          // this lane's selected candidates that fall in the part [plo, plo + STGE)
           const int o0 = slot - wb - plo;
           uint32_t bits = sel;
           if (o0 < 0) {  // skip the ones staged by an earlier part
             for (int k = 0; k < -o0 && bits; ++k) bits &= bits - 1;
           }
-          for (int o = max(o0, 0); bits && o < C::STG; ++o, bits &= bits - 1) {
+          for (int o = max(o0, 0); bits && o < STGE; ++o, bits &= bits - 1) {
             const int c = __ffs(bits) - 1;
             stg[o] = static_cast<uint32_t>(cx[cidx_pos(c, r)]);
           }
           __syncwarp();
-          const int n = min(wc - plo, C::STG);
+          const int n = min(wc - plo, STGE);
 #pragma unroll 4
           for (int x = lane; x < n; x += 32) orow[wb + plo + x] = static_cast<int32_t>(stg[x]);
           __syncwarp();
@@ -945,8 +966,8 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         if (p.out_scores) {
           float* srow = p.out_scores + orow_off;
           const uint32_t any = __reduce_or_sync(0xffffffffu, sel);
-          for (int part = 0; part * C::STG < wc; ++part) {
-            const int plo = part * C::STG;
+          for (int part = 0; part * STGE < wc; ++part) {
+            const int plo = part * STGE;
             int o = slot - wb - plo;
             for (uint32_t a = any; a; a &= a - 1) {
               const int c = __ffs(a) - 1;
@@ -954,12 +975,12 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               tmem_ld_32x32b_x1(tl + c * 16 + i, v);
               tmem_ld_wait();
               if ((sel >> c) & 1u) {
-                if (o >= 0 && o < C::STG) stg[o] = v;
+                if (o >= 0 && o < STGE) stg[o] = v;
                 ++o;
               }
             }
             __syncwarp();
-            const int n = min(wc - plo, C::STG);
+            const int n = min(wc - plo, STGE);
             for (int x = lane; x < n; x += 32) srow[wb + plo + x] = __uint_as_float(stg[x]);
             __syncwarp();
           }
