@@ -17,6 +17,7 @@ workload on the host cores.
 """
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -73,6 +74,24 @@ def algorithmic(c):
         "proxy": ("hbm", float(L * H * d * 2 + G * H * d * 2)),
         "fallback": ("hbm", 0.0),
     }
+
+
+def measured_traffic(kernel, heads):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled
+    from its one-head capture to `heads` (the traffic grows with the heads);
+    None when there is no capture or the kernel's source changed since."""
+    if kernel != "refine":
+        return None
+    prof = os.path.join(ROOT, "profiles", "refine_c3_one_head.md")
+    src = os.path.join(ROOT, "query_group_top_b200", "csrc", "refine.cuh")
+    try:
+        fields = dict(line.split(": ", 1) for line in open(prof).read().splitlines() if ": " in line)
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if fields.get("source_sha256_16", "").strip() != digest:
+            return None
+        return float(fields["traffic_bytes_per_head_launch"]) * heads
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 class ClockSampler:
@@ -286,7 +305,7 @@ def main():
     else:
         achieved = work / t_launch / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": None, "kernel": dom,
+                "frac": achieved / pk["hbm"], "traffic": measured_traffic(dom, H), "kernel": dom,
                 "peak_note": f"{pk['src']} HBM copy bandwidth"}
     scan_t = trace.get("scan_filter", (0, 1))
     scan_tf = alg["scan_filter"][1] / (scan_t[0] / scan_t[1] / 1000.0) / 1e12 if scan_t[0] else None
