@@ -693,6 +693,10 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           if (a) bnd[i] = 0u;
         }
         const uint32_t anyc = __reduce_or_sync(0xffffffffu, cand4[0] | cand4[1] | cand4[2] | cand4[3]);
+        // common case: every candidate of every lane's block counts for all
+        // four members, so the pass needs no per-key candidate test
+        const uint32_t fullm = nch >= 32 ? 0xFFFFFFFFu : ((1u << nch) - 1u);
+        const bool dense4 = __all_sync(0xffffffffu, (cand4[0] & cand4[1] & cand4[2] & cand4[3]) == fullm);
 #pragma unroll 1
         for (int cb = 0; cb < nch; cb += 4) {
           if (((anyc >> cb) & 15u) != 0u) {
@@ -701,18 +705,32 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             for (int j = 0; j < 4; ++j)
               if (cb + j < nch) tmem_ld_32x32b_x4(tl + (cb + j) * 16, v[j]);
             tmem_ld_wait();
+            if (dense4 && cb + 4 <= nch) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int c = cb + j;
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t bit = 1u << (cb + j);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                reg_fence(v[j][i]);
-                const float f = __uint_as_float(v[j][i]);
-                const uint32_t in = c < nch ? (cand4[i] >> c) & 1u : 0u;
-                const uint32_t hi = f >= th4[i] ? in : 0u;
-                const uint32_t lo = f >= tl4[i] ? in : 0u;
-                gt[i] |= hi << c;
-                bnd[i] |= (lo & ~hi) << c;
+                for (int i = 0; i < 4; ++i) {
+                  reg_fence(v[j][i]);
+                  const float f = __uint_as_float(v[j][i]);
+                  if (f >= th4[i]) gt[i] |= bit;
+                  else if (f >= tl4[i]) bnd[i] |= bit;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int c = cb + j;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  reg_fence(v[j][i]);
+                  const float f = __uint_as_float(v[j][i]);
+                  const uint32_t in = c < nch ? (cand4[i] >> c) & 1u : 0u;
+                  const uint32_t hi = f >= th4[i] ? in : 0u;
+                  const uint32_t lo = f >= tl4[i] ? in : 0u;
+                  gt[i] |= hi << c;
+                  bnd[i] |= (lo & ~hi) << c;
+                }
               }
             }
             // this batch's boundary keys join their member's list, one
@@ -953,9 +971,19 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           if (o0 < 0) {  // skip the ones staged by an earlier part
             for (int k = 0; k < -o0 && bits; ++k) bits &= bits - 1;
           }
-          for (int o = max(o0, 0); bits && o < STGE; ++o, bits &= bits - 1) {
-            const int c = __ffs(bits) - 1;
-            stg[o] = static_cast<uint32_t>(cx[cidx_pos(c, r)]);
+          // two entries an iteration: their index loads overlap
+          int o = max(o0, 0);
+          while (bits != 0u && o < STGE) {
+            const int c1 = __ffs(bits) - 1;
+            bits &= bits - 1;
+            const bool two = bits != 0u && o + 1 < STGE;
+            const int c2 = two ? __ffs(bits) - 1 : c1;
+            if (two) bits &= bits - 1;
+            const uint32_t v1 = static_cast<uint32_t>(cx[cidx_pos(c1, r)]);
+            const uint32_t v2 = static_cast<uint32_t>(cx[cidx_pos(c2, r)]);
+            stg[o] = v1;
+            if (two) stg[o + 1] = v2;
+            o += two ? 2 : 1;
           }
           __syncwarp();
           const int n = min(wc - plo, STGE);
