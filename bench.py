@@ -94,6 +94,50 @@ def measured_traffic(kernel, heads):
         return None
 
 
+class RankGroup:
+    """One process per GPU (or per CPU rank in tests): the barrier and the
+    max-over-ranks reduction of the bench's timings.  Every rank takes the same
+    collective steps in the same order; rank 0 alone reports."""
+
+    def __init__(self, backend, device):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist = torch, dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.device = device
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, x):
+        if self.world == 1:
+            return x
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+def weak_value(world, L, H, ms_max):
+    """Whole-job throughput: every rank indexes its own L x H problem (weak
+    scaling), and the job takes as long as its slowest rank."""
+    return world * L * H / (ms_max / 1000.0)
+
+
+def rank_seed(base, rank):
+    """Each rank draws its own independent layer of the workload."""
+    return base + rank
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -230,31 +274,18 @@ def main():
         return
 
     import torch
-    import torch.distributed as dist
 
     import query_group_top_b200 as qg
     qg.load_library()
     torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = RankGroup("nccl", torch.device("cuda", local))
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     c = dict(synthetic.CONFIGS[WORKLOAD])
     if args.heads > 0:
         c["H"] = min(args.heads, c["H"])
     L, H, d, g, top_k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
-    q_np, k_np = synthetic.gen_prefill(L, H, d, c["seed"] + rank, c["rho"], c["heavy_frac"], c["heavy_scale"])
+    q_np, k_np = synthetic.gen_prefill(L, H, d, rank_seed(c["seed"], rank), c["rho"], c["heavy_frac"], c["heavy_scale"])
     q = torch.from_numpy(q_np.view(np.int16)).cuda().view(torch.bfloat16)
     k = torch.from_numpy(k_np.view(np.int16)).cuda().view(torch.bfloat16)
     out = torch.empty((L, H, top_k), dtype=torch.int32, device="cuda")
@@ -287,7 +318,7 @@ def main():
     clk = clocks.stop()
     flags = qg.sync_status()
     ms_max = max_over_ranks(ms)
-    value = world * L * H / (ms_max / 1000.0)
+    value = weak_value(world, L, H, ms_max)
 
     # roofline of the dominant kernel
     pk = peaks()
@@ -345,7 +376,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps)
-        e2e = {"value": world * L * H / (e2e_ms / 1000.0), "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e = {"value": weak_value(world, L, H, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(q.numel() * 2 + k.numel() * 2),
                "d2h_bytes_per_step": int(out.numel() * 4), "pinned_output": pinned}
         del q_h, k_h, out_h, q_d, k_d
@@ -383,7 +414,7 @@ def main():
         del out_dense
         # MTP decode workload: one step over 64 sequences (keys drawn on the device)
         dc = synthetic.CONFIGS["C4"]
-        dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], dc["seed"] + rank,
+        dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], rank_seed(dc["seed"], rank),
                                                          dc["lo"], dc["hi"], dc["rho"], dc["heavy_frac"],
                                                          dc["heavy_scale"])
         max_seqlen = int((n_ctx + dc["g"]).max())
@@ -425,9 +456,7 @@ def main():
                 "roofline": roof, "scan_tflops": scan_tf, "kernels": kern, "gpu_launches": gpu_launches,
                 "status_flags": flags, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "extras": extras}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 if __name__ == "__main__":
