@@ -18,7 +18,8 @@ struct FinalizeParams {
   int G, L, H, g, bound_kind;
   int K_sel;       // keys kept per row
   int cap;         // spill capacity per row
-  int width;       // output row width (Kc for candidate rows, top_k for index rows)
+  int width;       // output row width: top_k for index rows; for candidate
+                   // rows the row stride, cand_row_words(K_sel)
   int broadcast;   // 0: write the candidate row; 1: write the row to every member's output row
   const uint2* spill;
   const int2* cnt;   // per row: entries stored upward from slot 0, and downward from slot cap-1
@@ -39,12 +40,13 @@ constexpr int kFinNT = 256;
 constexpr int kFbNT = 512;
 
 // Copies the K selected key indices (staged in shared memory) to their
-// destination row(s), coalesced, with -1 padding to `width`.
+// destination: a candidate row in the refine kernel's order (`stage` holds
+// cand_row_words(K) scratch words), or every member's index row, coalesced,
+// with -1 padding to `width`.
 __device__ __forceinline__ void write_rows(const FinalizeParams& p, int h, int i, const int32_t* sel,
-                                           const uint32_t* selk, int K) {
+                                           const uint32_t* selk, int K, int32_t* stage) {
   if (!p.broadcast) {
-    int32_t* dst = p.cand + (static_cast<long long>(h) * p.G + i) * p.width;
-    for (int t = threadIdx.x; t < p.width; t += blockDim.x) dst[t] = t < K ? sel[t] : -1;
+    write_cand_row(p.cand + (static_cast<long long>(h) * p.G + i) * p.width, sel, K, stage);
     return;
   }
   const int s = i * p.g, e = min(s + p.g, p.L);
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
       },
       sm);
   __syncthreads();
-  write_rows(p, h, i, sel, selk, K);
+  write_rows(p, h, i, sel, selk, K, reinterpret_cast<int32_t*>(ent));  // the entries are no longer needed
 }
 
 // Exact path for rows the filter could not settle: recompute the row's scores
@@ -106,6 +108,7 @@ __global__ void __launch_bounds__(kFbNT) fallback_kernel(FinalizeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   int32_t* sel = reinterpret_cast<int32_t*>(smem_raw);
   uint32_t* selk = reinterpret_cast<uint32_t*>(sel + p.K_sel);
+  int32_t* stage = reinterpret_cast<int32_t*>(selk + p.K_sel);   // cand_row_words(K_sel) words
   uint32_t* sc = p.fb_scratch + static_cast<long long>(blockIdx.x) * p.L;
   const int total = *p.fb_count;
   if (blockIdx.x == 0 && threadIdx.x == 0 && total > 0) atomicOr(p.status, kStFallback);
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kFbNT) fallback_kernel(FinalizeParams p) {
         },
         sm);
     __syncthreads();
-    write_rows(p, h, i, sel, selk, K);
+    write_rows(p, h, i, sel, selk, K, stage);
   }
 }
 

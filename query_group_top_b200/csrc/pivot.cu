@@ -201,7 +201,7 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   p.off_fbscratch = o;
   o += up(static_cast<size_t>(p.nfb) * L * sizeof(uint32_t));
   p.off_cand = o;
-  o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(H) * p.G * Kc * sizeof(int32_t)) : 0;
+  o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(H) * p.G * cand_row_words(Kc) * sizeof(int32_t)) : 0;
   p.total = o;
   return p;
 }
@@ -317,12 +317,13 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     fp.bound_kind = sp.bound_kind;
     fp.K_sel = pl.K_sel;
     fp.cap = pl.cap;
-    fp.width = refine ? Kc : top_k;
+    fp.width = refine ? cand_row_words(Kc) : top_k;
     fp.broadcast = refine ? 0 : 1;
     fp.spill = sp.spill;
     fp.cnt = sp.cnt;
     // Head-local row ids: shift the output bases by h0 heads.
-    fp.cand = refine ? reinterpret_cast<int32_t*>(w + pl.off_cand) + static_cast<size_t>(h0) * pl.G * Kc : nullptr;
+    fp.cand = refine ? reinterpret_cast<int32_t*>(w + pl.off_cand) + static_cast<size_t>(h0) * pl.G * cand_row_words(Kc)
+                     : nullptr;
     fp.out = refine ? nullptr : out + static_cast<size_t>(h0) * top_k;
     fp.out_scores = (refine || !out_scores) ? nullptr : out_scores + static_cast<size_t>(h0) * top_k;
     fp.fb_list = reinterpret_cast<int*>(w + pl.off_fblist);
@@ -340,7 +341,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
       finalize_kernel<<<static_cast<unsigned>(nh * pl.G), kFinNT, fin_smem, st>>>(fp);
     }
     CUDA_TRY(cudaGetLastError());
-    const int fb_smem = pl.K_sel * 8;
+    const int fb_smem = pl.K_sel * 8 + cand_row_words(pl.K_sel) * 4;
     CUDA_TRY(cudaFuncSetAttribute(fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fb_smem));
     {
       TraceScope tr("fallback", st);
@@ -375,7 +376,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
 size_t decode_ws_size(int B, int H, int d, int Kc, int mode, int max_seqlen) {
   size_t o = up(static_cast<size_t>(B) * H * d * 2);                        // proxies
   o += up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t));       // order keys
-  if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(H) * B * Kc * sizeof(int32_t));
+  if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
   return o;
 }
 
@@ -437,7 +438,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     decode_scan_kernel<64><<<grid, kDecNT, 0, st>>>(dp);
   }
   CUDA_TRY(cudaGetLastError());
-  const int sel_smem = dp.K_sel * 8;
+  const int sel_smem = dp.K_sel * 8 + cand_row_words(dp.K_sel) * 4;
   CUDA_TRY(cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem));
   {
     TraceScope tr("decode_select", st);

@@ -62,7 +62,7 @@ struct DecodeParams {
   const uint16_t* P;        // [B][H][d] proxies
   const int32_t* cu;        // [B+1]
   uint32_t* scores;         // [H*B][max_seqlen] order keys
-  int32_t* cand;            // [H][B][width] (Refine)
+  int32_t* cand;            // [H][B][cand_row_words(K_sel)] candidate rows (Refine)
   int32_t* out;             // [B][g][H][width] (Reuse)
   float* out_scores;        // [B][g][H][width] or null (Reuse)
   int B, H, d, g;
@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(kDecSelNT) decode_select_kernel(DecodeParams p
       sm);
   __syncthreads();
   if (p.mode == 0) {
-    int32_t* dst = p.cand + (static_cast<long long>(h) * p.B + b) * p.width;
-    for (int t = threadIdx.x; t < p.width; t += kDecSelNT) dst[t] = t < K ? sel[t] : -1;
+    // stage: the cand_row_words(K_sel) words after sel and selk
+    write_cand_row(p.cand + (static_cast<long long>(h) * p.B + b) * cand_row_words(p.K_sel), sel, K,
+                   reinterpret_cast<int32_t*>(selk + p.K_sel));
   } else {
     for (int m = 0; m < p.g; ++m) {
       int32_t* dst = p.out + ((static_cast<long long>(b) * p.g + m) * p.H + h) * p.width;

@@ -98,6 +98,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm,
       "l"(tm), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// Contiguous bulk copy global -> shared (16-byte aligned addresses, size a
+// multiple of 16), completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tm) : "memory");
 }
@@ -231,6 +238,11 @@ __device__ __forceinline__ void red_shared_max(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
+// Arrive on `bar` once every cp.async this thread has issued so far has
+// landed (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -251,6 +263,30 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred
 }
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ candidate rows
+// Candidate rows are stored in the order the refine kernel reads them.  A row
+// of n candidates (ascending key indices) has nch = ceil(n / 128) chunks;
+// candidate t = r*nch + c (r < 128, c < nch) sits at word c*128 + ((r+c) & 127)
+// of the row, so that both a chunk (fixed c) and a thread's block (fixed r)
+// are free of shared-memory bank conflicts.  Words of slots t >= n hold -1.
+// A row's stride is cand_row_words(Kc).
+__host__ __device__ inline int cand_row_words(int Kc) { return (Kc + 127) / 128 * 128; }
+__host__ __device__ inline int cand_word(int t, int nch) {
+  const int r = t / nch, c = t - r * nch;
+  return c * 128 + ((r + c) & 127);
+}
+// Writes the n selected key indices sel[0..n) as a candidate row at dst,
+// staging the reordering in shared memory `stage` (cand_row_words(n) words);
+// the whole block calls it.
+__device__ inline void write_cand_row(int32_t* __restrict__ dst, const int32_t* sel, int n, int32_t* stage) {
+  if (n <= 0) return;
+  const int nch = (n + 127) / 128, words = nch * 128;
+  __syncthreads();
+  for (int t = threadIdx.x; t < words; t += blockDim.x) stage[cand_word(t, nch)] = t < n ? sel[t] : -1;
+  __syncthreads();
+  for (int w = threadIdx.x; w < words; w += blockDim.x) dst[w] = stage[w];
 }
 
 // ------------------------------------------------------------------ score keys

@@ -9,10 +9,11 @@
 // (unit = (group, head), in batches of up to 16 members) with three roles
 // that run concurrently, so that one unit's selection overlaps the next
 // unit's gather and MMAs:
-//  * producers (warps 0-2) stage the unit's candidate list in shared memory
+//  * producers (warps 0-2) fetch the unit's candidate row with one bulk copy
 //    and gather the candidate keys 128 rows per chunk with 16-byte cp.async
 //    into the 128-byte-swizzled K-major layout (plus the member queries as the
-//    B operand); a stage is handed over on an mbarrier once it has landed;
+//    B operand); each thread's arrival on the stage's mbarrier fires once its
+//    copies have landed;
 //  * the MMA warp (warp 3) issues tcgen05.mma with M = 128 candidate rows,
 //    N = 16 member queries, K = d, into TMEM columns [16c, 16c+16) for chunk
 //    c, and signals "chunk c scored" on a per-chunk mbarrier;
@@ -50,7 +51,7 @@ namespace pivot {
 struct RefineParams {
   const uint16_t* q;      // prefill [L][H][d]; decode [B][g][H][d]
   const uint16_t* keys;   // prefill [L][H][d]; decode packed cache [rows][H][d]
-  const int32_t* cand;    // [H][G][Kc], ascending, -1 padded
+  const int32_t* cand;    // [H][G][cand_row_words(Kc)] candidate rows in read order (ptx.cuh)
   int32_t* out;           // prefill [L][H][top_k]; decode [B][g][H][top_k]
   float* out_scores;      // same shape as out, or null
   const int32_t* cu;      // decode: [B+1] cache row offsets; null for prefill
@@ -115,8 +116,6 @@ struct RefineCfg {
   static constexpr int NSEL = 512;
   static constexpr int NT = 640;
   static constexpr int NS = 4;                          // gather stages
-  static constexpr int LA = 3;                          // chunks in flight before a stage is handed over
-  static_assert(LA <= NS - 1, "a stage is handed over before its producer waits for it again");
   static constexpr int KATOMS = D / 64;
   static constexpr int ATOM_A = 128 * 128;              // 128 rows x 128 bytes
   static constexpr int STAGE = KATOMS * ATOM_A;
@@ -267,7 +266,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       mbar_init(smem_u32(&M->empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&M->cready[b]), C::NPROD);
+      mbar_init(smem_u32(&M->cready[b]), 1);
       mbar_init(smem_u32(&M->cfree[b]), C::NSEL / 32);
     }
     for (int c = 0; c < 32; ++c) {
@@ -289,42 +288,36 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 
   if (warp < C::MMA_WARP) {
     // ======================================================== producers
+    // Thread 0 fetches each unit's candidate row (stored in this kernel's
+    // read order) with one bulk copy; then all 96 producer threads gather the
+    // candidate key rows of each chunk with 16-byte cp.async into the
+    // 128-byte-swizzled K-major layout, and each thread's arrival on the
+    // stage's "full" barrier fires once its own copies have landed, so no
+    // producer ever waits for a copy before issuing the next chunk.
     const int pt = tid;
     int sseq = 0;     // chunks issued so far (all items)
-    int handed = 0;   // chunks handed over to the MMA warp so far
     int kk = 0;       // items processed so far
     bool ok = true;
+    constexpr int RSTEP = C::NPROD / 8;
+    const int p8 = pt & 7, rr0 = pt >> 3;   // 16-byte piece p8 (of each K atom) of rows rr0, rr0 + RSTEP, ...
+    const long long rowstride = static_cast<long long>(p.H) * D;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
       const RefineItem it = refine_item(p, item);
       if (it.nb <= 0) continue;
       const int buf = kk & 1;
-      int32_t* cx = cidx0 + buf * CW;
-      // hand over what is still in flight before the next list is read
-      if (handed < sseq) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        for (; handed < sseq; ++handed) mbar_arrive(smem_u32(&M->full[handed % C::NS]));
-      }
-      if (kk >= 2 && ok)
+      const int32_t* cx = cidx0 + buf * CW;
+      const uint32_t cbar = smem_u32(&M->cready[buf]);
+      // the list and B buffers of this parity are free once the select warps
+      // are done with the item two back
+      if (kk >= 2 && ok && warp == 0)
         ok = mbar_wait(smem_u32(&M->cfree[buf]), ((kk >> 1) - 1) & 1, abort_flag, p.status, 256);
-      if (ok) {
-        // the unit's candidate list, transposed on the fly; all copies in flight at once
-        const int32_t* crow = p.cand + (static_cast<long long>(it.h) * p.G + it.u) * p.Kc;
-        for (int t = pt; t < it.nch * 128; t += C::NPROD) {
-          const int rr = t / it.nch, c = t - rr * it.nch;
-          if (t < it.nc) cp_async_4(smem_u32(cx + cidx_pos(c, rr)), crow + t);
-          else cx[cidx_pos(c, rr)] = -1;
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
+      ok = !named_barrier_or(1, C::NPROD, !ok);
+      if (ok && pt == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(it.nch) * 128u * 4u;
+        mbar_arrive_expect_tx(cbar, bytes);
+        if (bytes) bulk_copy_g2s(smem_u32(cx), p.cand + (static_cast<long long>(it.h) * p.G + it.u) * CW, bytes, cbar);
       }
-      named_barrier(1, C::NPROD);
-      mbar_arrive(smem_u32(&M->cready[buf]));
-      // this thread copies the 16-byte pieces p8, p8 + 8, ... (one per K atom,
-      // same swizzle) of rows rr0, rr0 + RSTEP, ...
-      constexpr int RSTEP = C::NPROD / 8;
-      const int p8 = pt & 7, rr0 = pt >> 3;
-      const long long rowstride = static_cast<long long>(p.H) * D;
+      if (ok) ok = mbar_wait(cbar, (kk >> 1) & 1, abort_flag, p.status, 128);
       const uint16_t* kbase = p.keys + (it.key_row0 * p.H + it.h) * static_cast<long long>(D) + p8 * 8;
       const uint32_t bB = sB + buf * C::B_BYTES;
       for (int c = 0; c < it.nch; ++c) {
@@ -340,7 +333,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             const int j = cxc[(rr + c) & 127];
             const uint16_t* src = kbase + max(j, 0) * rowstride;
             const uint32_t dst = dst0 + rr * 128 + ((p8 ^ (rr & 7)) << 4);
-            const uint32_t nbytes = j >= 0 ? 16u : 0u;
+            const uint32_t nbytes = j >= 0 ? 16u : 0u;   // a missing candidate reads as zeros
 #pragma unroll
             for (int a = 0; a < C::KATOMS; ++a) cp_async_16(dst + a * C::ATOM_A, src + a * 64, nbytes);
           }
@@ -348,30 +341,24 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             // member queries of this batch -> B operand, zero rows past nb
             for (int id = pt; id < 16 * (D / 8); id += C::NPROD) {
               const int rr = id / (D / 8), piece = id % (D / 8);
-              const int a = piece >> 3, p8 = piece & 7;
+              const int a = piece >> 3, q8 = piece & 7;
               const bool real = rr < it.nb;
               const uint16_t* src =
                   p.q + (real ? ((it.qrow0 + it.mb + rr) * p.H + it.h) * static_cast<long long>(D) + piece * 8 : 0);
-              cp_async_16(bB + a * C::ATOM_B + rr * 128 + ((p8 ^ (rr & 7)) << 4), src, real ? 16u : 0u);
+              cp_async_16(bB + a * C::ATOM_B + rr * 128 + ((q8 ^ (rr & 7)) << 4), src, real ? 16u : 0u);
             }
           }
+          cp_async_arrive_noinc(smem_u32(&M->full[s]));
         }
-        cp_async_commit();
         ++sseq;
-        if (sseq - handed > C::LA) {
-          // the oldest chunk in flight has landed: hand its stage over
-          cp_async_wait<C::LA>();
-          fence_proxy_async_smem();
-          mbar_arrive(smem_u32(&M->full[handed % C::NS]));
-          ++handed;
-        }
       }
       ++kk;
       if (named_barrier_or(1, C::NPROD, !ok)) break;
     }
+    // never leave the CTA with a copy still landing in its shared memory
     cp_async_wait<0>();
-    fence_proxy_async_smem();
-    for (; handed < sseq; ++handed) mbar_arrive(smem_u32(&M->full[handed % C::NS]));
+    if (pt == 0)
+      for (int q = max(0, kk - 2); q < kk; ++q) mbar_wait_cleanup(smem_u32(&M->cready[q & 1]), (q >> 1) & 1);
   } else if (warp == C::MMA_WARP) {
     // ======================================================== MMA issuer
     constexpr uint32_t idesc = umma_idesc_bf16(128, 16);
@@ -391,6 +378,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           ok = __all_sync(0xffffffffu, ok);
           if (ok && lane == 0) {
             tc_fence_after();
+            // the stage was written by other threads' cp.async (generic proxy)
+            // and is read by the MMAs (async proxy)
+            fence_proxy_async_smem();
 #pragma unroll
             for (int kq = 0; kq < D / 16; ++kq) {
               const int a = kq >> 2, k4 = kq & 3;
@@ -1016,6 +1006,13 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         }
         for (int x = K + r; x < p.top_k; x += 128) orow[x] = -1;
       }
+      // Chunks past this item's list got their "scored" commit without MMAs.
+      // Wait for those commits too before giving the chunks back: every
+      // release then answers a commit of this item, and the MMA warp can never
+      // find a chunk's "free" barrier two phases ahead of its wait.
+      for (int c = nch; c < NCH; ++c)
+        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+      ok = __all_sync(0xffffffffu, ok);
       // this item's TMEM columns and candidate list are free
       release_upto(NCH);
       __syncwarp();
