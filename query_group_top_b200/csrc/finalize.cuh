@@ -22,7 +22,7 @@ struct FinalizeParams {
                    // rows the row stride, cand_row_words(K_sel)
   int broadcast;   // 0: write the candidate row; 1: write the row to every member's output row
   const uint2* spill;
-  const int2* cnt;   // per row: entries stored upward from slot 0, and downward from slot cap-1
+  const int4* cnt;   // per row: the four runs' entry counts (layout in ScanParams)
   int32_t* cand;   // [H*G][width] when broadcast == 0
   int32_t* out;    // [L][H][width] when broadcast == 1
   float* out_scores;  // [L][H][width] or null (broadcast == 1 only)
@@ -36,7 +36,7 @@ struct FinalizeParams {
   uint32_t* fb_scratch;   // [gridDim.x][L] order keys
 };
 
-constexpr int kFinNT = 256;
+constexpr int kFinNT = 512;
 constexpr int kFbNT = 512;
 
 // Copies the K selected key indices (staged in shared memory) to their
@@ -74,20 +74,32 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
   sp.G = p.G; sp.L = p.L; sp.g = p.g; sp.bound_kind = p.bound_kind;
   const int bound = row_bound(sp, i);
   const int K = min(p.K_sel, bound);
-  const int2 c2 = p.cnt[row_id];
-  const int n = c2.x + c2.y;
-  if (n > p.cap || (bound > p.cap && n < K)) {
+  const int4 c4 = p.cnt[row_id];
+  const int capH = p.cap / 2;
+  const int n = c4.x + c4.y + c4.z + c4.w;
+  // a spill region that overflowed, or too few survivors of a thresholded row
+  if (c4.x + c4.y > capH || c4.z + c4.w > capH || (bound > capH && n < K)) {
     if (threadIdx.x == 0) {
       const int slot = atomicAdd(p.fb_count, 1);
       p.fb_list[slot] = static_cast<int>(row_id);
     }
     return;
   }
-  // the upward run (lower key indices) first, then the downward run reversed:
-  // entries in ascending key-index order
-  const int nn = n;
+  // runs 0..3 cover ascending quarters of the keys; odd runs were stored
+  // downward from the end of their region: copied in this order, the entries
+  // are in ascending key-index order.  Every copy of the row is in flight at
+  // once; then the scores become order keys.
   const uint2* src = p.spill + row_id * p.cap;
-  for (int e = threadIdx.x; e < nn; e += kFinNT) ent[e] = e < c2.x ? src[e] : src[p.cap - 1 - (e - c2.x)];
+  const int o1 = c4.x, o2 = o1 + c4.y, o3 = o2 + c4.z;
+  for (int e = threadIdx.x; e < n; e += kFinNT) {
+    const int at = e < o1 ? e : (e < o2 ? capH - 1 - (e - o1) : (e < o3 ? capH + (e - o2) : p.cap - 1 - (e - o3)));
+    cp_async_8(smem_u32(&ent[e]), src + at);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += kFinNT) ent[e].x = score_key(__uint_as_float(ent[e].x));
+  const int nn = n;
   __syncthreads();
   block_select_emit<kFinNT>(
       nn, K, [&](int e) { return ent[e].x; },

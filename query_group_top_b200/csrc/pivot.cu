@@ -168,10 +168,11 @@ struct Plan {
 // Sample stride and spill capacity for a select of K_sel keys per row over
 // prefixes up to L keys.
 void filter_shape(int K_sel, int L, int* cap, int* S) {
-  const int BN = 256;
-  int c = std::max(2 * K_sel, 2 * BN);
+  const int BN = 128;  // keys per scan tile
+  int c = std::max(2 * K_sel, 4 * BN);
   int s = std::max(1, std::min(16, c / BN));
-  const int min_s = (L + BN * 255 - 1) / (BN * 255);  // at most 255 sampled tiles per row
+  // at most 511 sampled tiles per row, so a row's sample fits 16-bit bin counts
+  const int min_s = (L + BN * 511 - 1) / (BN * 511);
   s = std::max(s, min_s);
   c = std::max(c, s * BN);
   *cap = (c + 7) / 8 * 8;
@@ -193,7 +194,7 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   p.off_spill = o;
   o += up(rows_pass * p.cap * sizeof(uint2));
   p.off_cnt = o;
-  o += up(rows_pass * sizeof(int2));
+  o += up(rows_pass * sizeof(int4));
   p.off_fb = o;
   o += up(sizeof(int));
   p.off_fblist = o;
@@ -292,7 +293,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     const uint16_t* Kh = static_cast<const uint16_t*>(k) + static_cast<size_t>(h0) * d;
     CUtensorMap tmP, tmK;
     if (int rc = make_rows_map(&tmP, Ph, pl.G, nh, H, d, 128)) return rc;
-    if (int rc = make_rows_map(&tmK, Kh, L, nh, H, d, 256)) return rc;
+    if (int rc = make_rows_map(&tmK, Kh, L, nh, H, d, ScanCfg<128>::BN)) return rc;
     ScanParams sp{};
     sp.G = pl.G;
     sp.L = L;
@@ -302,9 +303,9 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     sp.K_sel = pl.K_sel;
     sp.cap = pl.cap;
     sp.S = pl.S;
-    sp.tiles_per_head = (pl.G + 127) / 128;
+    sp.tiles_per_head = (pl.G + ScanCfg<128>::BM - 1) / ScanCfg<128>::BM;
     sp.spill = reinterpret_cast<uint2*>(w + pl.off_spill);
-    sp.cnt = reinterpret_cast<int2*>(w + pl.off_cnt);
+    sp.cnt = reinterpret_cast<int4*>(w + pl.off_cnt);
     sp.status = dev->status;
     int rc = (d == 128) ? launch_scan<128>(tmP, tmK, sp, nh, st) : launch_scan<64>(tmP, tmK, sp, nh, st);
     if (rc) return rc;
