@@ -73,7 +73,9 @@ enum : int {
   kMTies = 6,    // boundary keys all equal: the first need_eq in order
 };
 
-constexpr int kRefBins = 1024;
+constexpr int kRefBins = 512;
+// 2^23: a float in [2^23, 2^24) is an integer, held in its low mantissa bits
+constexpr float kMagic = 8388608.0f;
 constexpr int kListCap = 256;
 // Each key-linear round shrinks a boundary's key range by a factor of about
 // 256, so 32-bit keys need at most five rounds after round 0.
@@ -124,10 +126,10 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
   static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
-  // histograms: 16 members x 1024 bins of 16-bit counts (two per word); the
-  // same bytes later hold the boundary lists, and together with the decision
-  // bitmaps that follow them, the per-warp output staging
-  static constexpr int HIST_BYTES = 16 * (kRefBins / 2) * 4;
+  // histograms: 16 members x 512 bins of 32-bit counts; the same bytes later
+  // hold the boundary lists, and together with the decision bitmaps that
+  // follow them, the per-warp output staging
+  static constexpr int HIST_BYTES = 16 * kRefBins * 4;
   static_assert(16 * 2 * kListCap * 4 <= HIST_BYTES, "lists alias the histograms");
   // output staging entries per select warp: the histogram and bitmap bytes
   __host__ __device__ static int stg_entries(int Kc) { return (HIST_BYTES / 4 + 16 * 2 * bm_words(Kc)) / 16; }
@@ -149,13 +151,16 @@ __device__ __forceinline__ int key_bin(uint32_t key, uint32_t lo, float scale) {
   return static_cast<int>(min(b, static_cast<uint32_t>(kRefBins - 1)));
 }
 
-// Linear bin of a score, trunc(s * scale + off) clamped to [0, 511]: one
-// rounding (the fma) of a function increasing in s, so the bins are ordered
-// like the scores, and -0 and +0 share a bin.  Scores of real data spread
-// evenly over such bins, while the order keys of scores on both sides of zero
-// crowd into a few of the key-linear ones.
-__device__ __forceinline__ int value_bin(float s, float scale, float off) {
-  return static_cast<int>(min(__float2uint_rz(__fmaf_rn(s, scale, off)), static_cast<uint32_t>(kRefBins - 1)));
+// Linear bin of a score, round(s * scale + off) clamped to [0, 511], with
+// offm = off + 2^23 (as a float): the fma rounds s*scale + offm to an integer
+// in [2^23, 2^23 + 511] after the clamps, and the bin is its low mantissa
+// bits.  One rounding of a function increasing in s, then monotone clamps, so
+// the bins are ordered like the scores, and -0 and +0 share a bin.  Scores of
+// real data spread evenly over such bins, while the order keys of scores on
+// both sides of zero crowd into a few of the key-linear ones.
+__device__ __forceinline__ int value_bin(float s, float scale, float offm) {
+  const float t = fminf(fmaxf(__fmaf_rn(s, scale, offm), kMagic), kMagic + static_cast<float>(kRefBins - 1));
+  return static_cast<int>(__float_as_uint(t) & static_cast<uint32_t>(kRefBins - 1));
 }
 
 // Bin of an order key under either bin function; key patterns beyond the
@@ -174,7 +179,9 @@ __device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float 
   if (bin_of_key(0xFFFFFFFFu, lo, scale, off, vmode) < b) return false;
   uint32_t guess;
   if (vmode) {
-    guess = score_key(__fdiv_rn(__fsub_rn(static_cast<float>(b), off), scale));
+    // the score where round(s * scale + offm) reaches 2^23 + b
+    guess = score_key(static_cast<float>((static_cast<double>(kMagic) + b - 0.5 - static_cast<double>(off)) /
+                                         static_cast<double>(scale)));
   } else {
     const float dk = __fdiv_rn(static_cast<float>(b), scale);
     guess = dk >= 4294967040.0f ? 0xFFFFFFFFu : lo + min(__float2uint_rz(dk), 0xFFFFFFFFu - lo);
@@ -498,7 +505,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           }
           const float vmin = key_score(mn), vmax = key_score(mx);
           const float vsc = static_cast<float>(kRefBins) / __fsub_rn(vmax, vmin);
-          const float voff = __fmul_rn(-vmin, vsc);
+          const float voff = __fadd_rn(__fmul_rn(-vmin, vsc), kMagic);   // offset + 2^23
           const bool vm = mn < mx && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f && isfinite(voff);
           if (vm) {
             ob4[i] = __float_as_uint(voff);
@@ -519,17 +526,30 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           }
         }
       };
+      // shared-memory address of this thread's members' histograms
+      uint32_t hrow[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hrow[i] = smem_u32(hist + (4 * grp + i) * kRefBins);
+      // chunks where all four members count every score of this thread's block
+      uint32_t allc = 0;
       auto hist_chunk = [&](int c) {
         uint32_t v[4];
         tmem_ld_32x32b_x4(tl + c * 16, v);
         tmem_ld_wait();
-        if (vm4 == hm) {  // every counted member has score-linear bins (the rule)
+        if ((allc >> c) & 1u) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            reg_fence(v[i]);
+            const int b = value_bin(__uint_as_float(v[i]), sc4[i], __uint_as_float(ob4[i]));
+            red_shared_add(hrow[i] + 4u * b, 1u);
+          }
+        } else if (vm4 == hm) {  // every counted member has score-linear bins (the rule)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             reg_fence(v[i]);
             const bool cnt = ((hm >> i) & (um[i] >> c) & 1u) != 0u;
             const int b = value_bin(__uint_as_float(v[i]), sc4[i], __uint_as_float(ob4[i]));
-            if (cnt) red_shared_add(smem_u32(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)]), 1u << ((b & 1) << 4));
+            if (cnt) red_shared_add(hrow[i] + 4u * b, 1u);
           }
         } else {
 #pragma unroll
@@ -539,7 +559,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               const float f = __uint_as_float(v[i]);
               const int b = ((vm4 >> i) & 1u) ? value_bin(f, sc4[i], __uint_as_float(ob4[i]))
                                               : key_bin(score_key(f), ob4[i], sc4[i]);
-              red_shared_add(smem_u32(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)]), 1u << ((b & 1) << 4));
+              red_shared_add(hrow[i] + 4u * b, 1u);
             }
           }
         }
@@ -556,6 +576,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           } else {
             if (c == 1) {
               set_range();
+              allc = (hm == 0xFu && vm4 == 0xFu) ? (um[0] & um[1] & um[2] & um[3]) : 0u;
               hist_chunk(0);
             }
             hist_chunk(c);
@@ -565,6 +586,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       }
       if (ok && nch == 1 && hm != 0) {
         set_range();
+        allc = (hm == 0xFu && vm4 == 0xFu) ? (um[0] & um[1] & um[2] & um[3]) : 0u;
         hist_chunk(0);
       }
       if (named_barrier_or(2, C::NSEL, !ok)) break;
@@ -594,17 +616,15 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         // (a) warp sw: boundary bin and key thresholds of member sw
         if (sw < nb && M->ms[sw].active) {
           MemberSel& S = M->ms[sw];
-          const uint32_t* hw = hist + sw * (kRefBins / 2);
+          const uint32_t* hw = hist + sw * kRefBins;
           const int need = S.need;
-          // lane l owns words [512 - 16(l+1), 512 - 16l), i.e. 32 bins, in
-          // descending order by lane; a word holds bins 2w (low half) and 2w+1
-          const int w0 = kRefBins / 2 - 16 * (lane + 1);
+          // lane l owns bins [512 - 16(l+1), 512 - 16l), in descending order by lane
+          const int b0 = kRefBins - 16 * (lane + 1);
           int s = 0;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint4 x = reinterpret_cast<const uint4*>(hw + w0)[(i + lane) & 3];
-            s += static_cast<int>((x.x & 0xFFFFu) + (x.x >> 16) + (x.y & 0xFFFFu) + (x.y >> 16) + (x.z & 0xFFFFu) +
-                                  (x.z >> 16) + (x.w & 0xFFFFu) + (x.w >> 16));
+            const uint4 x = reinterpret_cast<const uint4*>(hw + b0)[(i + lane) & 3];
+            s += static_cast<int>(x.x + x.y + x.z + x.w);
           }
           int incl = s;
 #pragma unroll
@@ -616,12 +636,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
           const int L = hit ? __ffs(hit) - 1 : 31;
           const int exclL = __shfl_sync(0xffffffffu, incl - s, L);
-          // lane i < 16: word (512 - 16L - 1 - i), bins 2w+1 then 2w
-          const int w = kRefBins / 2 - 16 * L - 1 - lane;
-          const uint32_t wv = lane < 16 ? hw[w] : 0u;
-          const int chi = static_cast<int>(wv >> 16), clo = static_cast<int>(wv & 0xFFFFu);
-          const int s2 = chi + clo;
-          int incl2 = s2;
+          // lane i < 16: bin 512 - 16L - 1 - i
+          const int cb = lane < 16 ? static_cast<int>(hw[kRefBins - 16 * L - 1 - lane]) : 0;
+          int incl2 = cb;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, incl2, o);
@@ -629,13 +646,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           }
           const unsigned hit2 = __ballot_sync(0xffffffffu, exclL + incl2 >= need);
           const int i2 = hit2 ? __ffs(hit2) - 1 : 15;
-          const int before = __shfl_sync(0xffffffffu, exclL + incl2 - s2, i2);
-          const int hi2 = __shfl_sync(0xffffffffu, chi, i2), lo2 = __shfl_sync(0xffffffffu, clo, i2);
-          const int w2 = kRefBins / 2 - 16 * L - 1 - i2;
-          const bool upper = before + hi2 >= need;
-          const int bstar = upper ? 2 * w2 + 1 : 2 * w2;
-          const int above = upper ? before : before + hi2;
-          const int cntb = upper ? hi2 : lo2;
+          const int above = __shfl_sync(0xffffffffu, exclL + incl2 - cb, i2);
+          const int cntb = __shfl_sync(0xffffffffu, cb, i2);
+          const int bstar = kRefBins - 16 * L - 1 - i2;
           const uint32_t lo = S.lo;
           const float sc = S.scale, off = S.off;
           const bool vm = S.vmode != 0;
@@ -862,7 +875,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               reg_fence(v[i]);
               if ((c4[i] >> c) & 1u) {
                 const int b = key_bin(score_key(__uint_as_float(v[i])), lo_[i], sc_[i]);
-                red_shared_add(smem_u32(&hist[(4 * grp + i) * (kRefBins / 2) + (b >> 1)]), 1u << ((b & 1) << 4));
+                red_shared_add(hrow[i] + 4u * b, 1u);
               }
             }
           }
