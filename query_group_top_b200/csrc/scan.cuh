@@ -243,6 +243,8 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
     const int dir = (e & 1) ? -1 : 1;
     int cnt = 0;
     float tau = -__int_as_float(0x7f800000);    // -inf: keep everything
+    // the largest float below tau: for finite scores, v >= tau <=> v > tau_below
+    float tau_below = tau;
     int n_sample = 0;
     int b1 = -1, rem = 0;
     const bool row_samples = sampling && bound > capH;
@@ -300,6 +302,10 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
               cum += cb;
             }
             tau = key_lower_edge_value((static_cast<uint32_t>(b1) << 24) | (static_cast<uint32_t>(b2) << 16));
+            const uint32_t u = __float_as_uint(tau);
+            if (tau == -__int_as_float(0x7f800000)) tau_below = tau;
+            else if ((u & 0x7FFFFFFFu) == 0u) tau_below = __uint_as_float(0x80000001u);  // below +-0
+            else tau_below = __uint_as_float((u >> 31) ? u + 1u : u - 1u);
           }
           // the main pass reuses the histogram space for staging
           named_barrier(1, C::NEPI);
@@ -317,16 +323,22 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
       if (j0 >= bound) return;
       const uint32_t live = (j0 + C::CW <= bound) ? (0xFFFFFFFFu >> (32 - C::CW)) : ((1u << (bound - j0)) - 1u);
       if (phase == 2) {
-        // four independent compare chains
-        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+        // bit x = (v[x] >= tau) = the sign of tau_below - v[x] (an fadd, on the
+        // FMA pipe), shifted into the mask by one funnel shift; four chains of
+        // four consecutive keys, taken from the top so each bit lands in place
+        uint32_t c4[C::CW / 4];
 #pragma unroll
-        for (int x = 0; x < C::CW; x += 4) {
-          m0 |= (__uint_as_float(v[x]) >= tau ? 1u : 0u) << x;
-          m1 |= (__uint_as_float(v[x + 1]) >= tau ? 2u : 0u) << x;
-          m2 |= (__uint_as_float(v[x + 2]) >= tau ? 4u : 0u) << x;
-          m3 |= (__uint_as_float(v[x + 3]) >= tau ? 8u : 0u) << x;
+        for (int k = 0; k < C::CW / 4; ++k) {
+          uint32_t c = 0;
+#pragma unroll
+          for (int x = 4 * k + 3; x >= 4 * k; --x)
+            c = __funnelshift_l(__float_as_uint(__fsub_rn(tau_below, __uint_as_float(v[x]))), c, 1);
+          c4[k] = c;
         }
-        uint32_t m = (m0 | m1 | m2 | m3) & live;
+        uint32_t m = 0;
+#pragma unroll
+        for (int k = 0; k < C::CW / 4; ++k) m |= c4[k] << (4 * k);
+        m &= live;
         if (m == 0) return;
 #pragma unroll
         for (int q4 = 0; q4 < Q4; ++q4)
