@@ -101,6 +101,33 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
   for (int e = threadIdx.x; e < n; e += kFinNT) ent[e].x = score_key(__uint_as_float(ent[e].x));
   const int nn = n;
   __syncthreads();
+  if (!p.broadcast) {
+    // candidate row: each selected index goes straight to its word of the
+    // row in the refine kernel's read order (no staging, so the kernel needs
+    // only the entries' shared memory); a thread's slots arrive in ascending
+    // order, so their (r, c) position is stepped rather than divided out
+    int32_t* dst = p.cand + row_id * p.width;
+    const int nch = (K + 127) / 128;
+    int last = -2, rr = 0, cc = 0;
+    block_select_emit<kFinNT>(
+        nn, K, [&](int e) { return ent[e].x; },
+        [&](int slot, int e) {
+          if (slot == last + 1) {
+            if (++cc == nch) {
+              cc = 0;
+              ++rr;
+            }
+          } else {
+            rr = slot / nch;
+            cc = slot - rr * nch;
+          }
+          last = slot;
+          dst[cc * 128 + ((rr + cc) & 127)] = static_cast<int32_t>(ent[e].y);
+        },
+        sm);
+    for (int t = K + static_cast<int>(threadIdx.x); t < nch * 128; t += kFinNT) dst[cand_word(t, nch)] = -1;
+    return;
+  }
   block_select_emit<kFinNT>(
       nn, K, [&](int e) { return ent[e].x; },
       [&](int slot, int e) {

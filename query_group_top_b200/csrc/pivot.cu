@@ -335,7 +335,8 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     fp.d = d;
     fp.fb_scratch = reinterpret_cast<uint32_t*>(w + pl.off_fbscratch);
     CUDA_TRY(cudaMemsetAsync(fp.fb_count, 0, sizeof(int), st));
-    const int fin_smem = pl.cap * 8 + pl.K_sel * 8;
+    // candidate rows are written straight from the select; index rows are staged
+    const int fin_smem = pl.cap * 8 + (refine ? 0 : pl.K_sel * 8);
     CUDA_TRY(cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fin_smem));
     {
       TraceScope tr("finalize", st);

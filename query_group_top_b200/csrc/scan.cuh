@@ -82,7 +82,7 @@ struct ScanCfg {
   static constexpr uint32_t TMEM_COLS = NACC * BN;
   static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr int CW = 16;                       // columns per TMEM load (one chunk)
-  static_assert(NACC * (CW / 4) * BM * 16 <= HIST_BYTES, "main-pass staging aliases the histograms");
+  static_assert(NACC * (2 * CW / 4) * BM * 16 <= HIST_BYTES, "main-pass staging (a chunk pair) aliases the histograms");
 };
 
 // The CTA's work, in one order shared by the producer, the MMA issuer and the
@@ -314,57 +314,78 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
       }
     };
 
-    // Main-pass staging for survivor lookups: this thread's CW values of the
-    // current chunk as CW/4 float4 at [((e*CW/4 + i)*128 + r)*4].
-    constexpr int Q4 = C::CW / 4;
+    // Main-pass staging for survivor lookups: this thread's values of a pair
+    // of chunks (2*CW of them) as 2*CW/4 float4 at [((e*Q4 + i)*128 + r)*4].
+    // The survivors of both chunks of a pair go out in one loop, which halves
+    // how often a warp waits for its lane with the most survivors.
+    constexpr int Q4 = 2 * C::CW / 4;
     float* stage = reinterpret_cast<float*>(hist);
     const float* st_r = stage + (static_cast<long long>(e) * Q4 * C::BM + r) * 4;
-    auto process = [&](const uint32_t (&v)[C::CW], int j0, int phase) {
+    uint32_t pend = 0;   // survivors of the pair's first chunk (bits 0..CW-1)
+    // bit x = (v[x] >= tau) = the sign of tau_below - v[x] (an fadd, on the
+    // FMA pipe), shifted into the mask by one funnel shift; four chains of
+    // four consecutive keys, taken from the top so each bit lands in place
+    auto chunk_mask = [&](const uint32_t (&v)[C::CW], uint32_t live) -> uint32_t {
+      uint32_t c4[C::CW / 4];
+#pragma unroll
+      for (int k = 0; k < C::CW / 4; ++k) {
+        uint32_t c = 0;
+#pragma unroll
+        for (int x = 4 * k + 3; x >= 4 * k; --x)
+          c = __funnelshift_l(__float_as_uint(__fsub_rn(tau_below, __uint_as_float(v[x]))), c, 1);
+        c4[k] = c;
+      }
+      uint32_t m = 0;
+#pragma unroll
+      for (int k = 0; k < C::CW / 4; ++k) m |= c4[k] << (4 * k);
+      return m & live;
+    };
+    // survivors of a pair (bit x: key j0 + x) in ascending order, two per
+    // step: (score bits, key index)
+    auto flush = [&](uint32_t m, int j0) {
+      if (cnt + __popc(m) > capH) {
+        // the region is full: only count (the row goes to the exact fallback)
+        cnt += __popc(m);
+        return;
+      }
+      while (m) {
+        const int x1 = __ffs(m) - 1;
+        m &= m - 1;
+        const uint32_t s1 = __float_as_uint(st_r[(x1 >> 2) * (C::BM * 4) + (x1 & 3)]);
+        run[dir * cnt] = make_uint2(s1, static_cast<uint32_t>(j0 + x1));
+        ++cnt;
+        if (m) {
+          const int x2 = __ffs(m) - 1;
+          m &= m - 1;
+          const uint32_t s2 = __float_as_uint(st_r[(x2 >> 2) * (C::BM * 4) + (x2 & 3)]);
+          run[dir * cnt] = make_uint2(s2, static_cast<uint32_t>(j0 + x2));
+          ++cnt;
+        }
+      }
+    };
+    // half: 0 for the first chunk of a pair, 1 for the second (keys j0 - CW ...)
+    auto process = [&](const uint32_t (&v)[C::CW], int j0, int phase, int half) {
+      if (phase == 2) {
+        const uint32_t live =
+            j0 >= bound ? 0u : ((j0 + C::CW <= bound) ? (0xFFFFFFFFu >> (32 - C::CW)) : ((1u << (bound - j0)) - 1u));
+        const uint32_t m = live ? chunk_mask(v, live) : 0u;
+        if (m) {
+#pragma unroll
+          for (int q4 = 0; q4 < C::CW / 4; ++q4)
+            reinterpret_cast<uint4*>(stage)[(e * Q4 + half * (C::CW / 4) + q4) * C::BM + r] =
+                make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        }
+        if (half == 0) {
+          pend = m;
+        } else {
+          const uint32_t mm = pend | (m << C::CW);
+          if (mm) flush(mm, j0 - C::CW);
+        }
+        return;
+      }
       if (j0 >= bound) return;
       const uint32_t live = (j0 + C::CW <= bound) ? (0xFFFFFFFFu >> (32 - C::CW)) : ((1u << (bound - j0)) - 1u);
-      if (phase == 2) {
-        // bit x = (v[x] >= tau) = the sign of tau_below - v[x] (an fadd, on the
-        // FMA pipe), shifted into the mask by one funnel shift; four chains of
-        // four consecutive keys, taken from the top so each bit lands in place
-        uint32_t c4[C::CW / 4];
-#pragma unroll
-        for (int k = 0; k < C::CW / 4; ++k) {
-          uint32_t c = 0;
-#pragma unroll
-          for (int x = 4 * k + 3; x >= 4 * k; --x)
-            c = __funnelshift_l(__float_as_uint(__fsub_rn(tau_below, __uint_as_float(v[x]))), c, 1);
-          c4[k] = c;
-        }
-        uint32_t m = 0;
-#pragma unroll
-        for (int k = 0; k < C::CW / 4; ++k) m |= c4[k] << (4 * k);
-        m &= live;
-        if (m == 0) return;
-#pragma unroll
-        for (int q4 = 0; q4 < Q4; ++q4)
-          reinterpret_cast<uint4*>(stage)[(e * Q4 + q4) * C::BM + r] =
-              make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-        // survivors in ascending order, two per step: (score bits, key index)
-        if (cnt + __popc(m) <= capH) {
-          while (m) {
-            const int x1 = __ffs(m) - 1;
-            m &= m - 1;
-            const uint32_t s1 = __float_as_uint(st_r[(x1 >> 2) * (C::BM * 4) + (x1 & 3)]);
-            run[dir * cnt] = make_uint2(s1, static_cast<uint32_t>(j0 + x1));
-            ++cnt;
-            if (m) {
-              const int x2 = __ffs(m) - 1;
-              m &= m - 1;
-              const uint32_t s2 = __float_as_uint(st_r[(x2 >> 2) * (C::BM * 4) + (x2 & 3)]);
-              run[dir * cnt] = make_uint2(s2, static_cast<uint32_t>(j0 + x2));
-              ++cnt;
-            }
-          }
-        } else {
-          // the region is full: only count (the row goes to the exact fallback)
-          cnt += __popc(m);
-        }
-      } else if (phase == 0) {
+      if (phase == 0) {
 #pragma unroll
         for (int x = 0; x < C::CW; ++x)
           if ((live >> x) & 1u) bin_add(static_cast<int>(score_key(__uint_as_float(v[x])) >> 24));
@@ -403,7 +424,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
 #pragma unroll 1
       for (int c = 0; c < NCK; c += 2) {
         tmem_ld_32x32b_x16(taddr + (c + 1) * C::CW, vb);
-        process(va, jt * C::BN + c * C::CW, phase);
+        process(va, jt * C::BN + c * C::CW, phase, 0);
         tmem_ld_wait();
 #pragma unroll
         for (int x = 0; x < C::CW; ++x) reg_fence(vb[x]);
@@ -414,7 +435,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
           tc_fence_before();
           mbar_arrive(tempty_bar(e));
         }
-        process(vb, jt * C::BN + (c + 1) * C::CW, phase);
+        process(vb, jt * C::BN + (c + 1) * C::CW, phase, 1);
         if (c + 2 < NCK) {
           tmem_ld_wait();
 #pragma unroll
