@@ -128,8 +128,9 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
  * allocator of its own and must not own device buffers.  Its scratch is a
  * 32 MiB array built into the library (held by every GPU that loads it until
  * the process exits); a call whose scratch need -- proxies B*H*d*2 + order keys
- * H*B*max_seqlen*4 + (Refine) candidates H*B*Kc*4 bytes, each rounded up to
- * 256 -- exceeds 32 MiB is rejected with PIVOT_ERR_WORKSPACE and a message.
+ * H*B*max_seqlen*4 + (Refine) candidates H*B*CW*4 bytes, CW = Kc rounded up to
+ * a multiple of 128, each rounded up to 256 -- exceeds 32 MiB is rejected with
+ * PIVOT_ERR_WORKSPACE and a message.
  * The first call on each device looks the array's address up (once, with that
  * device current); make that first call before any stream capture.  All calls
  * share the one array and it keeps the previous call's contents (nothing in it
