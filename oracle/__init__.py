@@ -28,6 +28,10 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 REFINE, REUSE = 0, 1
+# The listing's own Refine ("Show Me The Code", pivot_refine): a proxy scan over
+# each member's own prefix.  Oracle only; it measures what the single-scan
+# reading of Refine changes.
+REFINE_PER_MEMBER = 2
 
 
 def build(force: bool = False) -> str:
@@ -67,7 +71,8 @@ def _u16(a):
 
 
 def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False):
-    """PIVOT (Refine mode=0, Reuse mode=1) on the listed (group, head) units.
+    """PIVOT (Refine mode=0, Reuse mode=1, per-member-scan Refine mode=2) on the
+    listed (group, head) units.
 
     Returns dict: out [n,g,top_k] int32, score [n,g,top_k] f64, edge [n,g,2] f64,
     cand [n,Kc] int32 and cand_edge [n,2] (Refine), proxy [n,d] uint16.

@@ -27,6 +27,11 @@
  *    with the listing's per-member prefix), candidate set C = top-min(Kc,last)
  *    of the proxy scores; member pos keeps V = {j in C : j < pos}, re-scores V
  *    with its own query and keeps top-min(top_k, |V|).
+ *  - The listing's own Refine (mode 2, kept to measure the difference the
+ *    reading above makes): every member re-runs the proxy scan over its own
+ *    prefix j < pos, takes C_pos = top-min(Kc, pos) of it, re-scores C_pos
+ *    with its own query and keeps top-min(top_k, |C_pos|) ("Show Me The
+ *    Code", pivot_refine: the scan k_h[:pos] inside the member loop).
  *  - Reuse: the proxy's top-min(top_k, s) over keys j < s (s = group start,
  *    strictly causal for every member; group 0 gets nothing), shared by all
  *    members.
@@ -137,7 +142,7 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
                      int32_t *cand, double *cand_edge, uint16_t *proxy_out)
 {
     uint16_t *p = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)d);
-    int bound = (mode == 0) ? last : s;
+    int bound = (mode == 1) ? s : last;
     scored_t *sig = (scored_t *)malloc(sizeof(scored_t) * (size_t)(bound > 0 ? bound : 1));
     scored_t *v = (scored_t *)malloc(sizeof(scored_t) * (size_t)(Kc > 0 ? Kc : 1));
     if (!p || !sig || !v) { free(p); free(sig); free(v); return -1; }
@@ -171,6 +176,22 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
             if (edge) { edge[2 * m] = e2[0]; edge[2 * m + 1] = e2[1]; }
         }
         free(row); free(rsc);
+    } else if (mode == 2) {
+        /* The listing's Refine: a proxy scan over each member's own prefix. */
+        scored_t *own = (scored_t *)malloc(sizeof(scored_t) * (size_t)(bound > 0 ? bound : 1));
+        int32_t *C = (int32_t *)malloc(sizeof(int32_t) * (size_t)(Kc > 0 ? Kc : 1));
+        for (int m = 0; m < nm; ++m) {
+            int pos = mpos[m];
+            memcpy(own, sig, sizeof(scored_t) * (size_t)pos);
+            int nC = select_top(own, pos, Kc, Kc, C, NULL, NULL);
+            for (int t = 0; t < nC; ++t) {
+                v[t].j = C[t];
+                v[t].s = dot(mq[m], kbase + (long)C[t] * kstride, d);
+            }
+            select_top(v, nC, top_k, top_k, out + (long)m * top_k,
+                       out_sc ? out_sc + (long)m * top_k : NULL, edge ? edge + 2 * m : NULL);
+        }
+        free(own); free(C);
     } else {
         /* Refine: candidate set from the one proxy scan, then per-member re-score. */
         int32_t *C = (int32_t *)malloc(sizeof(int32_t) * (size_t)(Kc > 0 ? Kc : 1));
@@ -196,7 +217,8 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
 
 /*
  * Prefill PIVOT for a list of (group, head) units.
- * q, k: bf16 bits [L, H, d].  mode 0 = Refine, 1 = Reuse.
+ * q, k: bf16 bits [L, H, d].  mode 0 = Refine, 1 = Reuse, 2 = the listing's
+ * per-member-scan Refine (cand / cand_edge are not written in mode 2).
  * Per unit u: out [g, top_k] (member m = position i*g + m), out_sc [g, top_k]
  * (nullable), edge [g, 2] (nullable), cand [Kc] (nullable), cand_edge [2]
  * (nullable), proxy [d] (nullable).  Returns 0, or -1 on bad arguments.
@@ -207,7 +229,7 @@ int oracle_prefill_units(const uint16_t *q, const uint16_t *k, int L, int H, int
                          int32_t *out, double *out_sc, double *edge,
                          int32_t *cand, double *cand_edge, uint16_t *proxy)
 {
-    if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || (mode != 0 && mode != 1))
+    if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 2)
         return -1;
     int G = (L + g - 1) / g;
     const uint16_t **mq = (const uint16_t **)malloc(sizeof(*mq) * (size_t)g);

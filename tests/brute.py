@@ -52,6 +52,12 @@ def _group_rows(q, k, members, positions, s, last, top_k, Kc, mode):
         j = np.arange(s)
         sel = top_set(k[:s] @ proxy, j, min(top_k, s))
         rows = [pad(sel, top_k) for _ in members]
+    elif mode == 2:
+        # the listing's Refine: each member scans its own prefix j < pos
+        for m, pos in zip(members, positions):
+            C = top_set(k[:pos] @ proxy, np.arange(pos), min(Kc, pos))
+            r = k[C] @ q[m]
+            rows.append(pad(top_set(r, C, min(top_k, len(C))), top_k))
     else:
         j = np.arange(last)
         C = top_set(k[:last] @ proxy, j, min(Kc, last))

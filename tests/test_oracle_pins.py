@@ -41,7 +41,7 @@ def test_prefill_matches_brute_force_exact_inputs(seed):
     top_k = int(rng.integers(1, 9))
     Kc = int(rng.integers(top_k, 3 * top_k + 1))
     q, k = int_inputs(rng, L, H, d, -2, 2)
-    for mode in (oracle.REFINE, oracle.REUSE):
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
         got = oracle.prefill(q, k, g, top_k, Kc, mode)["out"]
         want = brute.prefill(q, k, g, top_k, Kc, mode)
         np.testing.assert_array_equal(got, want, err_msg=f"mode={mode} L={L} g={g} k={top_k} Kc={Kc}")
@@ -55,7 +55,7 @@ def test_prefill_matches_brute_force_gaussian(seed):
     L = int(rng.integers(20, 120))
     g = int(rng.choice([2, 4, 8]))
     q, k = synthetic.gen_prefill(L, 2, 16, seed=seed, rho=0.9)
-    for mode in (oracle.REFINE, oracle.REUSE):
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
         got = oracle.prefill(q, k, g, 6, 12, mode)["out"]
         np.testing.assert_array_equal(got, brute.prefill(q, k, g, 6, 12, mode))
     np.testing.assert_array_equal(oracle.dense(q, k, 6)["out"], brute.dense(q, k, 6))
@@ -232,3 +232,24 @@ def test_demo_shape_c0():
     assert r["out"].shape == (1024, 8, 64)
     assert np.all(r["out"][0] == -1)
     assert np.all((r["out"] >= 0).sum(-1)[1:] == np.minimum(64, np.arange(1, 1024))[:, None])
+
+
+# ------------------------------------------------- the listing's own Refine
+@pytest.mark.parametrize("seed", range(4))
+def test_per_member_refine_reductions(seed):
+    """The listing's Refine (a proxy scan per member over its own prefix):
+    with g = 1 the proxy is the query, so it is the dense indexer; with
+    Kc >= L every prefix is whole, so again dense; and a group's last member
+    scans exactly the prefix of the single-scan reading, so its rows agree."""
+    rng = np.random.default_rng(300 + seed)
+    L, H, d, top_k = 150, 2, 16, 7
+    q, k = synthetic.gen_prefill(L, H, d, seed=seed, rho=0.9)
+    dense = oracle.dense(q, k, top_k)["out"]
+    pm = oracle.REFINE_PER_MEMBER
+    np.testing.assert_array_equal(oracle.prefill(q, k, 1, top_k, 2 * top_k, pm)["out"], dense)
+    g = int(rng.choice([3, 4, 8]))
+    np.testing.assert_array_equal(oracle.prefill(q, k, g, top_k, L, pm)["out"], dense)
+    a = oracle.prefill(q, k, g, top_k, 2 * top_k, pm)["out"]
+    b = oracle.prefill(q, k, g, top_k, 2 * top_k, oracle.REFINE)["out"]
+    last = np.minimum(np.arange(0, L, g) + g, L) - 1
+    np.testing.assert_array_equal(a[last], b[last])
