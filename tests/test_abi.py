@@ -64,3 +64,43 @@ def test_no_device_means_unsupported(lib):
     p = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16
     assert lib.pivot_index(p, p, 16, 1, 64, 4, 2, 4, 0, p, None) == 2
     assert b"sm_100" in lib.pivot_last_error() or b"device" in lib.pivot_last_error()
+
+
+def header_declarations():
+    """{name: (return kind, [parameter kinds])} from include/pivot.h, kinds
+    'p' (pointer), 'i' (int), 'z' (size_t)."""
+    text = open(os.path.join(ROOT, "include", "pivot.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    decls = {}
+    for ret, name, params in re.findall(r"\b(int|size_t|const char\s*\*)\s*([a-z_]+)\s*\(([^)]*)\)\s*;", text, re.S):
+        kinds = []
+        for prm in params.split(","):
+            prm = prm.strip()
+            if not prm or prm == "void":
+                continue
+            kinds.append("p" if "*" in prm else ("z" if "size_t" in prm else "i"))
+        decls[name] = ("p" if "*" in ret else ("z" if ret == "size_t" else "i"), kinds)
+    return decls
+
+
+def ctypes_kind(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (t is not None and hasattr(t, "_type_") and t.__name__.startswith("LP_")):
+        return "p"
+    if t is ctypes.c_size_t:
+        return "z"
+    if t is ctypes.c_int:
+        return "i"
+    return repr(t)
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every entry point is called with the argument kinds, count and return
+    type that include/pivot.h declares (a drift here would pass a size_t
+    where an int is read, or drop an argument)."""
+    decls = header_declarations()
+    assert set(decls) == set(qg.EXPORTED)
+    for name, (ret, kinds) in decls.items():
+        f = getattr(lib, name)
+        assert [ctypes_kind(t) for t in f.argtypes] == kinds, name
+        assert ctypes_kind(f.restype) == ret, name
