@@ -32,6 +32,10 @@ REFINE, REUSE = 0, 1
 # each member's own prefix.  Oracle only; it measures what the single-scan
 # reading of Refine changes.
 REFINE_PER_MEMBER = 2
+# Refine with the proxy rounded to fp32 only (not to bf16): what a hi/lo pair of
+# bf16 scan operands would give.  Oracle only; it measures what the bf16
+# proxy changes.
+REFINE_FP32_PROXY = 3
 
 
 def build(force: bool = False) -> str:
@@ -71,8 +75,8 @@ def _u16(a):
 
 
 def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False):
-    """PIVOT (Refine mode=0, Reuse mode=1, per-member-scan Refine mode=2) on the
-    listed (group, head) units.
+    """PIVOT (Refine mode=0, Reuse mode=1, per-member-scan Refine mode=2,
+    fp32-proxy Refine mode=3) on the listed (group, head) units.
 
     Returns dict: out [n,g,top_k] int32, score [n,g,top_k] f64, edge [n,g,2] f64,
     cand [n,Kc] int32 and cand_edge [n,2] (Refine), proxy [n,d] uint16.

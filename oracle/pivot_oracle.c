@@ -32,6 +32,10 @@
  *    prefix j < pos, takes C_pos = top-min(Kc, pos) of it, re-scores C_pos
  *    with its own query and keeps top-min(top_k, |C_pos|) ("Show Me The
  *    Code", pivot_refine: the scan k_h[:pos] inside the member loop).
+ *  - Refine with the fp32 proxy (mode 3, kept to measure what rounding the
+ *    proxy to bf16 changes): as mode 0, but the scan uses the proxy rounded
+ *    to fp32 only, which a hi/lo pair of bf16 operands would reproduce to
+ *    within 2^-16 relative.
  *  - Reuse: the proxy's top-min(top_k, s) over keys j < s (s = group start,
  *    strictly causal for every member; group 0 gets nothing), shared by all
  *    members.
@@ -95,14 +99,16 @@ static double dot(const uint16_t *a, const uint16_t *b, int d)
     return acc;
 }
 
-/* Proxy query: mean of the n member rows (see the reading above). */
-static void proxy_of(const uint16_t *const *rows, int n, int d, uint16_t *p)
+/* Proxy query: mean of the n member rows (see the reading above); pf, when
+ * not NULL, receives the mean rounded to fp32 only. */
+static void proxy_of(const uint16_t *const *rows, int n, int d, uint16_t *p, double *pf)
 {
     for (int c = 0; c < d; ++c) {
         double acc = 0.0;
         for (int m = 0; m < n; ++m) acc += bf16_val(rows[m][c]);
         double mean = acc / (double)n;
         p[c] = bf16_round((float)mean);
+        if (pf) pf[c] = (double)(float)mean;
     }
 }
 
@@ -147,12 +153,21 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
     scored_t *v = (scored_t *)malloc(sizeof(scored_t) * (size_t)(Kc > 0 ? Kc : 1));
     if (!p || !sig || !v) { free(p); free(sig); free(v); return -1; }
 
-    proxy_of(mq, nm, d, p);
+    double *pf = (mode == 3) ? (double *)malloc(sizeof(double) * (size_t)d) : NULL;
+    proxy_of(mq, nm, d, p, pf);
     if (proxy_out) memcpy(proxy_out, p, sizeof(uint16_t) * (size_t)d);
     for (int j = 0; j < bound; ++j) {
-        sig[j].s = dot(p, kbase + (long)j * kstride, d);
+        if (pf) {
+            const uint16_t *kr = kbase + (long)j * kstride;
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += pf[c] * bf16_val(kr[c]);
+            sig[j].s = acc;
+        } else {
+            sig[j].s = dot(p, kbase + (long)j * kstride, d);
+        }
         sig[j].j = j;
     }
+    free(pf);
 
     for (int m = 0; m < g; ++m) {
         for (int t = 0; t < top_k; ++t) {
@@ -218,7 +233,8 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
 /*
  * Prefill PIVOT for a list of (group, head) units.
  * q, k: bf16 bits [L, H, d].  mode 0 = Refine, 1 = Reuse, 2 = the listing's
- * per-member-scan Refine (cand / cand_edge are not written in mode 2).
+ * per-member-scan Refine (cand / cand_edge are not written in mode 2),
+ * 3 = Refine with the fp32 proxy.
  * Per unit u: out [g, top_k] (member m = position i*g + m), out_sc [g, top_k]
  * (nullable), edge [g, 2] (nullable), cand [Kc] (nullable), cand_edge [2]
  * (nullable), proxy [d] (nullable).  Returns 0, or -1 on bad arguments.
@@ -229,7 +245,7 @@ int oracle_prefill_units(const uint16_t *q, const uint16_t *k, int L, int H, int
                          int32_t *out, double *out_sc, double *edge,
                          int32_t *cand, double *cand_edge, uint16_t *proxy)
 {
-    if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 2)
+    if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 3)
         return -1;
     int G = (L + g - 1) / g;
     const uint16_t **mq = (const uint16_t **)malloc(sizeof(*mq) * (size_t)g);

@@ -46,7 +46,11 @@ def dense(qb, kb, top_k):
 
 
 def _group_rows(q, k, members, positions, s, last, top_k, Kc, mode):
-    proxy = round_proxy(q[members].mean(axis=0))
+    if mode == 3:   # the proxy rounded to fp32 only
+        proxy = q[members].mean(axis=0).astype(np.float32).astype(np.float64)
+        mode = 0
+    else:
+        proxy = round_proxy(q[members].mean(axis=0))
     rows = []
     if mode == 1:
         j = np.arange(s)

@@ -41,7 +41,7 @@ def test_prefill_matches_brute_force_exact_inputs(seed):
     top_k = int(rng.integers(1, 9))
     Kc = int(rng.integers(top_k, 3 * top_k + 1))
     q, k = int_inputs(rng, L, H, d, -2, 2)
-    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER, oracle.REFINE_FP32_PROXY):
         got = oracle.prefill(q, k, g, top_k, Kc, mode)["out"]
         want = brute.prefill(q, k, g, top_k, Kc, mode)
         np.testing.assert_array_equal(got, want, err_msg=f"mode={mode} L={L} g={g} k={top_k} Kc={Kc}")
@@ -55,7 +55,7 @@ def test_prefill_matches_brute_force_gaussian(seed):
     L = int(rng.integers(20, 120))
     g = int(rng.choice([2, 4, 8]))
     q, k = synthetic.gen_prefill(L, 2, 16, seed=seed, rho=0.9)
-    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER, oracle.REFINE_FP32_PROXY):
         got = oracle.prefill(q, k, g, 6, 12, mode)["out"]
         np.testing.assert_array_equal(got, brute.prefill(q, k, g, 6, 12, mode))
     np.testing.assert_array_equal(oracle.dense(q, k, 6)["out"], brute.dense(q, k, 6))
@@ -253,3 +253,12 @@ def test_per_member_refine_reductions(seed):
     b = oracle.prefill(q, k, g, top_k, 2 * top_k, oracle.REFINE)["out"]
     last = np.minimum(np.arange(0, L, g) + g, L) - 1
     np.testing.assert_array_equal(a[last], b[last])
+
+
+def test_fp32_proxy_refine_reduces_to_refine_for_single_members():
+    """With g = 1 the mean of one bf16 query is that query exactly, in fp32 as
+    in bf16, so the fp32-proxy Refine is the Refine."""
+    q, k = synthetic.gen_prefill(120, 2, 16, seed=4, rho=0.9)
+    a = oracle.prefill(q, k, 1, 5, 10, oracle.REFINE_FP32_PROXY)["out"]
+    b = oracle.prefill(q, k, 1, 5, 10, oracle.REFINE)["out"]
+    np.testing.assert_array_equal(a, b)
