@@ -455,6 +455,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     rp.out = out;
     rp.out_scores = out_scores;
     rp.cu = cu;
+    rp.max_seqlen = max_seqlen;
     rp.G = B;
     rp.L = 0;
     rp.H = H;

@@ -145,7 +145,21 @@ __global__ void __launch_bounds__(kDecSelNT) decode_select_kernel(DecodeParams p
   uint32_t* selk = reinterpret_cast<uint32_t*>(sel + p.K_sel);
   const int h = blockIdx.x / p.B, b = blockIdx.x % p.B;
   int n_b, bound;
-  if (!decode_unit(p, b, n_b, bound)) return;
+  if (!decode_unit(p, b, n_b, bound)) {
+    // skipped sequence (reported by the scan): Reuse rows are empty; the
+    // refine kernel gives Refine members empty rows without reading a
+    // candidate row
+    if (p.mode != 0) {
+      for (int m = 0; m < p.g; ++m) {
+        const long long o = ((static_cast<long long>(b) * p.g + m) * p.H + h) * p.width;
+        for (int t = threadIdx.x; t < p.width; t += kDecSelNT) {
+          p.out[o + t] = -1;
+          if (p.out_scores) p.out_scores[o + t] = __int_as_float(0x7fc00000);
+        }
+      }
+    }
+    return;
+  }
   const int K = min(p.K_sel, bound);
   const uint32_t* srow = p.scores + (static_cast<long long>(h) * p.B + b) * p.max_seqlen;
   block_select_emit<kDecSelNT>(

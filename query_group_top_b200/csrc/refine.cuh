@@ -56,6 +56,7 @@ struct RefineParams {
   float* out_scores;      // same shape as out, or null
   const int32_t* cu;      // decode: [B+1] cache row offsets; null for prefill
   int G, L, H, g, top_k, Kc, d;
+  int max_seqlen;         // decode: sequences with more cache rows (or fewer than g) are skipped
   int n_items;            // H * G units x member batches
   int nbatch;             // member batches of up to 16 per unit
   uint32_t tmem_cols;
@@ -215,6 +216,7 @@ __device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float 
 // One work item: a unit's batch of up to 16 members.
 struct RefineItem {
   int h, u, mb, nb, pos0, nc, nch;
+  int jlim;             // candidate key indices lie in [0, jlim): the scan's bound
   long long key_row0;   // cache row of key index 0
   long long qrow0;      // row (before *H) of member 0's query and output
 };
@@ -235,13 +237,25 @@ __device__ __forceinline__ RefineItem refine_item(const RefineParams& p, int ite
   } else {
     nm = p.g;
     it.key_row0 = p.cu[it.u];
-    it.pos0 = p.cu[it.u + 1] - p.cu[it.u] - p.g;
+    const int len = p.cu[it.u + 1] - p.cu[it.u];
+    it.pos0 = len - p.g;
     it.qrow0 = static_cast<long long>(it.u) * p.g;
+    if (len > p.max_seqlen || it.pos0 < 0) {
+      // A sequence the decode scan skipped (longer than max_seqlen, or
+      // shorter than one step) has no candidate row: its members get
+      // empty rows and no key is read.
+      it.nb = min(16, nm - it.mb);
+      it.nc = 0;
+      it.nch = 0;
+      it.jlim = 0;
+      return it;
+    }
   }
   it.nb = min(16, nm - it.mb);
   const int last = it.pos0 + nm - 1;
   it.nc = min(p.Kc, max(last, 0));
   it.nch = (it.nc + 127) / 128;
+  it.jlim = max(last, 0);
   return it;
 }
 
@@ -338,9 +352,12 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           const int32_t* cxc = cx + c * 128;
           for (int rr = rr0; rr < 128; rr += RSTEP) {
             const int j = cxc[(rr + c) & 127];
-            const uint16_t* src = kbase + max(j, 0) * rowstride;
+            // a missing candidate (-1 padding) reads as zeros; so would an
+            // index outside the scan's bound, which no candidate row holds
+            const bool in = j >= 0 && j < it.jlim;
+            const uint16_t* src = kbase + (in ? j : 0) * rowstride;
             const uint32_t dst = dst0 + rr * 128 + ((p8 ^ (rr & 7)) << 4);
-            const uint32_t nbytes = j >= 0 ? 16u : 0u;   // a missing candidate reads as zeros
+            const uint32_t nbytes = in ? 16u : 0u;
 #pragma unroll
             for (int a = 0; a < C::KATOMS; ++a) cp_async_16(dst + a * C::ATOM_A, src + a * 64, nbytes);
           }

@@ -252,3 +252,64 @@ def test_c4_decode_sampled():
         del out, sc
     del kc
     torch.cuda.empty_cache()
+
+
+def _bad_length_batch(g, H, d):
+    """Three sequences: 0 is valid, 1 holds fewer cache rows than one step,
+    2 is longer than the max_seqlen the call declares."""
+    dec = synthetic.gen_decode(3, H, d, g, seed=77, lo=300, hi=2000)
+    lens = np.diff(dec.cu_seqlens).astype(np.int64)
+    if lens[2] <= lens[0]:
+        lens[[0, 2]] = lens[[2, 0]]
+        rows = [dec.kcache[dec.cu_seqlens[2]:dec.cu_seqlens[3]], dec.kcache[dec.cu_seqlens[1]:dec.cu_seqlens[2]],
+                dec.kcache[dec.cu_seqlens[0]:dec.cu_seqlens[1]]]
+        q = dec.q[[2, 1, 0]]
+    else:
+        rows = [dec.kcache[dec.cu_seqlens[b]:dec.cu_seqlens[b + 1]] for b in range(3)]
+        q = dec.q
+    rows[1] = rows[1][:g - 1]
+    kc = np.ascontiguousarray(np.concatenate(rows, axis=0))
+    cu = np.zeros(4, np.int32)
+    cu[1:] = np.cumsum([r.shape[0] for r in rows])
+    max_seqlen = int(rows[0].shape[0])
+    assert rows[2].shape[0] > max_seqlen >= g > rows[1].shape[0]
+    return np.ascontiguousarray(q), kc, cu, max_seqlen
+
+
+@pytest.mark.parametrize("entry", ["ws", "noalloc"])
+@pytest.mark.parametrize("mode", ["reuse", "refine"])
+def test_decode_bad_lengths_are_skipped_and_reported(mode, entry):
+    """A sequence longer than max_seqlen, or with fewer cache rows than one
+    MTP step, is skipped on the device: its rows come back empty (-1), the
+    status reads PIVOT_ERR_INVALID_ARG, and the valid sequence is exact."""
+    import ctypes
+    g, top_k, Kc, H, d = 3, 16, 40, 2, 64
+    m = oracle.REFINE if mode == "refine" else oracle.REUSE
+    q, kc, cu, max_seqlen = _bad_length_batch(g, H, d)
+    qd, kd, cud = to_dev(q), to_dev(kc), torch.from_numpy(cu).cuda()
+    lib = qg.load_library()
+    qg.sync_status()  # start from a clear status word
+    out = torch.full((3, g, H, top_k), -7, dtype=torch.int32, device="cuda")
+    sc = torch.empty((3, g, H, top_k), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    if entry == "ws":
+        qg.pivot_decode_index(qd, kd, cud, g, top_k, Kc, m, max_seqlen=max_seqlen, out=out, out_scores=sc)
+    else:
+        rc = lib.pivot_decode_index_noalloc(qd.data_ptr(), kd.data_ptr(), cud.data_ptr(), 3, H, d, g, top_k, Kc, m,
+                                            max_seqlen, out.data_ptr(), sc.data_ptr(), stream)
+        assert rc == 0, lib.pivot_last_error()
+    flags = ctypes.c_int(0)
+    rc = lib.pivot_sync_status(stream, ctypes.byref(flags))
+    assert rc == 1 and flags.value & qg.FLAG_BADLEN, (rc, flags.value)
+    assert qg.sync_status() == 0  # the status word was cleared
+    o = out.cpu().numpy()
+    assert np.all(o[1:] == -1)
+    cub = np.array([0, cu[1]], np.int32)
+    r = oracle.decode_units(q[:1], kc[:cu[1]], cub, g, top_k, Kc, m, np.zeros(H, np.int32),
+                            np.arange(H, dtype=np.int32))
+    n0 = cu[1] - g
+    pos = np.broadcast_to((n0 + np.arange(g))[:, None], (g, H))
+    cedge = np.broadcast_to(r["cand_edge"][None], (g, H, 2)) if m == oracle.REFINE else None
+    res = compare(o[0], r["out"].transpose(1, 0, 2), r["edge"].transpose(1, 0, 2), pos, cedge,
+                  sc.cpu().numpy()[0], r["score"].transpose(1, 0, 2))
+    assert_parity(res, f"bad-length batch, valid sequence, {mode} {entry}")
