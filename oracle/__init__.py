@@ -29,13 +29,11 @@ _lib = None
 
 REFINE, REUSE = 0, 1
 # The listing's own Refine ("Show Me The Code", pivot_refine): a proxy scan over
-# each member's own prefix.  Oracle only; it measures what the single-scan
-# reading of Refine changes.
+# each member's own prefix.
 REFINE_PER_MEMBER = 2
-# Refine with the proxy rounded to fp32 only (not to bf16): what a hi/lo pair of
-# bf16 scan operands would give.  Oracle only; it measures what the bf16
-# proxy changes.
-REFINE_FP32_PROXY = 3
+# Proxy precision: the scan operand is the fp32 mean of the group ("fp32") --
+# the method -- or that mean rounded once more to bf16 ("bf16"), a variant.
+PROXY_PRECISIONS = ("fp32", "bf16")
 
 
 def build(force: bool = False) -> str:
@@ -54,9 +52,9 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         P = ctypes.c_void_p
         i = ctypes.c_int
-        lib.oracle_prefill_units.argtypes = [P, P, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P]
+        lib.oracle_prefill_units.argtypes = [P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P]
         lib.oracle_dense_units.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P]
-        lib.oracle_decode_units.argtypes = [P, P, P, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P]
+        lib.oracle_decode_units.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P]
         for f in (lib.oracle_prefill_units, lib.oracle_dense_units, lib.oracle_decode_units):
             f.restype = ctypes.c_int
         _lib = lib
@@ -74,14 +72,22 @@ def _u16(a):
     return a
 
 
-def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False):
-    """PIVOT (Refine mode=0, Reuse mode=1, per-member-scan Refine mode=2,
-    fp32-proxy Refine mode=3) on the listed (group, head) units.
+def _proxy_flag(proxy):
+    if proxy not in PROXY_PRECISIONS:
+        raise ValueError(f"proxy must be one of {PROXY_PRECISIONS}")
+    return 1 if proxy == "bf16" else 0
+
+
+def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False, proxy="fp32"):
+    """PIVOT (Refine mode=0, Reuse mode=1, per-member-scan Refine mode=2) on the
+    listed (group, head) units; `proxy` is the scan operand's precision.
 
     Returns dict: out [n,g,top_k] int32, score [n,g,top_k] f64, edge [n,g,2] f64,
-    cand [n,Kc] int32 and cand_edge [n,2] (Refine), proxy [n,d] uint16.
+    cand [n,Kc] int32 and cand_edge [n,2] (Refine), proxy [n,d] float32 (the
+    fp32 mean) and proxy_bf16 [n,d] uint16 (its bf16 rounding).
     """
     lib = _load()
+    pb = _proxy_flag(proxy)
     q = _u16(q)
     k = _u16(k)
     L, H, d = q.shape
@@ -93,27 +99,29 @@ def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False):
     edge = np.empty((n, g, 2), np.float64)
     cand = np.empty((n, Kc), np.int32) if want_cand else None
     cedge = np.empty((n, 2), np.float64)
-    proxy = np.empty((n, d), np.uint16)
-    rc = lib.oracle_prefill_units(_p(q), _p(k), L, H, d, g, top_k, Kc, mode, n, _p(groups), _p(heads),
-                                  _p(out), _p(sc), _p(edge), _p(cand), _p(cedge), _p(proxy))
+    p32 = np.empty((n, d), np.float32)
+    p16 = np.empty((n, d), np.uint16)
+    rc = lib.oracle_prefill_units(_p(q), _p(k), L, H, d, g, top_k, Kc, mode, pb, n, _p(groups), _p(heads),
+                                  _p(out), _p(sc), _p(edge), _p(cand), _p(cedge), _p(p32), _p(p16))
     if rc != 0:
         raise ValueError("oracle_prefill_units rejected its arguments")
-    return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, proxy=proxy)
+    return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, proxy=p32, proxy_bf16=p16)
 
 
-def prefill(q, k, g, top_k, Kc, mode, want_cand=False):
+def prefill(q, k, g, top_k, Kc, mode, want_cand=False, proxy="fp32"):
     """Full prefill PIVOT: out [L,H,top_k] int32 plus per-row scores/edges."""
     L, H, _ = q.shape
     G = (L + g - 1) // g
     gi, hi = np.meshgrid(np.arange(G, dtype=np.int32), np.arange(H, dtype=np.int32), indexing="ij")
-    r = prefill_units(q, k, g, top_k, Kc, mode, gi.ravel(), hi.ravel(), want_cand)
+    r = prefill_units(q, k, g, top_k, Kc, mode, gi.ravel(), hi.ravel(), want_cand, proxy)
     # [G*H, g, k] -> [G, H, g, k] -> [G, g, H, k] -> [G*g, H, k] -> [:L]
     def fold(a):
         a = a.reshape(G, H, g, *a.shape[2:])
         a = np.swapaxes(a, 1, 2).reshape(G * g, H, *a.shape[3:])
         return np.ascontiguousarray(a[:L])
     res = dict(out=fold(r["out"]), score=fold(r["score"]), edge=fold(r["edge"]),
-               cand_edge=r["cand_edge"].reshape(G, H, 2), proxy=r["proxy"].reshape(G, H, -1))
+               cand_edge=r["cand_edge"].reshape(G, H, 2), proxy=r["proxy"].reshape(G, H, -1),
+               proxy_bf16=r["proxy_bf16"].reshape(G, H, -1))
     if want_cand:
         res["cand"] = r["cand"].reshape(G, H, Kc)
     return res
@@ -147,9 +155,10 @@ def dense(q, k, top_k):
                 edge=r["edge"].reshape(L, H, 2))
 
 
-def decode_units(q, kcache, cu_seqlens, g, top_k, Kc, mode, seqs, heads, want_cand=False):
+def decode_units(q, kcache, cu_seqlens, g, top_k, Kc, mode, seqs, heads, want_cand=False, proxy="fp32"):
     """Decode PIVOT on (sequence, head) units; q [B,g,H,d], kcache [rows,H,d]."""
     lib = _load()
+    pb = _proxy_flag(proxy)
     q = _u16(q)
     kcache = _u16(kcache)
     B, gq, H, d = q.shape
@@ -164,10 +173,11 @@ def decode_units(q, kcache, cu_seqlens, g, top_k, Kc, mode, seqs, heads, want_ca
     edge = np.empty((n, g, 2), np.float64)
     cand = np.empty((n, Kc), np.int32) if want_cand else None
     cedge = np.empty((n, 2), np.float64)
-    proxy = np.empty((n, d), np.uint16)
-    rc = lib.oracle_decode_units(_p(q), _p(kcache), _p(cu), B, H, d, g, top_k, Kc, mode, n,
+    p32 = np.empty((n, d), np.float32)
+    p16 = np.empty((n, d), np.uint16)
+    rc = lib.oracle_decode_units(_p(q), _p(kcache), _p(cu), B, H, d, g, top_k, Kc, mode, pb, n,
                                  _p(seqs), _p(heads), _p(out), _p(sc), _p(edge), _p(cand),
-                                 _p(cedge), _p(proxy))
+                                 _p(cedge), _p(p32), _p(p16))
     if rc != 0:
         raise ValueError("oracle_decode_units rejected its arguments")
-    return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, proxy=proxy)
+    return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, proxy=p32, proxy_bf16=p16)

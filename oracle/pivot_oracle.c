@@ -18,8 +18,11 @@
  *    may be partial and its proxy is the mean over its actual members
  *    ("Show Me The Code", the g_start/g_end loop).
  *  - Proxy: the mean of the members' queries, accumulated in fp64 in member
- *    order, divided by the member count in fp64, rounded to fp32 and then to
- *    bf16 (round to nearest even); the bf16 proxy is the scan operand.
+ *    order (exact for bf16 inputs of ordinary range), divided by the member
+ *    count in fp64 and rounded to fp32 (round to nearest even): the fp32 mean
+ *    is the scan operand.  Option proxy_bf16 rounds that mean once more, to
+ *    bf16, and scans with the bf16 value instead (what a scan that feeds the
+ *    mean to the tensor cores as a single bf16 operand computes).
  *  - Causality: a query at position pos sees keys j < pos (the listing scans
  *    k_h[:pos]).
  *  - Refine: ONE proxy scan per group over j < last, last = the largest
@@ -32,10 +35,6 @@
  *    prefix j < pos, takes C_pos = top-min(Kc, pos) of it, re-scores C_pos
  *    with its own query and keeps top-min(top_k, |C_pos|) ("Show Me The
  *    Code", pivot_refine: the scan k_h[:pos] inside the member loop).
- *  - Refine with the fp32 proxy (mode 3, kept to measure what rounding the
- *    proxy to bf16 changes): as mode 0, but the scan uses the proxy rounded
- *    to fp32 only, which a hi/lo pair of bf16 operands would reproduce to
- *    within 2^-16 relative.
  *  - Reuse: the proxy's top-min(top_k, s) over keys j < s (s = group start,
  *    strictly causal for every member; group 0 gets nothing), shared by all
  *    members.
@@ -99,17 +98,29 @@ static double dot(const uint16_t *a, const uint16_t *b, int d)
     return acc;
 }
 
-/* Proxy query: mean of the n member rows (see the reading above); pf, when
- * not NULL, receives the mean rounded to fp32 only. */
-static void proxy_of(const uint16_t *const *rows, int n, int d, uint16_t *p, double *pf)
+/* Proxy query: mean of the n member rows (see the reading above).  p
+ * receives the scan operand (the fp32 mean, or its bf16 rounding when
+ * proxy_bf16), p32 / pb (nullable) the fp32 mean and its bf16 rounding. */
+static void proxy_of(const uint16_t *const *rows, int n, int d, int proxy_bf16,
+                     double *p, float *p32, uint16_t *pb)
 {
     for (int c = 0; c < d; ++c) {
         double acc = 0.0;
         for (int m = 0; m < n; ++m) acc += bf16_val(rows[m][c]);
-        double mean = acc / (double)n;
-        p[c] = bf16_round((float)mean);
-        if (pf) pf[c] = (double)(float)mean;
+        float mean = (float)(acc / (double)n);
+        uint16_t b = bf16_round(mean);
+        p[c] = proxy_bf16 ? bf16_val(b) : (double)mean;
+        if (p32) p32[c] = mean;
+        if (pb) pb[c] = b;
     }
+}
+
+/* Scan score of the proxy against one key row. */
+static double proxy_dot(const double *p, const uint16_t *k, int d)
+{
+    double acc = 0.0;
+    for (int c = 0; c < d; ++c) acc += p[c] * bf16_val(k[c]);
+    return acc;
 }
 
 /*
@@ -143,31 +154,21 @@ static int select_top(scored_t *v, int n, int K, int width, int32_t *idx, double
  */
 static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int g,
                      const uint16_t *kbase, long kstride, int d, int s, int last,
-                     int top_k, int Kc, int mode,
+                     int top_k, int Kc, int mode, int proxy_bf16,
                      int32_t *out, double *out_sc, double *edge,
-                     int32_t *cand, double *cand_edge, uint16_t *proxy_out)
+                     int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb)
 {
-    uint16_t *p = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)d);
+    double *p = (double *)malloc(sizeof(double) * (size_t)d);
     int bound = (mode == 1) ? s : last;
     scored_t *sig = (scored_t *)malloc(sizeof(scored_t) * (size_t)(bound > 0 ? bound : 1));
     scored_t *v = (scored_t *)malloc(sizeof(scored_t) * (size_t)(Kc > 0 ? Kc : 1));
     if (!p || !sig || !v) { free(p); free(sig); free(v); return -1; }
 
-    double *pf = (mode == 3) ? (double *)malloc(sizeof(double) * (size_t)d) : NULL;
-    proxy_of(mq, nm, d, p, pf);
-    if (proxy_out) memcpy(proxy_out, p, sizeof(uint16_t) * (size_t)d);
+    proxy_of(mq, nm, d, proxy_bf16, p, proxy32, proxyb);
     for (int j = 0; j < bound; ++j) {
-        if (pf) {
-            const uint16_t *kr = kbase + (long)j * kstride;
-            double acc = 0.0;
-            for (int c = 0; c < d; ++c) acc += pf[c] * bf16_val(kr[c]);
-            sig[j].s = acc;
-        } else {
-            sig[j].s = dot(p, kbase + (long)j * kstride, d);
-        }
+        sig[j].s = proxy_dot(p, kbase + (long)j * kstride, d);
         sig[j].j = j;
     }
-    free(pf);
 
     for (int m = 0; m < g; ++m) {
         for (int t = 0; t < top_k; ++t) {
@@ -233,19 +234,22 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
 /*
  * Prefill PIVOT for a list of (group, head) units.
  * q, k: bf16 bits [L, H, d].  mode 0 = Refine, 1 = Reuse, 2 = the listing's
- * per-member-scan Refine (cand / cand_edge are not written in mode 2),
- * 3 = Refine with the fp32 proxy.
+ * per-member-scan Refine (cand / cand_edge are not written in mode 2).
+ * proxy_bf16 = 0: scan with the fp32 mean (the method); 1: with its bf16
+ * rounding (the variant).
  * Per unit u: out [g, top_k] (member m = position i*g + m), out_sc [g, top_k]
  * (nullable), edge [g, 2] (nullable), cand [Kc] (nullable), cand_edge [2]
- * (nullable), proxy [d] (nullable).  Returns 0, or -1 on bad arguments.
+ * (nullable), proxy32 [d] fp32 mean (nullable), proxyb [d] its bf16 rounding
+ * (nullable).  Returns 0, or -1 on bad arguments.
  */
 int oracle_prefill_units(const uint16_t *q, const uint16_t *k, int L, int H, int d,
-                         int g, int top_k, int Kc, int mode,
+                         int g, int top_k, int Kc, int mode, int proxy_bf16,
                          int n_units, const int32_t *unit_group, const int32_t *unit_head,
                          int32_t *out, double *out_sc, double *edge,
-                         int32_t *cand, double *cand_edge, uint16_t *proxy)
+                         int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb)
 {
-    if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 3)
+    if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 2 ||
+        proxy_bf16 < 0 || proxy_bf16 > 1)
         return -1;
     int G = (L + g - 1) / g;
     const uint16_t **mq = (const uint16_t **)malloc(sizeof(*mq) * (size_t)g);
@@ -260,13 +264,14 @@ int oracle_prefill_units(const uint16_t *q, const uint16_t *k, int L, int H, int
             mpos[m] = s + m;
         }
         rc = one_group(mq, mpos, nm, g, k + (long)h * d, (long)H * d, d, s, e - 1,
-                       top_k, Kc, mode,
+                       top_k, Kc, mode, proxy_bf16,
                        out + (long)u * g * top_k,
                        out_sc ? out_sc + (long)u * g * top_k : NULL,
                        edge ? edge + (long)u * g * 2 : NULL,
                        cand ? cand + (long)u * Kc : NULL,
                        cand_edge ? cand_edge + (long)u * 2 : NULL,
-                       proxy ? proxy + (long)u * d : NULL);
+                       proxy32 ? proxy32 + (long)u * d : NULL,
+                       proxyb ? proxyb + (long)u * d : NULL);
     }
     free(mq); free(mpos);
     return rc;
@@ -299,19 +304,21 @@ int oracle_dense_units(const uint16_t *q, const uint16_t *k, int L, int H, int d
 }
 
 /*
- * Decode PIVOT for a list of (sequence, head) units.
+ * Decode PIVOT for a list of (sequence, head) units (modes and proxy_bf16 as
+ * in oracle_prefill_units).
  * q: bf16 bits [B, g, H, d]; kcache: bf16 bits [cu[B], H, d]; sequence b's
  * keys are cache rows cu[b] .. cu[b+1]-1 and it holds n_b + g of them, so
  * n_b = cu[b+1] - cu[b] - g.  Member i sits at position n_b + i.
  * Outputs per unit as in oracle_prefill_units.
  */
 int oracle_decode_units(const uint16_t *q, const uint16_t *kcache, const int32_t *cu,
-                        int B, int H, int d, int g, int top_k, int Kc, int mode,
+                        int B, int H, int d, int g, int top_k, int Kc, int mode, int proxy_bf16,
                         int n_units, const int32_t *unit_seq, const int32_t *unit_head,
                         int32_t *out, double *out_sc, double *edge,
-                        int32_t *cand, double *cand_edge, uint16_t *proxy)
+                        int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb)
 {
-    if (B < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || (mode != 0 && mode != 1))
+    if (B < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 2 ||
+        proxy_bf16 < 0 || proxy_bf16 > 1)
         return -1;
     const uint16_t **mq = (const uint16_t **)malloc(sizeof(*mq) * (size_t)g);
     int32_t *mpos = (int32_t *)malloc(sizeof(int32_t) * (size_t)g);
@@ -326,13 +333,14 @@ int oracle_decode_units(const uint16_t *q, const uint16_t *kcache, const int32_t
             mpos[m] = n_b + m;
         }
         rc = one_group(mq, mpos, g, g, kcache + ((long)cu[b] * H + h) * d, (long)H * d, d,
-                       n_b, n_b + g - 1, top_k, Kc, mode,
+                       n_b, n_b + g - 1, top_k, Kc, mode, proxy_bf16,
                        out + (long)u * g * top_k,
                        out_sc ? out_sc + (long)u * g * top_k : NULL,
                        edge ? edge + (long)u * g * 2 : NULL,
                        cand ? cand + (long)u * Kc : NULL,
                        cand_edge ? cand_edge + (long)u * 2 : NULL,
-                       proxy ? proxy + (long)u * d : NULL);
+                       proxy32 ? proxy32 + (long)u * d : NULL,
+                       proxyb ? proxyb + (long)u * d : NULL);
     }
     free(mq); free(mpos);
     return rc;

@@ -13,7 +13,7 @@ def decode_bf16(bits):
 
 
 def round_proxy(mean64):
-    """fp64 -> fp32 -> bf16 (torch's round-to-nearest-even) -> float64."""
+    """fp64 -> fp32 -> bf16 (torch's round-to-nearest-even) -> float64 (the bf16 proxy variant)."""
     t = torch.from_numpy(np.asarray(mean64, dtype=np.float64).astype(np.float32))
     return t.to(torch.bfloat16).to(torch.float64).numpy()
 
@@ -45,12 +45,12 @@ def dense(qb, kb, top_k):
     return out
 
 
-def _group_rows(q, k, members, positions, s, last, top_k, Kc, mode):
-    if mode == 3:   # the proxy rounded to fp32 only
-        proxy = q[members].mean(axis=0).astype(np.float32).astype(np.float64)
-        mode = 0
-    else:
-        proxy = round_proxy(q[members].mean(axis=0))
+def _group_rows(q, k, members, positions, s, last, top_k, Kc, mode, proxy_prec="fp32"):
+    mean = q[members].mean(axis=0)
+    if proxy_prec == "fp32":
+        proxy = mean.astype(np.float32).astype(np.float64)
+    else:   # the bf16 variant: the fp32 mean rounded once more, to bf16
+        proxy = round_proxy(mean)
     rows = []
     if mode == 1:
         j = np.arange(s)
@@ -72,7 +72,7 @@ def _group_rows(q, k, members, positions, s, last, top_k, Kc, mode):
     return proxy, rows
 
 
-def prefill(qb, kb, g, top_k, Kc, mode):
+def prefill(qb, kb, g, top_k, Kc, mode, proxy_prec="fp32"):
     q = decode_bf16(qb)
     k = decode_bf16(kb)
     L, H, _ = q.shape
@@ -81,13 +81,13 @@ def prefill(qb, kb, g, top_k, Kc, mode):
         for s in range(0, L, g):
             e = min(s + g, L)
             mem = list(range(s, e))
-            _, rows = _group_rows(q[:, h], k[:, h], mem, mem, s, e - 1, top_k, Kc, mode)
+            _, rows = _group_rows(q[:, h], k[:, h], mem, mem, s, e - 1, top_k, Kc, mode, proxy_prec)
             for pos, r in zip(mem, rows):
                 out[pos, h] = r
     return out
 
 
-def decode(qb, kcb, cu, g, top_k, Kc, mode):
+def decode(qb, kcb, cu, g, top_k, Kc, mode, proxy_prec="fp32"):
     q = decode_bf16(qb)          # [B, g, H, d]
     kc = decode_bf16(kcb)        # [rows, H, d]
     B, _, H, _ = q.shape
@@ -98,7 +98,7 @@ def decode(qb, kcb, cu, g, top_k, Kc, mode):
         for h in range(H):
             pos = [n_b + i for i in range(g)]
             _, rows = _group_rows(q[b, :, h], keys[:, h], list(range(g)), pos, n_b, n_b + g - 1,
-                                  top_k, Kc, mode)
+                                  top_k, Kc, mode, proxy_prec)
             for i, r in enumerate(rows):
                 out[b, i, h] = r
     return out

@@ -41,10 +41,11 @@ def test_prefill_matches_brute_force_exact_inputs(seed):
     top_k = int(rng.integers(1, 9))
     Kc = int(rng.integers(top_k, 3 * top_k + 1))
     q, k = int_inputs(rng, L, H, d, -2, 2)
-    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER, oracle.REFINE_FP32_PROXY):
-        got = oracle.prefill(q, k, g, top_k, Kc, mode)["out"]
-        want = brute.prefill(q, k, g, top_k, Kc, mode)
-        np.testing.assert_array_equal(got, want, err_msg=f"mode={mode} L={L} g={g} k={top_k} Kc={Kc}")
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
+        for prec in oracle.PROXY_PRECISIONS:
+            got = oracle.prefill(q, k, g, top_k, Kc, mode, proxy=prec)["out"]
+            want = brute.prefill(q, k, g, top_k, Kc, mode, prec)
+            np.testing.assert_array_equal(got, want, err_msg=f"mode={mode} {prec} L={L} g={g} k={top_k} Kc={Kc}")
     got = oracle.dense(q, k, top_k)["out"]
     np.testing.assert_array_equal(got, brute.dense(q, k, top_k))
 
@@ -55,9 +56,10 @@ def test_prefill_matches_brute_force_gaussian(seed):
     L = int(rng.integers(20, 120))
     g = int(rng.choice([2, 4, 8]))
     q, k = synthetic.gen_prefill(L, 2, 16, seed=seed, rho=0.9)
-    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER, oracle.REFINE_FP32_PROXY):
-        got = oracle.prefill(q, k, g, 6, 12, mode)["out"]
-        np.testing.assert_array_equal(got, brute.prefill(q, k, g, 6, 12, mode))
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
+        for prec in oracle.PROXY_PRECISIONS:
+            got = oracle.prefill(q, k, g, 6, 12, mode, proxy=prec)["out"]
+            np.testing.assert_array_equal(got, brute.prefill(q, k, g, 6, 12, mode, prec), err_msg=f"{mode} {prec}")
     np.testing.assert_array_equal(oracle.dense(q, k, 6)["out"], brute.dense(q, k, 6))
 
 
@@ -73,10 +75,26 @@ def test_decode_matches_brute_force(seed):
     q = synthetic.bf16_from_f32(rng.integers(-2, 3, size=(B, g, H, d)).astype(np.float32))
     kc = synthetic.bf16_from_f32(rng.integers(-2, 3, size=(int(cu[-1]), H, d)).astype(np.float32))
     bi, hi = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
+        for prec in oracle.PROXY_PRECISIONS:
+            r = oracle.decode_units(q, kc, cu, g, 4, 9, mode, bi.ravel(), hi.ravel(), proxy=prec)
+            got = r["out"].reshape(B, H, g, 4).transpose(0, 2, 1, 3)
+            np.testing.assert_array_equal(got, brute.decode(q, kc, cu, g, 4, 9, mode, prec), err_msg=f"{mode} {prec}")
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_decode_gaussian_matches_brute_force(seed):
+    """Gaussian decode inputs (fp32 means that are not bf16 values) for both
+    proxy precisions."""
+    g = 2 + seed % 2
+    dec = synthetic.gen_decode(3, 2, 16, g, seed=50 + seed, lo=5, hi=60)
+    bi, hi = np.meshgrid(np.arange(3), np.arange(2), indexing="ij")
     for mode in (oracle.REFINE, oracle.REUSE):
-        r = oracle.decode_units(q, kc, cu, g, 4, 9, mode, bi.ravel(), hi.ravel())
-        got = r["out"].reshape(B, H, g, 4).transpose(0, 2, 1, 3)
-        np.testing.assert_array_equal(got, brute.decode(q, kc, cu, g, 4, 9, mode))
+        for prec in oracle.PROXY_PRECISIONS:
+            r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, g, 5, 11, mode, bi.ravel(), hi.ravel(),
+                                    proxy=prec)
+            got = r["out"].reshape(3, 2, g, 5).transpose(0, 2, 1, 3)
+            np.testing.assert_array_equal(got, brute.decode(dec.q, dec.kcache, dec.cu_seqlens, g, 5, 11, mode, prec))
 
 
 # ------------------------------------------------------------ golden fixtures
@@ -109,21 +127,58 @@ def test_worked_example():
             m = oracle.REFINE if mode == "refine" else oracle.REUSE
             r = oracle.prefill(q, k, 2, top_k, Kc, m)
             got = r["out"][:, 0]
-            proxies = synthetic.bf16_to_f32(r["proxy"][:, 0])
-            np.testing.assert_array_equal(proxies, np.asarray(vals["proxies"], np.float32))
+            np.testing.assert_array_equal(r["proxy"][:, 0], np.asarray(vals["proxies"], np.float32))
         np.testing.assert_array_equal(got, np.asarray(want), err_msg=f"{mode} k={top_k} Kc={Kc}")
 
 
-def test_proxy_rounding_fixture():
-    with open(os.path.join(GOLD, "proxy_rounding.txt")) as f:
-        cases = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
-    for members, want in cases:
-        m = [float(x) for x in members.split(",")]
-        n = len(m)
-        q = bits(m)[:, None, None]                       # [n, 1, 1]: one group of n members
-        k = bits([1.0] * n)[:, None, None]
-        r = oracle.prefill_units(q, k, n, 1, 1, oracle.REFINE, [0], [0])
-        assert synthetic.bf16_to_f32(r["proxy"][0])[0] == np.float32(float(want)), members
+def _proxy_cases(name):
+    with open(os.path.join(GOLD, name)) as f:
+        for ln in f:
+            if ln.strip() and not ln.startswith("#"):
+                members, want = ln.split()
+                m = [float(x) for x in members.split(",")]
+                n = len(m)
+                q = bits(m)[:, None, None]                       # [n, 1, 1]: one group of n members
+                k = bits([1.0] * n)[:, None, None]
+                yield members, want, oracle.prefill_units(q, k, n, 1, 1, oracle.REFINE, [0], [0])
+
+
+def test_proxy_rounding_fixture_fp32():
+    """The proxy is the fp32 mean: hand-rounded cases, ties to even included."""
+    from fractions import Fraction
+    for members, want, r in _proxy_cases("proxy_rounding_fp32.txt"):
+        got = r["proxy"][0][0]
+        assert Fraction(float(got)) == Fraction(want), (members, float(got))
+
+
+def test_proxy_rounding_fixture_bf16_variant():
+    """The bf16 variant rounds the fp32 mean once more, to bf16."""
+    for members, want, r in _proxy_cases("proxy_rounding.txt"):
+        assert synthetic.bf16_to_f32(r["proxy_bf16"][0])[0] == np.float32(float(want)), members
+
+
+def test_fp32_proxy_changes_the_candidate_set_where_bf16_rounding_would():
+    """Closed form: two keys e_1 (index 0) and e_0 (index 1); a group of four
+    members whose mean is (1 + 1/256, 1 + 1/512).  Both coordinates are exact
+    in fp32, so key 1 (score 1 + 1/256) beats key 0 (score 1 + 1/512).  Rounded
+    to bf16 both coordinates become 1, the scores tie and the tie goes to key 0.
+    Keys 2..7 score -2.  With Kc = top_k = 1 every member of the group keeps
+    the single candidate, and Reuse shares it."""
+    L, d, g = 8, 2, 4
+    k = np.full((L, 1, d), -1.0, np.float32)
+    k[0, 0] = (0.0, 1.0)
+    k[1, 0] = (1.0, 0.0)
+    q = np.zeros((L, 1, d), np.float32)
+    q[4:, 0, 0] = (1.0, 1.0, 1.0078125, 1.0078125)
+    q[4:, 0, 1] = (1.0, 1.0, 1.0, 1.0078125)
+    qb, kb = synthetic.bf16_from_f32(q), synthetic.bf16_from_f32(k)
+    for mode in (oracle.REFINE, oracle.REUSE):
+        f32 = oracle.prefill(qb, kb, g, 1, 1, mode)
+        b16 = oracle.prefill(qb, kb, g, 1, 1, mode, proxy="bf16")
+        assert f32["proxy"][1, 0].tolist() == [1.00390625, 1.001953125]
+        assert synthetic.bf16_to_f32(b16["proxy_bf16"][1, 0]).tolist() == [1.0, 1.0]
+        assert np.all(f32["out"][4:, 0, 0] == 1), f32["out"][4:, 0]
+        assert np.all(b16["out"][4:, 0, 0] == 0), b16["out"][4:, 0]
 
 
 # --------------------------------------------------------------- closed forms
@@ -255,10 +310,11 @@ def test_per_member_refine_reductions(seed):
     np.testing.assert_array_equal(a[last], b[last])
 
 
-def test_fp32_proxy_refine_reduces_to_refine_for_single_members():
+def test_proxy_precisions_agree_for_single_members():
     """With g = 1 the mean of one bf16 query is that query exactly, in fp32 as
-    in bf16, so the fp32-proxy Refine is the Refine."""
+    in bf16, so both proxy precisions give the same rows (all three modes)."""
     q, k = synthetic.gen_prefill(120, 2, 16, seed=4, rho=0.9)
-    a = oracle.prefill(q, k, 1, 5, 10, oracle.REFINE_FP32_PROXY)["out"]
-    b = oracle.prefill(q, k, 1, 5, 10, oracle.REFINE)["out"]
-    np.testing.assert_array_equal(a, b)
+    for mode in (oracle.REFINE, oracle.REUSE, oracle.REFINE_PER_MEMBER):
+        a = oracle.prefill(q, k, 1, 5, 10, mode)["out"]
+        b = oracle.prefill(q, k, 1, 5, 10, mode, proxy="bf16")["out"]
+        np.testing.assert_array_equal(a, b)
