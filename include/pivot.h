@@ -40,6 +40,18 @@ extern "C" {
 
 typedef enum { PIVOT_REFINE = 0, PIVOT_REUSE = 1 } pivot_mode_t;
 
+/*
+ * Option bit OR-ed into `mode`: scan with the group mean rounded to bf16
+ * instead of the fp32 mean.  This is a variant of the method, not the method:
+ * the pages define the proxy as the group mean ("How It Works": proxy_q =
+ * mean(group)) and this library takes it in fp32 by default, which the
+ * tensor-core scan carries as three bf16 terms (three MMA passes per key
+ * tile).  With the flag the scan makes one pass; candidate sets then differ
+ * from the fp32-mean ones wherever the bf16 rounding reorders near-boundary
+ * keys.
+ */
+enum { PIVOT_PROXY_BF16 = 0x100 };
+
 typedef enum {
   PIVOT_OK = 0,
   PIVOT_ERR_INVALID_ARG = 1,
@@ -53,14 +65,16 @@ typedef enum {
  * PIVOT prefill indexer for one layer, all heads.
  * Paper abstract and "How It Works": consecutive queries form groups of g
  * (starting at 0, g, 2g, ...; the last may be partial); each group's proxy is
- * the mean of its queries (fp64 sum, rounded to fp32 then bf16); one scan of
- * the proxy over the group's causal prefix gives a candidate set.
+ * the mean of its queries (fp64 sum divided by the member count, rounded to
+ * fp32); one scan of the proxy over the group's causal prefix gives a
+ * candidate set.
  *   mode = PIVOT_REFINE ("How It Works" per-query refine; listing pivot_refine):
  *     scan keys j < last (the group's largest position), C = top-min(Kc,last);
  *     member pos re-scores {j in C : j < pos} with its own query and keeps
  *     top-min(top_k, that count).
  *   mode = PIVOT_REUSE (listing pivot_reuse): scan keys j < s (group start);
  *     every member gets the proxy's top-min(top_k, s).  Kc is not used.
+ *   Either may be OR-ed with PIVOT_PROXY_BF16 (the bf16-proxy variant).
  * q, k:     bf16 [L][H][d].
  * out_idx:  int32 [L][H][top_k].
  * Temporary device memory is taken with cudaMallocAsync on `stream` and freed
@@ -120,6 +134,27 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * As the _ws variants, with two more nullable outputs that expose the
+ * method's intermediate results ("How It Works": the proxy of each group and
+ * its candidate set C = top-Kc of the proxy scores):
+ *   out_proxy: float32 [G][H][d] (decode: [B][H][d]), each group's proxy --
+ *              the fp32 mean of its queries (or its bf16 rounding under
+ *              PIVOT_PROXY_BF16), 16-byte aligned;
+ *   out_cand:  int32 [G][H][Kc] (decode: [B][H][Kc]), PIVOT_REFINE only (else
+ *              PIVOT_ERR_INVALID_ARG): each group's candidate key indices in
+ *              ascending order, -1 padded; a decode sequence skipped for its
+ *              length gets an all -1 row.
+ * G = ceil(L / g).
+ */
+int pivot_index_ex(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
+                   int32_t* out_idx, float* out_scores, float* out_proxy, int32_t* out_cand, void* workspace,
+                   size_t workspace_bytes, void* stream);
+int pivot_decode_index_ex(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d, int g,
+                          int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx, float* out_scores,
+                          float* out_proxy, int32_t* out_cand, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
  * Decode without any device allocation (the paper has no counterpart; this is
  * a deployment variant of pivot_decode_index, same arguments and results).
  * For callers that cannot allocate device memory during a decode step: an
@@ -127,7 +162,7 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
  * so a cudaMalloc there would fail or fragment it, or host code that has no
  * allocator of its own and must not own device buffers.  Its scratch is a
  * 32 MiB array built into the library (held by every GPU that loads it until
- * the process exits); a call whose scratch need -- proxies B*H*d*2 + order keys
+ * the process exits); a call whose scratch need -- proxies B*H*d*4 + order keys
  * H*B*max_seqlen*4 + (Refine) candidates H*B*CW*4 bytes, CW = Kc rounded up to
  * a multiple of 128, each rounded up to 256 -- exceeds 32 MiB is rejected with
  * PIVOT_ERR_WORKSPACE and a message.

@@ -6,6 +6,7 @@ device memory and streams.  There is no CPU fallback: without the built
 library or an sm_100 device every call raises.
 
     idx = pivot_index(q, k, g=16, top_k=2048, Kc=4096, mode=REFINE)   # [L, H, top_k] int32
+    idx = pivot_index(q, k, 16, 2048, 4096, REFINE, proxy="bf16")      # the bf16-proxy variant
     idx = dense_index(q, k, top_k=2048)
     idx = pivot_decode_index(q, kcache, cu_seqlens, g=2, top_k=2048, Kc=4096, max_seqlen=...)
 """
@@ -20,6 +21,7 @@ __all__ = ["REFINE", "REUSE", "PivotError", "pivot_index", "dense_index", "pivot
            "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED"]
 
 REFINE, REUSE = 0, 1
+PROXY_BF16 = 0x100          # option bit of `mode`: scan with the bf16-rounded mean
 FLAG_TIMEOUT, FLAG_BADLEN, FLAG_FALLBACK, FLAG_NOCONVERGE = 1, 2, 4, 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,6 +34,7 @@ EXPORTED = (
     "pivot_workspace_size", "pivot_index_ws", "dense_workspace_size", "dense_index_ws",
     "pivot_decode_workspace_size", "pivot_decode_index_ws", "pivot_sync_status", "pivot_last_error",
     "pivot_trace_enable", "pivot_trace_collect", "pivot_decode_index_noalloc",
+    "pivot_index_ex", "pivot_decode_index_ex",
 )
 
 
@@ -67,6 +70,8 @@ def load_library():
         "pivot_trace_enable": ([I], I),
         "pivot_trace_collect": ([ctypes.c_char_p, Z, P, P, I], I),
         "pivot_decode_index_noalloc": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P], I),
+        "pivot_index_ex": ([P, P, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
+        "pivot_decode_index_ex": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -117,9 +122,29 @@ def _out(out, shape, dtype, device, name):
     return out
 
 
-def pivot_index(q, k, g, top_k, Kc, mode=REFINE, out=None, out_scores=None, stream=None):
-    """PIVOT prefill indexer: q, k bf16 [L, H, d] -> int32 [L, H, top_k] (ascending, -1 padded)."""
+def _mode_bits(mode, proxy):
+    if mode not in (REFINE, REUSE):
+        raise PivotError("mode must be REFINE or REUSE")
+    if proxy not in ("fp32", "bf16"):
+        raise PivotError('proxy must be "fp32" (the method) or "bf16" (the variant)')
+    return mode | (PROXY_BF16 if proxy == "bf16" else 0)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def pivot_index(q, k, g, top_k, Kc, mode=REFINE, out=None, out_scores=None, stream=None, proxy="fp32",
+                out_proxy=None, out_cand=None):
+    """PIVOT prefill indexer: q, k bf16 [L, H, d] -> int32 [L, H, top_k] (ascending, -1 padded).
+
+    proxy: "fp32" scans with the fp32 group mean (the method), "bf16" with its
+    bf16 rounding (a variant).  out_proxy (float32 [G, H, d]) and out_cand
+    (int32 [G, H, Kc], Refine only) receive the groups' proxies and candidate
+    sets when given (G = ceil(L / g)).
+    """
     lib = load_library()
+    bits = _mode_bits(mode, proxy)
     _check_bf16("q", q, 3)
     _check_bf16("k", k, 3)
     if q.shape != k.shape:
@@ -128,11 +153,20 @@ def pivot_index(q, k, g, top_k, Kc, mode=REFINE, out=None, out_scores=None, stre
     out = _out(out, (L, H, top_k), torch.int32, q.device, "out")
     if out_scores is not None:
         out_scores = _out(out_scores, (L, H, top_k), torch.float32, q.device, "out_scores")
+    G = (L + g - 1) // g if g >= 1 else 0
+    if out_proxy is not None:
+        out_proxy = _out(out_proxy, (G, H, d), torch.float32, q.device, "out_proxy")
+    if out_cand is not None:
+        out_cand = _out(out_cand, (G, H, Kc), torch.int32, q.device, "out_cand")
     sp = _stream_ptr(stream)
-    n = lib.pivot_workspace_size(L, H, d, g, top_k, Kc, mode)
+    n = lib.pivot_workspace_size(L, H, d, g, top_k, Kc, bits)
     ws = _workspace(n, q.device, sp)
-    rc = lib.pivot_index_ws(q.data_ptr(), k.data_ptr(), L, H, d, g, top_k, Kc, mode, out.data_ptr(),
-                            None if out_scores is None else out_scores.data_ptr(), ws.data_ptr(), ws.numel(), sp)
+    if out_proxy is None and out_cand is None:
+        rc = lib.pivot_index_ws(q.data_ptr(), k.data_ptr(), L, H, d, g, top_k, Kc, bits, out.data_ptr(),
+                                _ptr(out_scores), ws.data_ptr(), ws.numel(), sp)
+    else:
+        rc = lib.pivot_index_ex(q.data_ptr(), k.data_ptr(), L, H, d, g, top_k, Kc, bits, out.data_ptr(),
+                                _ptr(out_scores), _ptr(out_proxy), _ptr(out_cand), ws.data_ptr(), ws.numel(), sp)
     _err(lib, rc)
     return out
 
@@ -158,10 +192,12 @@ def dense_index(q, k, top_k, out=None, out_scores=None, stream=None):
 
 
 def pivot_decode_index(q, kcache, cu_seqlens, g, top_k, Kc, mode=REFINE, max_seqlen=None, out=None,
-                       out_scores=None, stream=None):
+                       out_scores=None, stream=None, proxy="fp32", out_proxy=None, out_cand=None):
     """PIVOT decode indexer: q bf16 [B, g, H, d], kcache bf16 [rows, H, d], cu_seqlens int32 [B+1]
-    (device) -> int32 [B, g, H, top_k].  max_seqlen bounds every sequence's cache rows."""
+    (device) -> int32 [B, g, H, top_k].  max_seqlen bounds every sequence's cache rows.
+    out_proxy (float32 [B, H, d]) and out_cand (int32 [B, H, Kc], Refine only) as in pivot_index."""
     lib = load_library()
+    bits = _mode_bits(mode, proxy)
     _check_bf16("q", q, 4)
     _check_bf16("kcache", kcache, 3)
     B, gq, H, d = q.shape
@@ -174,13 +210,21 @@ def pivot_decode_index(q, kcache, cu_seqlens, g, top_k, Kc, mode=REFINE, max_seq
     out = _out(out, (B, g, H, top_k), torch.int32, q.device, "out")
     if out_scores is not None:
         out_scores = _out(out_scores, (B, g, H, top_k), torch.float32, q.device, "out_scores")
+    if out_proxy is not None:
+        out_proxy = _out(out_proxy, (B, H, d), torch.float32, q.device, "out_proxy")
+    if out_cand is not None:
+        out_cand = _out(out_cand, (B, H, Kc), torch.int32, q.device, "out_cand")
     sp = _stream_ptr(stream)
-    n = lib.pivot_decode_workspace_size(B, H, d, g, top_k, Kc, mode, int(max_seqlen))
+    n = lib.pivot_decode_workspace_size(B, H, d, g, top_k, Kc, bits, int(max_seqlen))
     ws = _workspace(n, q.device, sp)
-    rc = lib.pivot_decode_index_ws(q.data_ptr(), kcache.data_ptr(), cu_seqlens.data_ptr(), B, H, d, g, top_k, Kc,
-                                   mode, int(max_seqlen), out.data_ptr(),
-                                   None if out_scores is None else out_scores.data_ptr(), ws.data_ptr(),
-                                   ws.numel(), sp)
+    if out_proxy is None and out_cand is None:
+        rc = lib.pivot_decode_index_ws(q.data_ptr(), kcache.data_ptr(), cu_seqlens.data_ptr(), B, H, d, g, top_k,
+                                       Kc, bits, int(max_seqlen), out.data_ptr(), _ptr(out_scores), ws.data_ptr(),
+                                       ws.numel(), sp)
+    else:
+        rc = lib.pivot_decode_index_ex(q.data_ptr(), kcache.data_ptr(), cu_seqlens.data_ptr(), B, H, d, g, top_k,
+                                       Kc, bits, int(max_seqlen), out.data_ptr(), _ptr(out_scores),
+                                       _ptr(out_proxy), _ptr(out_cand), ws.data_ptr(), ws.numel(), sp)
     _err(lib, rc)
     return out
 

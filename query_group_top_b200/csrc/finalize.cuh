@@ -29,8 +29,9 @@ struct FinalizeParams {
   int* fb_list;    // rows handed to the fallback kernel
   int* fb_count;
   int* status;
-  // fallback only
-  const uint16_t* proxy;  // [G][H][d] bf16 bits (the scan's A operand)
+  // fallback only: the scan's operand, one of
+  const float* proxy32;   // [G][H][d] fp32 proxies (PIVOT)
+  const uint16_t* proxy16;  // [G][H][d] bf16 bits (dense: the queries)
   const uint16_t* keys;   // [L][H][d] bf16 bits
   int d;
   uint32_t* fb_scratch;   // [gridDim.x][L] order keys
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
 }
 
 // Exact path for rows the filter could not settle: recompute the row's scores
-// over its whole prefix (CUDA cores, fp32) and select from all of them.
+// over its whole prefix (CUDA cores, fp32 proxy times bf16 keys, fp32
+// accumulation) and select from all of them.
 __global__ void __launch_bounds__(kFbNT) fallback_kernel(FinalizeParams p) {
   __shared__ SelectSmem<kFbNT> sm;
   __shared__ float pv[128];
@@ -160,8 +162,8 @@ __global__ void __launch_bounds__(kFbNT) fallback_kernel(FinalizeParams p) {
     const int K = min(p.K_sel, bound);
     __syncthreads();
     for (int c = threadIdx.x; c < p.d; c += kFbNT) {
-      const uint32_t b = static_cast<uint32_t>(p.proxy[(static_cast<long long>(i) * p.H + h) * p.d + c]) << 16;
-      pv[c] = __uint_as_float(b);
+      const long long o = (static_cast<long long>(i) * p.H + h) * p.d + c;
+      pv[c] = p.proxy32 ? p.proxy32[o] : __uint_as_float(static_cast<uint32_t>(p.proxy16[o]) << 16);
     }
     __syncthreads();
     for (int j = threadIdx.x; j < bound; j += kFbNT) {

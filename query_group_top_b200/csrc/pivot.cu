@@ -2,7 +2,8 @@
 // workspace layout, TMA descriptors and the launch sequence of each call.
 //
 // Prefill (pivot_index / dense_index), per head pass:
-//   proxy_kernel        group means -> bf16 proxies          (skipped for dense)
+//   proxy_kernel        group means -> fp32 proxies and their three bf16
+//                       terms                                 (skipped for dense)
 //   scan_filter_kernel  tcgen05 prefix scan + threshold filter -> spill lists
 //   finalize_kernel     exact top-K per row from the spill list
 //   fallback_kernel     exact recompute for rows the filter could not settle
@@ -189,8 +190,9 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   p.nfb = 2 * std::max(1, sms);
   const size_t rows_pass = static_cast<size_t>(p.heads_per_pass) * p.G;
   size_t o = 0;
+  // fp32 proxies [G][H][d], then their bf16 terms [3][G][H][d]
   p.off_proxy = o;
-  o += dense ? 0 : up(static_cast<size_t>(p.G) * H * d * 2);
+  o += dense ? 0 : up(static_cast<size_t>(p.G) * H * d * 4) + up(static_cast<size_t>(3) * p.G * H * d * 2);
   p.off_spill = o;
   o += up(rows_pass * p.cap * sizeof(uint2));
   p.off_cnt = o;
@@ -216,6 +218,10 @@ uint32_t tmem_cols_for(int Kc) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The mode argument: PIVOT_REFINE or PIVOT_REUSE, optionally OR-ed with PIVOT_PROXY_BF16.
+int base_mode(int mode) { return mode & ~static_cast<int>(PIVOT_PROXY_BF16); }
+bool proxy_bf16(int mode) { return (mode & PIVOT_PROXY_BF16) != 0; }
+
 int check_common(const void* q, const void* k, int H, int d, int top_k, int Kc, int mode, const void* out) {
   if (!q || !k || !out) return fail(PIVOT_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(out))
@@ -224,7 +230,8 @@ int check_common(const void* q, const void* k, int H, int d, int top_k, int Kc, 
   if (d != 64 && d != 128) return fail(PIVOT_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", d);
   if (top_k < 1 || Kc < top_k || Kc > 4096)
     return fail(PIVOT_ERR_INVALID_ARG, "need 1 <= top_k <= Kc <= 4096 (top_k=%d, Kc=%d)", top_k, Kc);
-  if (mode != PIVOT_REFINE && mode != PIVOT_REUSE) return fail(PIVOT_ERR_INVALID_ARG, "mode must be 0 or 1");
+  if (base_mode(mode) != PIVOT_REFINE && base_mode(mode) != PIVOT_REUSE)
+    return fail(PIVOT_ERR_INVALID_ARG, "mode must be PIVOT_REFINE or PIVOT_REUSE, optionally | PIVOT_PROXY_BF16");
   return PIVOT_OK;
 }
 
@@ -259,13 +266,40 @@ int launch_refine(RefineParams rp, int units, int sms, cudaStream_t st) {
 }
 
 // Shared prefill driver (PIVOT Refine/Reuse, and dense when `dense`).
-int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode, bool dense,
-                int32_t* out, float* out_scores, void* ws, size_t ws_bytes, cudaStream_t st) {
+// Copies candidate rows from the refine kernel's read order ([H][G][CW]) to
+// the plain layout out[unit][h][Kc]: ascending key indices, -1 padding.  Row
+// (h, u) holds n = min(Kc, bound) candidates; bound is the Refine scan bound
+// (prefill: the group's last position; decode: n_b + g - 1, or no candidates
+// for a sequence the decode scan skipped).
+__global__ void cand_export_kernel(const int32_t* __restrict__ cand, int32_t* __restrict__ out, int G, int H,
+                                   int Kc, int g, int L, const int32_t* __restrict__ cu, int max_seqlen) {
+  const int h = blockIdx.x / G, u = blockIdx.x % G;
+  int bound;
+  if (cu == nullptr) {
+    bound = min(u * g + g, L) - 1;
+  } else {
+    const int len = cu[u + 1] - cu[u];
+    bound = (len > max_seqlen || len < g) ? 0 : len - 1;
+  }
+  const int n = min(Kc, max(bound, 0));
+  const int nch = (n + 127) / 128;
+  const int32_t* row = cand + (static_cast<long long>(h) * G + u) * cand_row_words(Kc);
+  int32_t* dst = out + (static_cast<long long>(u) * H + h) * Kc;
+  for (int t = threadIdx.x; t < Kc; t += blockDim.x) dst[t] = t < n ? row[cand_word(t, nch)] : -1;
+}
+
+int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode_bits,
+                bool dense, int32_t* out, float* out_scores, float* out_proxy, int32_t* out_cand, void* ws,
+                size_t ws_bytes, cudaStream_t st) {
+  const int mode = base_mode(mode_bits);
   if (L < 1) return fail(PIVOT_ERR_INVALID_ARG, "L must be >= 1");
   if (!dense && g < 1) return fail(PIVOT_ERR_INVALID_ARG, "g must be >= 1");
   if (static_cast<long long>(L) * H * d >= (1ll << 40)) return fail(PIVOT_ERR_INVALID_ARG, "tensor too large");
   if (L >= (1 << 30)) return fail(PIVOT_ERR_INVALID_ARG, "L too large");
   if (out_scores && !aligned16(out_scores)) return fail(PIVOT_ERR_INVALID_ARG, "out_scores must be 16-byte aligned");
+  if (out_proxy && !aligned16(out_proxy)) return fail(PIVOT_ERR_INVALID_ARG, "out_proxy must be 16-byte aligned");
+  if (out_cand && mode != PIVOT_REFINE)
+    return fail(PIVOT_ERR_INVALID_ARG, "out_cand is only produced in PIVOT_REFINE mode");
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
   const Plan pl = plan_prefill(L, H, d, dense ? 1 : g, top_k, Kc, mode, dense, dev->sms);
@@ -274,16 +308,25 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return fail(PIVOT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   uint8_t* w = static_cast<uint8_t*>(ws);
-  const uint16_t* P = dense ? static_cast<const uint16_t*>(q) : reinterpret_cast<const uint16_t*>(w + pl.off_proxy);
+  // scan operand: the queries themselves (dense), else the proxies' bf16 terms
+  float* P32 = dense ? nullptr : reinterpret_cast<float*>(w + pl.off_proxy);
+  const uint16_t* P = dense ? static_cast<const uint16_t*>(q)
+                            : reinterpret_cast<const uint16_t*>(w + pl.off_proxy +
+                                                                up(static_cast<size_t>(pl.G) * H * d * 4));
   const int gg = dense ? 1 : g;
   const bool refine = !dense && mode == PIVOT_REFINE;
+  // a proxy of one member is that member's bf16 query: its mid and lo terms are zero
+  const int nterms = (dense || gg == 1 || proxy_bf16(mode_bits)) ? 1 : 3;
 
   if (!dense) {
     const long long n = static_cast<long long>(pl.G) * H * (d / 8);
     TraceScope tr("proxy", st);
     proxy_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-        static_cast<const uint16_t*>(q), reinterpret_cast<uint16_t*>(w + pl.off_proxy), pl.G, H, d, gg, L, 0);
+        static_cast<const uint16_t*>(q), P32, const_cast<uint16_t*>(P), pl.G, H, d, gg, L, 0,
+        proxy_bf16(mode_bits) ? 1 : 0);
     CUDA_TRY(cudaGetLastError());
+    if (out_proxy)
+      CUDA_TRY(cudaMemcpyAsync(out_proxy, P32, static_cast<size_t>(pl.G) * H * d * 4, cudaMemcpyDeviceToDevice, st));
   }
 
   for (int h0 = 0; h0 < H; h0 += pl.heads_per_pass) {
@@ -292,7 +335,8 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     const uint16_t* Ph = P + static_cast<size_t>(h0) * d;
     const uint16_t* Kh = static_cast<const uint16_t*>(k) + static_cast<size_t>(h0) * d;
     CUtensorMap tmP, tmK;
-    if (int rc = make_rows_map(&tmP, Ph, pl.G, nh, H, d, 128)) return rc;
+    // the proxy view spans the three term tensors: term t's rows start at t*G
+    if (int rc = make_rows_map(&tmP, Ph, dense ? pl.G : 3 * pl.G, nh, H, d, 128)) return rc;
     if (int rc = make_rows_map(&tmK, Kh, L, nh, H, d, ScanCfg<128>::BN)) return rc;
     ScanParams sp{};
     sp.G = pl.G;
@@ -304,6 +348,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     sp.cap = pl.cap;
     sp.S = pl.S;
     sp.tiles_per_head = (pl.G + ScanCfg<128>::BM - 1) / ScanCfg<128>::BM;
+    sp.nterms = nterms;
     sp.spill = reinterpret_cast<uint2*>(w + pl.off_spill);
     sp.cnt = reinterpret_cast<int4*>(w + pl.off_cnt);
     sp.status = dev->status;
@@ -330,7 +375,8 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     fp.fb_list = reinterpret_cast<int*>(w + pl.off_fblist);
     fp.fb_count = reinterpret_cast<int*>(w + pl.off_fb);
     fp.status = dev->status;
-    fp.proxy = Ph;
+    fp.proxy32 = dense ? nullptr : P32 + static_cast<size_t>(h0) * d;
+    fp.proxy16 = dense ? Ph : nullptr;
     fp.keys = Kh;
     fp.d = d;
     fp.fb_scratch = reinterpret_cast<uint32_t*>(w + pl.off_fbscratch);
@@ -369,6 +415,11 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.d = d;
     rp.tmem_cols = tmem_cols_for(Kc);
     rp.status = dev->status;
+    if (out_cand) {
+      cand_export_kernel<<<static_cast<unsigned>(H * pl.G), 256, 0, st>>>(rp.cand, out_cand, pl.G, H, Kc, g, L,
+                                                                          nullptr, 0);
+      CUDA_TRY(cudaGetLastError());
+    }
     int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, dev->sms, st) : launch_refine<64>(rp, H * pl.G, dev->sms, st);
     if (rc) return rc;
   }
@@ -376,7 +427,8 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
 }
 
 size_t decode_ws_size(int B, int H, int d, int Kc, int mode, int max_seqlen) {
-  size_t o = up(static_cast<size_t>(B) * H * d * 2);                        // proxies
+  mode = base_mode(mode);
+  size_t o = up(static_cast<size_t>(B) * H * d * 4);                        // fp32 proxies
   o += up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t));       // order keys
   if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
   return o;
@@ -393,9 +445,13 @@ int check_decode(const void* q, const void* kc, const int32_t* cu, int B, int H,
 }
 
 int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, int d, int g, int top_k, int Kc,
-               int mode, int max_seqlen, int32_t* out, float* out_scores, void* ws, size_t ws_bytes,
-               cudaStream_t st) {
-  if (int rc = check_decode(q, kc, cu, B, H, d, g, top_k, Kc, mode, max_seqlen, out, out_scores)) return rc;
+               int mode_bits, int max_seqlen, int32_t* out, float* out_scores, float* out_proxy, int32_t* out_cand,
+               void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (int rc = check_decode(q, kc, cu, B, H, d, g, top_k, Kc, mode_bits, max_seqlen, out, out_scores)) return rc;
+  const int mode = base_mode(mode_bits);
+  if (out_proxy && !aligned16(out_proxy)) return fail(PIVOT_ERR_INVALID_ARG, "out_proxy must be 16-byte aligned");
+  if (out_cand && mode != PIVOT_REFINE)
+    return fail(PIVOT_ERR_INVALID_ARG, "out_cand is only produced in PIVOT_REFINE mode");
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
   const size_t need = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
@@ -403,17 +459,20 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return fail(PIVOT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   uint8_t* w = static_cast<uint8_t*>(ws);
-  uint16_t* P = reinterpret_cast<uint16_t*>(w);
-  uint32_t* scores = reinterpret_cast<uint32_t*>(w + up(static_cast<size_t>(B) * H * d * 2));
-  int32_t* cand = reinterpret_cast<int32_t*>(w + up(static_cast<size_t>(B) * H * d * 2) +
+  float* P = reinterpret_cast<float*>(w);
+  uint32_t* scores = reinterpret_cast<uint32_t*>(w + up(static_cast<size_t>(B) * H * d * 4));
+  int32_t* cand = reinterpret_cast<int32_t*>(w + up(static_cast<size_t>(B) * H * d * 4) +
                                              up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t)));
   const long long n = static_cast<long long>(B) * H * (d / 8);
   {
+    // the decode scan multiplies by the fp32 proxy directly: no bf16 terms
     TraceScope tr("proxy", st);
-    proxy_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(static_cast<const uint16_t*>(q), P, B, H,
-                                                                          d, g, 0, 1);
+    proxy_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(static_cast<const uint16_t*>(q), P, nullptr,
+                                                                          B, H, d, g, 0, 1,
+                                                                          proxy_bf16(mode_bits) ? 1 : 0);
   }
   CUDA_TRY(cudaGetLastError());
+  if (out_proxy) CUDA_TRY(cudaMemcpyAsync(out_proxy, P, static_cast<size_t>(B) * H * d * 4, cudaMemcpyDeviceToDevice, st));
   DecodeParams dp{};
   dp.kcache = static_cast<const uint16_t*>(kc);
   dp.P = P;
@@ -465,6 +524,10 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     rp.d = d;
     rp.tmem_cols = tmem_cols_for(Kc);
     rp.status = dev->status;
+    if (out_cand) {
+      cand_export_kernel<<<static_cast<unsigned>(H * B), 256, 0, st>>>(cand, out_cand, B, H, Kc, g, 0, cu, max_seqlen);
+      CUDA_TRY(cudaGetLastError());
+    }
     int rc = (d == 128) ? launch_refine<128>(rp, H * B, dev->sms, st) : launch_refine<64>(rp, H * B, dev->sms, st);
     if (rc) return rc;
   }
@@ -541,14 +604,14 @@ int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t*
   if (int rc = noalloc_scratch(&scratch)) return rc;
   // Nothing in the decode scratch has to start at zero: every word is written
   // before it is read within the call.
-  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, scratch,
-                    kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
+  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
+                    nullptr, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
 
 size_t pivot_workspace_size(int L, int H, int d, int g, int top_k, int Kc, int mode) {
   if (L < 1 || H < 1 || g < 1 || top_k < 1 || Kc < top_k) return 0;
-  return plan_prefill(L, H, d, g, top_k, Kc, mode, false, device_sms()).total;
+  return plan_prefill(L, H, d, g, top_k, Kc, base_mode(mode), false, device_sms()).total;
 }
 
 size_t dense_workspace_size(int L, int H, int d, int top_k) {
@@ -566,8 +629,16 @@ size_t pivot_decode_workspace_size(int B, int H, int d, int g, int top_k, int Kc
 int pivot_index_ws(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
                    int32_t* out_idx, float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
   if (int rc = check_common(q, k, H, d, top_k, Kc, mode, out_idx)) return rc;
-  return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, out_scores, workspace, workspace_bytes,
-                     static_cast<cudaStream_t>(stream));
+  return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, out_scores, nullptr, nullptr, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pivot_index_ex(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
+                   int32_t* out_idx, float* out_scores, float* out_proxy, int32_t* out_cand, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (int rc = check_common(q, k, H, d, top_k, Kc, mode, out_idx)) return rc;
+  return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, out_scores, out_proxy, out_cand, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int pivot_index(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
@@ -577,17 +648,17 @@ int pivot_index(const void* q, const void* k, int L, int H, int d, int g, int to
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = plan_prefill(L, H, d, g, top_k, Kc, mode, false, dev->sms).total;
+  const size_t bytes = plan_prefill(L, H, d, g, top_k, Kc, base_mode(mode), false, dev->sms).total;
   return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
-    return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, nullptr, ws, n, st);
+    return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, nullptr, nullptr, nullptr, ws, n, st);
   });
 }
 
 int dense_index_ws(const void* q, const void* k, int L, int H, int d, int top_k, int32_t* out_idx,
                    float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
   if (int rc = check_common(q, k, H, d, top_k, top_k, PIVOT_REUSE, out_idx)) return rc;
-  return run_prefill(q, k, L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, out_idx, out_scores, workspace,
-                     workspace_bytes, static_cast<cudaStream_t>(stream));
+  return run_prefill(q, k, L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, out_idx, out_scores, nullptr, nullptr,
+                     workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int dense_index(const void* q, const void* k, int L, int H, int d, int top_k, int32_t* out_idx, void* stream) {
@@ -598,15 +669,24 @@ int dense_index(const void* q, const void* k, int L, int H, int d, int top_k, in
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = plan_prefill(L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, dev->sms).total;
   return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
-    return run_prefill(q, k, L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, out_idx, nullptr, ws, n, st);
+    return run_prefill(q, k, L, H, d, 1, top_k, top_k, PIVOT_REUSE, true, out_idx, nullptr, nullptr, nullptr, ws,
+                       n, st);
   });
 }
 
 int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
                           int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
-  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, workspace,
-                    workspace_bytes, static_cast<cudaStream_t>(stream));
+  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
+                    nullptr, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pivot_decode_index_ex(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d, int g,
+                          int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx, float* out_scores,
+                          float* out_proxy, int32_t* out_cand, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, out_proxy,
+                    out_cand, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int pivot_decode_index(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d, int g,
@@ -618,7 +698,8 @@ int pivot_decode_index(const void* q, const void* kcache, const int32_t* cu_seql
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
   return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
-    return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr, ws, n, st);
+    return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr, nullptr,
+                      nullptr, ws, n, st);
   });
 }
 

@@ -1,18 +1,26 @@
 // Proxy build (prefill and decode) and the decode-side scan and select.
 //
 // Proxy: "PIVOT explained", "How It Works": proxy_q = mean(group); the mean is
-// accumulated in fp64 in member order, divided by the member count, rounded
-// to fp32 and then to bf16 (the scan's tensor-core operand).  A partial last
-// group averages over its actual members.
+// accumulated in fp64 in member order, divided by the member count and
+// rounded to fp32: the fp32 mean is the scan's operand.  A partial last group
+// averages over its actual members.  For the tensor-core scan the fp32 mean is
+// split exactly into three bf16 terms, p = hi + mid + lo: hi = bf16(p), mid =
+// bf16(p - hi), lo = p - hi - mid.  Each difference is exact in fp32 (the
+// operands lie within a factor of two of each other), p - hi carries at most
+// 16 significant bits and p - hi - mid at most 8, so lo is a bf16 value and
+// the three terms sum to p exactly (for |p| >= 2^-110 or p = 0, where lo is
+// not a bf16 subnormal that loses bits).  Three MMAs over the same key tile
+// then accumulate p . k with only fp32 accumulation error.  The variant
+// flag rounds the fp32 mean to bf16 and scans with that value alone.
 //
 // Decode (paper abstract: in decode a group is "the queries decoded together
 // in one multi-token prediction step"): one group per sequence, members at
 // positions n_b .. n_b+g-1 of a packed key cache.  With a single proxy row per
 // (sequence, head) the scan is a matrix-vector product bound by HBM: each warp
-// streams 16-byte slices of consecutive key rows, reduces each row's dot
-// product with shuffles and writes one 32-bit order key per key (4 bytes per
-// 256 key bytes read).  An exact block select then keeps the top-K per
-// (sequence, head).
+// streams 16-byte slices of consecutive key rows, multiplies them by the fp32
+// proxy, reduces each row's dot product with shuffles and writes one 32-bit
+// order key per key (4 bytes per 256 key bytes read).  An exact block select
+// then keeps the top-K per (sequence, head).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -22,10 +30,14 @@
 
 namespace pivot {
 
-// P[u][h][:] for units u < G.  Prefill: members are positions u*g .. min(u*g+g, L)-1
-// of q [L][H][d].  Decode (decode != 0): members are rows u*g .. u*g+g-1 of q [B*g][H][d].
-__global__ void proxy_kernel(const uint16_t* __restrict__ q, uint16_t* __restrict__ P, int G, int H, int d,
-                             int g, int L, int decode) {
+// Proxy of unit u (u < G), head h: P32[u][h][:] fp32 and, when P3 is not
+// null, its three bf16 terms P3[t][u][h][:] (t = 0 hi, 1 mid, 2 lo).
+// Prefill: members are positions u*g .. min(u*g+g, L)-1 of q [L][H][d].
+// Decode (decode != 0): members are rows u*g .. u*g+g-1 of q [B*g][H][d].
+// bf16_proxy != 0: the proxy is the fp32 mean rounded to bf16 (P32 holds that
+// value, hi is it, mid and lo are zero).
+__global__ void proxy_kernel(const uint16_t* __restrict__ q, float* __restrict__ P32, uint16_t* __restrict__ P3,
+                             int G, int H, int d, int g, int L, int decode, int bf16_proxy) {
   const long long total = static_cast<long long>(G) * H * (d / 8);
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= total) return;
@@ -45,21 +57,38 @@ __global__ void proxy_kernel(const uint16_t* __restrict__ q, uint16_t* __restric
       acc[2 * k + 1] += static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u));
     }
   }
-  uint32_t o[4];
+  float pm[8];
+  uint32_t th[8], tm[8], tl[8];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float lo = __double2float_rn(__ddiv_rn(acc[2 * k], static_cast<double>(n)));
-    const float hi = __double2float_rn(__ddiv_rn(acc[2 * k + 1], static_cast<double>(n)));
-    const uint32_t blo = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-    const uint32_t bhi = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    o[k] = blo | (bhi << 16);
+  for (int k = 0; k < 8; ++k) {
+    float p = __double2float_rn(__ddiv_rn(acc[k], static_cast<double>(n)));
+    if (bf16_proxy) p = __bfloat162float(__float2bfloat16_rn(p));
+    pm[k] = p;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+    const float r1 = __fsub_rn(p, __bfloat162float(hi));      // exact
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = __fsub_rn(r1, __bfloat162float(mid));    // exact, a bf16 value
+    th[k] = __bfloat16_as_ushort(hi);
+    tm[k] = __bfloat16_as_ushort(mid);
+    tl[k] = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
   }
-  *reinterpret_cast<uint4*>(P + (static_cast<long long>(u) * H + h) * d + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+  const long long o = (static_cast<long long>(u) * H + h) * d + c8 * 8;
+  reinterpret_cast<float4*>(P32 + o)[0] = make_float4(pm[0], pm[1], pm[2], pm[3]);
+  reinterpret_cast<float4*>(P32 + o)[1] = make_float4(pm[4], pm[5], pm[6], pm[7]);
+  if (P3) {
+    const long long term = static_cast<long long>(G) * H * d;
+    *reinterpret_cast<uint4*>(P3 + o) =
+        make_uint4(th[0] | th[1] << 16, th[2] | th[3] << 16, th[4] | th[5] << 16, th[6] | th[7] << 16);
+    *reinterpret_cast<uint4*>(P3 + term + o) =
+        make_uint4(tm[0] | tm[1] << 16, tm[2] | tm[3] << 16, tm[4] | tm[5] << 16, tm[6] | tm[7] << 16);
+    *reinterpret_cast<uint4*>(P3 + 2 * term + o) =
+        make_uint4(tl[0] | tl[1] << 16, tl[2] | tl[3] << 16, tl[4] | tl[5] << 16, tl[6] | tl[7] << 16);
+  }
 }
 
 struct DecodeParams {
   const uint16_t* kcache;   // [rows][H][d]
-  const uint16_t* P;        // [B][H][d] proxies
+  const float* P;           // [B][H][d] fp32 proxies
   const int32_t* cu;        // [B+1]
   uint32_t* scores;         // [H*B][max_seqlen] order keys
   int32_t* cand;            // [H][B][cand_row_words(K_sel)] candidate rows (Refine)
@@ -99,13 +128,10 @@ __global__ void __launch_bounds__(kDecNT) decode_scan_kernel(DecodeParams p) {
   const int sub = lane / LPK, part = lane % LPK;
   float pf[8];
   {
-    const uint4 v = *reinterpret_cast<const uint4*>(p.P + (static_cast<long long>(b) * p.H + h) * D + part * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      pf[2 * k] = __uint_as_float(w[k] << 16);
-      pf[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-    }
+    const float4* pp = reinterpret_cast<const float4*>(p.P + (static_cast<long long>(b) * p.H + h) * D + part * 8);
+    const float4 a = pp[0], c = pp[1];
+    pf[0] = a.x; pf[1] = a.y; pf[2] = a.z; pf[3] = a.w;
+    pf[4] = c.x; pf[5] = c.y; pf[6] = c.z; pf[7] = c.w;
   }
   const uint16_t* kb = p.kcache + (static_cast<long long>(p.cu[b]) * p.H + h) * D + part * 8;
   const long long kstride = static_cast<long long>(p.H) * D;

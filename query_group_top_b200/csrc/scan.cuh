@@ -9,7 +9,11 @@
 //
 // One CTA owns 128 proxy rows of one head (M = 128) and streams the head's
 // keys in tiles of 128 (N = 128, K = d) through a TMA -> shared -> tcgen05.mma
-// -> TMEM pipeline with four accumulators:
+// -> TMEM pipeline with four accumulators.  The proxy rows stay in shared
+// memory as nterms bf16 tiles: the exact three-term split of the fp32 mean
+// (hi + mid + lo), or one tile for the dense indexer (the query itself) and
+// for the bf16-proxy variant.  Every key tile is multiplied by each term into
+// the same accumulator, so a score is p . k with fp32 accumulation.
 //   warp 0      TMA producer (keys, and the proxy tile once)
 //   warp 1      TMEM allocator and MMA issuer (one elected thread)
 //   warps 2..17 epilogue, four groups of four: thread (e, r) owns TMEM lane r
@@ -47,6 +51,7 @@ struct ScanParams {
   int cap;         // spill capacity per row (entries, even)
   int S;           // sample stride in key tiles (every S-th tile is sampled)
   int tiles_per_head;
+  int nterms;      // bf16 proxy terms (1 or 3); term t's rows start at t*G in the proxy tensor map
   uint2* spill;    // [H*G][cap]: (score bits, key index); see cnt
   int4* cnt;       // [H*G]: survivors of the four runs (key quarters q = 0..3).
                    // Run q lives in region q/2 = [q/2 * cap/2, (q/2+1) * cap/2):
@@ -67,12 +72,13 @@ struct ScanCfg {
   static constexpr int BN = 128;                      // keys per tile (MMA N)
   static constexpr int NACC = 4;                      // TMEM accumulators = epilogue groups
   static constexpr int KATOMS = D / 64;               // 64-element (128-byte) K slices
-  static constexpr int NST = (D == 128) ? 4 : 8;      // key-tile stages in shared memory
-  static constexpr int A_BYTES = BM * D * 2;
+  static constexpr int NTERMS = 3;                    // proxy tiles held (the most any call uses)
+  static constexpr int NST = (D == 128) ? 2 : 6;      // key-tile stages in shared memory
+  static constexpr int A_BYTES = BM * D * 2;          // one proxy term
   static constexpr int B_BYTES = BN * D * 2;
   static constexpr int HIST_BYTES = 128 * BM * 4;     // [128 bin pairs][128 rows], two u16 counts per word
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + A_BYTES;
+  static constexpr int OFF_B = OFF_A + NTERMS * A_BYTES;
   static constexpr int OFF_HIST = OFF_B + NST * B_BYTES;
   static constexpr int OFF_MISC = OFF_HIST + HIST_BYTES;  // per-row sample counts
   static constexpr int OFF_BAR = OFF_MISC + BM * 4;
@@ -163,9 +169,10 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
     if (lane == 0 && 2 * ns + nkt > 0) {
       tma_prefetch_desc(&tm_proxy);
       tma_prefetch_desc(&tm_keys);
-      mbar_arrive_expect_tx(a_full, C::A_BYTES);
-      for (int a = 0; a < C::KATOMS; ++a)
-        tma_load_3d(sA + a * (C::BM * 128), &tm_proxy, a_full, a * 64, h, i0);
+      mbar_arrive_expect_tx(a_full, p.nterms * C::A_BYTES);
+      for (int tt = 0; tt < p.nterms; ++tt)
+        for (int a = 0; a < C::KATOMS; ++a)
+          tma_load_3d(sA + tt * C::A_BYTES + a * (C::BM * 128), &tm_proxy, a_full, a * 64, h, tt * p.G + i0);
       int step = 0, issued = 0;
       bool ok = true;
       for_each_step(ns, p.S, nkt, [&](int, int jt, int) {
@@ -208,12 +215,14 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + q * C::BN;
+        for (int tt = 0; tt < p.nterms; ++tt) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int a = kk >> 2, k4 = kk & 3;
-          const uint64_t adesc = sw128_kmajor_desc(sA + a * (C::BM * 128) + k4 * 32);
-          const uint64_t bdesc = sw128_kmajor_desc(sB + s * C::B_BYTES + a * (C::BN * 128) + k4 * 32);
-          umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int a = kk >> 2, k4 = kk & 3;
+            const uint64_t adesc = sw128_kmajor_desc(sA + tt * C::A_BYTES + a * (C::BM * 128) + k4 * 32);
+            const uint64_t bdesc = sw128_kmajor_desc(sB + s * C::B_BYTES + a * (C::BN * 128) + k4 * 32);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (tt > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(empty_bar(s));
         umma_commit(tfull_bar(q));

@@ -54,3 +54,23 @@ def assert_parity(res, what=""):
     assert res["mismatch"] == 0, f"{what}: {res}"
     assert res["invalid"] == 0, f"{what}: {res}"
     assert res.get("score_bad", 0) == 0, f"{what}: {res}"
+
+
+def oracle_threads(fn, q, k, g, top_k, Kc, mode, units_a, units_b, threads=None, **kw):
+    """Runs an oracle *_units function over its units on several host threads
+    (the oracle is plain C called through ctypes, which releases the GIL, and
+    keeps no global state) and joins the per-unit results in unit order."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    n = len(units_a)
+    threads = threads or max(1, min(len(os.sched_getaffinity(0)), 32, n))
+    cuts = np.linspace(0, n, threads + 1).astype(int)
+    parts = [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+    with ThreadPoolExecutor(len(parts)) as ex:
+        res = list(ex.map(lambda ab: fn(q, k, g, top_k, Kc, mode, units_a[ab[0]:ab[1]], units_b[ab[0]:ab[1]], **kw),
+                          parts))
+    out = {}
+    for key in res[0]:
+        vals = [r[key] for r in res]
+        out[key] = None if vals[0] is None else np.concatenate(vals, axis=0)
+    return out

@@ -12,7 +12,7 @@ import torch
 import oracle
 import query_group_top_b200 as qg
 import synthetic
-from tests.parity import assert_parity, compare, valid_rows
+from tests.parity import assert_parity, compare, near_tie, oracle_threads, valid_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -21,39 +21,40 @@ def to_dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def run_prefill(q, k, g, top_k, Kc, mode, dense=False):
+def run_prefill(q, k, g, top_k, Kc, mode, dense=False, proxy="fp32"):
     qd, kd = to_dev(q), to_dev(k)
     L, H, _ = q.shape
     sc = torch.empty((L, H, top_k), dtype=torch.float32, device="cuda")
     if dense:
         out = qg.dense_index(qd, kd, top_k, out_scores=sc)
     else:
-        out = qg.pivot_index(qd, kd, g, top_k, Kc, mode, out_scores=sc)
+        out = qg.pivot_index(qd, kd, g, top_k, Kc, mode, out_scores=sc, proxy=proxy)
     flags = qg.sync_status()
     return out.cpu().numpy(), sc.cpu().numpy(), flags
 
 
-def check_full(q, k, g, top_k, Kc, mode, dense=False):
-    got, gs, flags = run_prefill(q, k, g, top_k, Kc, mode, dense)
+def check_full(q, k, g, top_k, Kc, mode, dense=False, proxy="fp32"):
+    got, gs, flags = run_prefill(q, k, g, top_k, Kc, mode, dense, proxy)
     L, H, _ = q.shape
     pos = np.broadcast_to(np.arange(L)[:, None], (L, H))
     if dense:
         ref = oracle.dense(q, k, top_k)
         cedge = None
     else:
-        ref = oracle.prefill(q, k, g, top_k, Kc, mode)
+        ref = oracle.prefill(q, k, g, top_k, Kc, mode, proxy=proxy)
         cedge = ref["cand_edge"][np.arange(L) // g] if mode == oracle.REFINE else None
     res = compare(got, ref["out"], ref["edge"], pos, cedge, gs, ref["score"])
-    assert_parity(res, f"L={L} H={H} d={q.shape[2]} g={g} k={top_k} Kc={Kc} mode={mode} dense={dense}")
+    assert_parity(res, f"L={L} H={H} d={q.shape[2]} g={g} k={top_k} Kc={Kc} mode={mode} dense={dense} {proxy}")
     return res, flags
 
 
-@pytest.mark.parametrize("mode", ["refine", "reuse", "dense"])
+@pytest.mark.parametrize("mode", ["refine", "reuse", "dense", "refine-bf16", "reuse-bf16"])
 def test_c0_full(mode):
     c = synthetic.CONFIGS["C0"]
     q, k = synthetic.make_prefill("C0")
-    m = oracle.REFINE if mode == "refine" else oracle.REUSE
-    res, _ = check_full(q, k, c["g"], c["top_k"], c["Kc"], m, dense=(mode == "dense"))
+    m = oracle.REUSE if mode.startswith("reuse") else oracle.REFINE
+    proxy = "bf16" if mode.endswith("bf16") else "fp32"
+    res, _ = check_full(q, k, c["g"], c["top_k"], c["Kc"], m, dense=(mode == "dense"), proxy=proxy)
     assert res["exact"] + res["exempt"] == 1024 * 8
 
 
@@ -81,6 +82,32 @@ def test_small_shapes_all_modes(shape):
     check_full(q, k, g, top_k, Kc, oracle.REFINE)
     check_full(q, k, g, top_k, Kc, oracle.REUSE)
     check_full(q, k, g, top_k, Kc, oracle.REUSE, dense=True)
+    check_full(q, k, g, top_k, Kc, oracle.REFINE, proxy="bf16")
+    check_full(q, k, g, top_k, Kc, oracle.REUSE, proxy="bf16")
+
+
+@pytest.mark.parametrize("proxy", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(1024, 2, 128, 8, 64, 128), (3000, 3, 64, 5, 100, 300), (700, 1, 128, 16, 30, 64),
+                                   (2500, 2, 128, 3, 200, 2000)], ids=lambda s: "x".join(map(str, s)))
+def test_proxies_bit_exact_and_candidate_sets(shape, proxy):
+    """The proxy kernel's output equals the oracle's proxy bit for bit (the fp32
+    mean, or its bf16 rounding); every group's candidate set equals the
+    oracle's exactly unless its Kc-th and (Kc+1)-th proxy scores are a near tie."""
+    L, H, d, g, top_k, Kc = shape
+    q, k = synthetic.gen_prefill(L, H, d, seed=3 * L + g, rho=0.9)
+    G = (L + g - 1) // g
+    qd, kd = to_dev(q), to_dev(k)
+    P = torch.empty((G, H, d), dtype=torch.float32, device="cuda")
+    C = torch.empty((G, H, Kc), dtype=torch.int32, device="cuda")
+    qg.pivot_index(qd, kd, g, top_k, Kc, qg.REFINE, proxy=proxy, out_proxy=P, out_cand=C)
+    qg.sync_status()
+    ref = oracle.prefill(q, k, g, top_k, Kc, oracle.REFINE, want_cand=True, proxy=proxy)
+    want_p = ref["proxy"] if proxy == "fp32" else synthetic.bf16_to_f32(ref["proxy_bf16"])
+    np.testing.assert_array_equal(P.cpu().numpy().view(np.uint32), want_p.view(np.uint32))
+    cand = C.cpu().numpy()
+    eq = np.all(cand == ref["cand"], axis=-1)
+    assert np.all(eq | near_tie(ref["cand_edge"])), np.argwhere(~eq)[:5]
+    assert eq.mean() > 0.99
 
 
 def test_exact_ties_and_fallback_rows():
@@ -120,6 +147,24 @@ def sampled_units(G, H, n, seed):
     return gi.astype(np.int32), hi.astype(np.int32)
 
 
+def device_rows_valid(out, pos0, want_n=None):
+    """Properties of every row, checked on the device: an ascending prefix of
+    valid indices, -1 padding after it, every index < its position, and (when
+    want_n is given) want_n(pos) valid entries.  out [P, H, k] covers positions
+    pos0 .. pos0+P-1."""
+    P = out.shape[0]
+    for a in range(0, P, 2048):
+        o = out[a:a + 2048]
+        pos = torch.arange(pos0 + a, pos0 + a + o.shape[0], device=o.device, dtype=torch.int64)[:, None, None]
+        v = o >= 0
+        assert not bool((v[..., 1:] & ~v[..., :-1]).any()), "valid entry after padding"
+        assert bool(((o[..., 1:] > o[..., :-1]) | ~v[..., 1:]).all()), "not strictly ascending"
+        assert bool(((o < pos) | ~v).all()), "index not causal"
+        assert bool(((o == -1) | v).all()), "padding other than -1"
+        if want_n is not None:
+            assert bool((v.sum(-1) == want_n(pos[:, :, 0])).all()), "row size"
+
+
 def check_sampled(name, modes, n_units):
     c = synthetic.CONFIGS[name]
     q, k = synthetic.make_prefill(name)
@@ -131,37 +176,38 @@ def check_sampled(name, modes, n_units):
         sc = torch.empty((L, H, top_k), dtype=torch.float32, device="cuda")
         out = qg.pivot_index(qd, kd, g, top_k, Kc, mode, out_scores=sc)
         qg.sync_status()
-        # properties of every row
-        o = out.cpu().numpy()
-        pos = np.broadcast_to(np.arange(L)[:, None], (L, H))
-        assert valid_rows(o, pos).all()
-        if mode == oracle.REFINE:
-            want_n = np.minimum(top_k, np.arange(L))[:, None]
-            assert np.all((o >= 0).sum(-1) == want_n)
+        device_rows_valid(out, 0, (lambda p: torch.clamp(p, max=top_k)) if mode == oracle.REFINE else None)
         gi, hi = sampled_units(G, H, n_units, seed=L + mode)
-        r = oracle.prefill_units(q, k, g, top_k, Kc, mode, gi, hi)
-        s = sc.cpu().numpy()
+        r = oracle_threads(oracle.prefill_units, q, k, g, top_k, Kc, mode, gi, hi)
+        rows_all = np.concatenate([np.arange(i * g, min(i * g + g, L)) for i in gi])
+        head_all = np.concatenate([np.full(min(i * g + g, L) - i * g, h) for i, h in zip(gi, hi)])
+        ri = torch.from_numpy(rows_all).cuda()
+        hh = torch.from_numpy(head_all).cuda()
+        o = out[ri, hh].cpu().numpy()
+        s = sc[ri, hh].cpu().numpy()
+        at = 0
         for u, (i, h) in enumerate(zip(gi, hi)):
             rows = np.arange(i * g, min(i * g + g, L))
             nm = len(rows)
-            res = compare(o[rows, h], r["out"][u, :nm], r["edge"][u, :nm], rows,
+            res = compare(o[at:at + nm], r["out"][u, :nm], r["edge"][u, :nm], rows,
                           np.broadcast_to(r["cand_edge"][u], (nm, 2)) if mode == oracle.REFINE else None,
-                          s[rows, h], r["score"][u, :nm])
+                          s[at:at + nm], r["score"][u, :nm])
             assert_parity(res, f"{name} mode={mode} group={i} head={h}")
+            at += nm
         del out, sc
     torch.cuda.empty_cache()
 
 
 def test_c1_sampled():
-    check_sampled("C1", (oracle.REFINE, oracle.REUSE), 96)
+    check_sampled("C1", (oracle.REFINE, oracle.REUSE), 256)
 
 
 def test_c2_sampled():
-    check_sampled("C2", (oracle.REFINE, oracle.REUSE), 24)
+    check_sampled("C2", (oracle.REFINE, oracle.REUSE), 128)
 
 
 def test_c3_sampled():
-    check_sampled("C3", (oracle.REFINE, oracle.REUSE), 12)
+    check_sampled("C3", (oracle.REFINE, oracle.REUSE), 256)
 
 
 def test_c1_dense_sampled():
@@ -179,17 +225,41 @@ def test_c1_dense_sampled():
 
 
 # ------------------------------------------------------------------- decode
-def run_decode(dec, g, top_k, Kc, mode, max_seqlen):
+def run_decode(dec, g, top_k, Kc, mode, max_seqlen, proxy="fp32"):
     qd = to_dev(dec.q)
     kd = to_dev(dec.kcache)
     cu = torch.from_numpy(dec.cu_seqlens).cuda()
     B, _, H, _ = dec.q.shape
     sc = torch.empty((B, g, H, top_k), dtype=torch.float32, device="cuda")
-    out = qg.pivot_decode_index(qd, kd, cu, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sc)
+    out = qg.pivot_decode_index(qd, kd, cu, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sc, proxy=proxy)
     qg.sync_status()
     return out.cpu().numpy(), sc.cpu().numpy()
 
 
+@pytest.mark.parametrize("proxy", ["fp32", "bf16"])
+def test_decode_proxies_and_candidate_sets(proxy):
+    """Decode: the fp32 proxies bit for bit, and the candidate sets, against
+    the oracle (one sequence shorter than Kc, the others longer)."""
+    B, H, d, g, top_k, Kc = 4, 2, 128, 2, 64, 700
+    dec = synthetic.gen_decode(B, H, d, g, seed=91, lo=300, hi=6000)
+    max_seqlen = int(np.diff(dec.cu_seqlens).max())
+    qd, kd, cu = to_dev(dec.q), to_dev(dec.kcache), torch.from_numpy(dec.cu_seqlens).cuda()
+    P = torch.empty((B, H, d), dtype=torch.float32, device="cuda")
+    C = torch.empty((B, H, Kc), dtype=torch.int32, device="cuda")
+    qg.pivot_decode_index(qd, kd, cu, g, top_k, Kc, qg.REFINE, max_seqlen=max_seqlen, proxy=proxy, out_proxy=P,
+                          out_cand=C)
+    qg.sync_status()
+    bi, hh = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+    r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, g, top_k, Kc, oracle.REFINE, bi.ravel(), hh.ravel(),
+                            want_cand=True, proxy=proxy)
+    want_p = r["proxy"] if proxy == "fp32" else synthetic.bf16_to_f32(r["proxy_bf16"])
+    np.testing.assert_array_equal(P.cpu().numpy().reshape(B * H, d).view(np.uint32), want_p.view(np.uint32))
+    cand = C.cpu().numpy().reshape(B * H, Kc)
+    eq = np.all(cand == r["cand"], axis=-1)
+    assert np.all(eq | near_tie(r["cand_edge"])), np.argwhere(~eq)[:5]
+
+
+@pytest.mark.parametrize("proxy", ["fp32", "bf16"])
 @pytest.mark.parametrize("case", [
     # B, H, d, g, lo, hi, top_k, Kc
     (1, 1, 128, 1, 0, 0, 4, 8),
@@ -198,14 +268,15 @@ def run_decode(dec, g, top_k, Kc, mode, max_seqlen):
     (2, 1, 128, 3, 200, 9000, 300, 700),
     (5, 2, 64, 4, 50, 2500, 100, 200),
 ])
-def test_decode_small(case):
+def test_decode_small(case, proxy):
     B, H, d, g, lo, hi, top_k, Kc = case
     dec = synthetic.gen_decode(B, H, d, g, seed=B * 31 + g, lo=lo, hi=hi)
     max_seqlen = int(np.diff(dec.cu_seqlens).max())
     bi, hh = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
     for mode in (oracle.REFINE, oracle.REUSE):
-        got, gs = run_decode(dec, g, top_k, Kc, mode, max_seqlen)
-        r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, g, top_k, Kc, mode, bi.ravel(), hh.ravel())
+        got, gs = run_decode(dec, g, top_k, Kc, mode, max_seqlen, proxy)
+        r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, g, top_k, Kc, mode, bi.ravel(), hh.ravel(),
+                                proxy=proxy)
         want = r["out"].reshape(B, H, g, top_k).transpose(0, 2, 1, 3)
         edge = r["edge"].reshape(B, H, g, 2).transpose(0, 2, 1, 3)
         wsc = r["score"].reshape(B, H, g, top_k).transpose(0, 2, 1, 3)

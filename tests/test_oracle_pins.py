@@ -318,3 +318,17 @@ def test_proxy_precisions_agree_for_single_members():
         a = oracle.prefill(q, k, 1, 5, 10, mode)["out"]
         b = oracle.prefill(q, k, 1, 5, 10, mode, proxy="bf16")["out"]
         np.testing.assert_array_equal(a, b)
+
+
+def test_threaded_oracle_runs_equal_serial_runs():
+    """The tests and the bench spread oracle units over host threads; the
+    joined results must be those of one serial call."""
+    from tests.parity import oracle_threads
+    q, k = synthetic.gen_prefill(300, 3, 16, seed=12, rho=0.9)
+    gi = np.array([0, 5, 37, 12, 8, 20, 1], np.int32)
+    hi = np.array([0, 1, 2, 2, 1, 0, 1], np.int32)
+    for mode in (oracle.REFINE, oracle.REUSE):
+        a = oracle.prefill_units(q, k, 8, 5, 11, mode, gi, hi, want_cand=True)
+        b = oracle_threads(oracle.prefill_units, q, k, 8, 5, 11, mode, gi, hi, threads=3, want_cand=True)
+        for key in a:
+            np.testing.assert_array_equal(a[key], b[key], err_msg=key)
