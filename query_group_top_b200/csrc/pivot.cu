@@ -163,7 +163,7 @@ struct Plan {
   // sizes
   int G, cap, S, K_sel, heads_per_pass, nfb;
   // offsets
-  size_t off_proxy, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, total;
+  size_t off_proxy, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, off_miss, total;
 };
 
 // Sample stride and spill capacity for a select of K_sel keys per row over
@@ -179,6 +179,11 @@ void filter_shape(int K_sel, int L, int* cap, int* S) {
   *cap = (c + 7) / 8 * 8;
   *S = s;
 }
+
+// Refine's miss list: a counter, then one (item, member) entry per member of
+// every unit (the most the select can hand to the fallback).
+size_t miss_cap(size_t units, int g) { return units * static_cast<size_t>((g + 15) / 16) * 16; }
+size_t miss_bytes(size_t units, int g) { return up(sizeof(int)) + up(miss_cap(units, g) * sizeof(int2)); }
 
 Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool dense, int sms) {
   Plan p{};
@@ -205,6 +210,8 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   o += up(static_cast<size_t>(p.nfb) * L * sizeof(uint32_t));
   p.off_cand = o;
   o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(H) * p.G * cand_row_words(Kc) * sizeof(int32_t)) : 0;
+  p.off_miss = o;
+  o += (!dense && mode == PIVOT_REFINE) ? miss_bytes(static_cast<size_t>(H) * p.G, g) : 0;
   p.total = o;
   return p;
 }
@@ -251,16 +258,31 @@ int launch_scan(const CUtensorMap& tmP, const CUtensorMap& tmK, const ScanParams
   return PIVOT_OK;
 }
 
+// Refine, then the exact redo of the members its one-pass select missed.
+// `miss` points at the workspace region sized by miss_bytes(units, g).
 template <int D>
-int launch_refine(RefineParams rp, int units, int sms, cudaStream_t st) {
+int launch_refine(RefineParams rp, int units, int sms, uint8_t* miss, cudaStream_t st) {
   const int smem = RefineCfg<D>::smem_bytes(rp.Kc);
   CUDA_TRY(cudaFuncSetAttribute(refine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   rp.nbatch = (rp.g + 15) / 16;
   rp.n_items = units * rp.nbatch;
+  rp.miss_count = reinterpret_cast<int*>(miss);
+  rp.miss_list = reinterpret_cast<int2*>(miss + up(sizeof(int)));
+  rp.miss_cap = static_cast<int>(std::min<size_t>(miss_cap(units, rp.g), 0x7FFFFFFF));
+  CUDA_TRY(cudaMemsetAsync(rp.miss_count, 0, sizeof(int), st));
   // persistent: one CTA per SM walks the items
   const int grid = std::max(1, std::min(rp.n_items, sms));
-  TraceScope tr("refine", st);
-  refine_kernel<D><<<grid, RefineCfg<D>::NT, smem, st>>>(rp);
+  {
+    TraceScope tr("refine", st);
+    refine_kernel<D><<<grid, RefineCfg<D>::NT, smem, st>>>(rp);
+  }
+  CUDA_TRY(cudaGetLastError());
+  const int fsmem = (2 * cand_row_words(rp.Kc) + 2 * rp.top_k) * 4;
+  CUDA_TRY(cudaFuncSetAttribute(refine_fallback_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, fsmem));
+  {
+    TraceScope tr("refine_fallback", st);
+    refine_fallback_kernel<D><<<2 * std::max(1, sms), kRfbNT, fsmem, st>>>(rp);
+  }
   CUDA_TRY(cudaGetLastError());
   return PIVOT_OK;
 }
@@ -420,17 +442,20 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
                                                                           nullptr, 0);
       CUDA_TRY(cudaGetLastError());
     }
-    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, dev->sms, st) : launch_refine<64>(rp, H * pl.G, dev->sms, st);
+    uint8_t* miss = w + pl.off_miss;
+    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, dev->sms, miss, st)
+                        : launch_refine<64>(rp, H * pl.G, dev->sms, miss, st);
     if (rc) return rc;
   }
   return PIVOT_OK;
 }
 
-size_t decode_ws_size(int B, int H, int d, int Kc, int mode, int max_seqlen) {
+size_t decode_ws_size(int B, int H, int d, int g, int Kc, int mode, int max_seqlen) {
   mode = base_mode(mode);
   size_t o = up(static_cast<size_t>(B) * H * d * 4);                        // fp32 proxies
   o += up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t));       // order keys
   if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
+  if (mode == PIVOT_REFINE) o += miss_bytes(static_cast<size_t>(H) * B, g);
   return o;
 }
 
@@ -454,7 +479,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     return fail(PIVOT_ERR_INVALID_ARG, "out_cand is only produced in PIVOT_REFINE mode");
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
-  const size_t need = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  const size_t need = decode_ws_size(B, H, d, g, Kc, mode, max_seqlen);
   if (!ws || ws_bytes < need) return fail(PIVOT_ERR_WORKSPACE, "workspace too small: need %zu bytes", need);
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return fail(PIVOT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
@@ -528,7 +553,9 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
       cand_export_kernel<<<static_cast<unsigned>(H * B), 256, 0, st>>>(cand, out_cand, B, H, Kc, g, 0, cu, max_seqlen);
       CUDA_TRY(cudaGetLastError());
     }
-    int rc = (d == 128) ? launch_refine<128>(rp, H * B, dev->sms, st) : launch_refine<64>(rp, H * B, dev->sms, st);
+    uint8_t* miss = reinterpret_cast<uint8_t*>(cand) + up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
+    int rc = (d == 128) ? launch_refine<128>(rp, H * B, dev->sms, miss, st)
+                        : launch_refine<64>(rp, H * B, dev->sms, miss, st);
     if (rc) return rc;
   }
   return PIVOT_OK;
@@ -594,7 +621,7 @@ int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t*
     return rc;
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
-  const size_t need = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  const size_t need = decode_ws_size(B, H, d, g, Kc, mode, max_seqlen);
   if (need > kNoAllocScratchBytes)
     return fail(PIVOT_ERR_WORKSPACE,
                 "pivot_decode_index_noalloc: this call needs %zu bytes of scratch, more than the %zu-byte static "
@@ -620,10 +647,9 @@ size_t dense_workspace_size(int L, int H, int d, int top_k) {
 }
 
 size_t pivot_decode_workspace_size(int B, int H, int d, int g, int top_k, int Kc, int mode, int max_seqlen) {
-  (void)g;
   (void)top_k;
   if (B < 1 || H < 1 || max_seqlen < 1) return 0;
-  return decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  return decode_ws_size(B, H, d, g, Kc, mode, max_seqlen);
 }
 
 int pivot_index_ws(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode,
@@ -696,7 +722,7 @@ int pivot_decode_index(const void* q, const void* kcache, const int32_t* cu_seql
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = decode_ws_size(B, H, d, Kc, mode, max_seqlen);
+  const size_t bytes = decode_ws_size(B, H, d, g, Kc, mode, max_seqlen);
   return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
     return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr, nullptr,
                       nullptr, ws, n, st);

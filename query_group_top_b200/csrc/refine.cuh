@@ -22,29 +22,34 @@
 //    write the rows.
 // Chunk c's MMA row r holds candidate t = r*nch + c, so TMEM lane r owns the
 // contiguous, ascending candidates [r*nch, r*nch + nch).  With Kc <= 4096 a
-// unit's scores (4096 x 16 fp32 = 256 KB) fill TMEM; the select warps give
-// each chunk's columns back as soon as they no longer need them, and the MMA
-// warp writes the next unit into them.
+// unit's scores (4096 x 16 fp32 = 256 KB) fill TMEM; the select warps read
+// each chunk's columns once and give them back at once, so the MMA warp can
+// write the next unit into them while this unit is still being selected.
 //
-// Selection (exact, on 32-bit order keys, ties to the lower index):
-//  * round 0 follows the MMAs chunk by chunk: chunk 0 is a 128-candidate
-//    sample spread over the whole set; its score range sets a 512-bin
-//    histogram linear in the score (monotone, clamped at both ends), and
-//    every chunk is counted into it as soon as it is scored;
-//  * select warp w finds the boundary bin of member w with a two-level scan
-//    and inverts the bin function to key thresholds [kl, kh); one pass over
-//    the scores marks each candidate "above" (key >= kh) or "boundary" and
-//    collects the boundary keys in a shared list, after which the unit's TMEM
-//    columns are given back;
-//  * a list of up to kListCap keys is ranked exactly (the need-th largest key
-//    tk, and how many of its copies are taken) and its decisions go to
-//    per-member bitmaps; larger boundaries are narrowed by further key-linear
-//    rounds, and a boundary of equal keys takes its first keys in order;
-//  * one group scan gives every thread its output slot; each warp stages its
+// Selection (exact, on 32-bit order keys, ties to the lower index), in one
+// pass over the scores:
+//  * a member with at most kCap usable candidates sends all of them to its
+//    boundary list;
+//  * otherwise the first kSample chunks (a stride sample of the candidate
+//    set, since chunk c holds every nch-th candidate) give an interval
+//    [lo, hi) that holds the member's k-th score with overwhelming
+//    probability: a histogram linear in the score over chunk 0's range, and
+//    sample ranks kZ standard deviations on either side of the expected one;
+//  * one pass over all chunks marks candidates >= hi in per-thread bit masks
+//    and appends those in [lo, hi) to the member's list, and gives each
+//    chunk's TMEM columns back as soon as it is read;
+//  * the list is ranked exactly (a warp radix select: the need-th largest key
+//    and how many of its copies are taken, ties in candidate order), and its
+//    decisions go to a per-member bitmap;
+//  * one group scan gives every thread its output slots; each warp stages its
 //    slice of an output row in shared memory and writes it coalesced.
+// A member whose k-th score fell outside its interval, whose list overflowed,
+// or whose sample had no score range is not written here: it is recorded in a
+// miss list and refine_fallback_kernel redoes it exactly afterwards.
 #pragma once
 
 #include "ptx.cuh"
+#include "select.cuh"
 
 namespace pivot {
 
@@ -60,55 +65,48 @@ struct RefineParams {
   int n_items;            // H * G units x member batches
   int nbatch;             // member batches of up to 16 per unit
   uint32_t tmem_cols;
+  int2* miss_list;        // (item, member within the item) for refine_fallback_kernel
+  int* miss_count;        // zeroed before the launch
+  int miss_cap;
   int* status;
 };
 
 // member selection modes
 enum : int {
-  kMNone = 0,    // takes nothing (no usable candidate)
-  kMAll = 1,     // takes every usable candidate (top_k >= usable count)
-  kMSel = 2,     // narrowing: the boundary bin of the current round is open
-  kMWhole = 3,   // every key of the boundary bin is taken
-  kMList = 4,    // boundary ranked from the shared list
-  kMNarrow = 5,  // boundary too large for the list: another round
-  kMTies = 6,    // boundary keys all equal: the first need_eq in order
+  kMNone = 0,   // takes nothing (no usable candidate)
+  kMAll = 1,    // takes every usable candidate (top_k >= usable count)
+  kMList = 2,   // few usable candidates: all of them go to the list
+  kMBand = 3,   // sampled interval: >= hi taken, [lo, hi) to the list
+  kMMiss = 4,   // redone by refine_fallback_kernel
 };
 
-constexpr int kRefBins = 512;
+constexpr int kBins = 512;          // sample histogram bins per member
 // 2^23: a float in [2^23, 2^24) is an integer, held in its low mantissa bits
 constexpr float kMagic = 8388608.0f;
-constexpr int kListCap = 256;
-// Each key-linear round shrinks a boundary's key range by a factor of about
-// 256, so 32-bit keys need at most five rounds after round 0.
-constexpr int kMaxRounds = 8;
+constexpr int kCap = 512;           // boundary list entries per member
+constexpr int kSample = 16;         // sampled chunks
+constexpr float kZ = 4.0f;          // interval half-width, in standard deviations of the sample rank
 
 struct MemberSel {
   int nv;           // usable candidates: the ascending prefix with j < pos
   int K;            // min(top_k, nv)
   int mode;
-  int active;       // takes part in the current round
-  int need;         // keys still to take from the current candidate interval
-  int cnt;          // keys in the boundary bin
-  uint32_t lo;      // key-linear bins: origin; both: scale; score-linear: offset
-  float scale, off;
-  int vmode;        // bins linear in the score (1) or in the order key (0)
-  uint32_t kl, kh;  // boundary bin = keys in [kl, kh); kh_inf: no upper edge
-  int kh_inf;
-  uint32_t bmin, bmax;
-  uint32_t tk;      // final rule: keys > tk, then keys == tk in order up to need_eq
+  int nlist;        // list entries appended (may exceed kCap: overflow)
+  int nabove;       // candidates >= hi
+  int nsamp;        // usable sampled scores
+  float lo, hi;     // list interval [lo, hi); hi = +inf: no "above" region
+  uint32_t kmin, kmax;  // chunk 0's usable score range as order keys
+  uint32_t tk, tmask;   // list rule: (key & tmask) > tk, or == tk and among the first need_eq
   int need_eq;
-  int nlist;
 };
 
 struct RefineMisc {
   MemberSel ms[16];
-  uint32_t pmin[4][16], pmax[4][16];
-  int gscan[4][4][8];
+  int gscan[4][4][4];
   uint64_t full[4], empty[4], cready[2], cfree[2], drain;
   uint64_t tready[32], tfree[32];
   uint32_t tmem_slot;
   int abort_flag;
-  int more;
 };
 
 template <int D>
@@ -118,7 +116,7 @@ struct RefineCfg {
   static constexpr int SEL_WARP0 = 4;                   // select warps 4-19
   static constexpr int NSEL = 512;
   static constexpr int NT = 640;
-  static constexpr int NS = 4;                          // gather stages
+  static constexpr int NS = 3;                          // gather stages
   static constexpr int KATOMS = D / 64;
   static constexpr int ATOM_A = 128 * 128;              // 128 rows x 128 bytes
   static constexpr int STAGE = KATOMS * ATOM_A;
@@ -127,74 +125,53 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
   static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
-  // histograms: 16 members x 512 bins of 32-bit counts; the same bytes later
-  // hold the boundary lists, and together with the decision bitmaps that
-  // follow them, the per-warp output staging
-  static constexpr int HIST_BYTES = 16 * kRefBins * 4;
-  static_assert(16 * 2 * kListCap * 4 <= HIST_BYTES, "lists alias the histograms");
-  // output staging entries per select warp: the histogram and bitmap bytes
-  __host__ __device__ static int stg_entries(int Kc) { return (HIST_BYTES / 4 + 16 * 2 * bm_words(Kc)) / 16; }
+  // per member kBins 32-bit words: the sample histogram; later the list's
+  // 256-bin radix histogram (words 0..255) and the decision bitmap (words
+  // 256..383, one bit per candidate)
+  static constexpr int HIST_BYTES = 16 * kBins * 4;
+  static constexpr int LK_BYTES = 16 * kCap * 4;        // list keys
+  static constexpr int LT_BYTES = 16 * kCap * 2;        // list candidate slots
+  // output staging entries per select warp: the list bytes, once ranked
+  static constexpr int STGE = (LK_BYTES + LT_BYTES) / 4 / 16;
   __host__ __device__ static int nch_max(int Kc) { return (Kc + 127) / 128; }
   __host__ __device__ static int cidx_words(int Kc) { return nch_max(Kc) * 128; }
-  // list decisions: per member, "above" and "equal" bitmaps over candidates
-  __host__ __device__ static int bm_words(int Kc) { return nch_max(Kc) * 4; }
+  __host__ __device__ static int off_hist(int Kc) { return OFF_C + 2 * cidx_words(Kc) * 4; }
   static int smem_bytes(int Kc) {
-    return OFF_C + 2 * cidx_words(Kc) * 4 + HIST_BYTES + 16 * 2 * bm_words(Kc) * 4 +
-           static_cast<int>(sizeof(RefineMisc)) + 1024;
+    return off_hist(Kc) + HIST_BYTES + LK_BYTES + LT_BYTES + static_cast<int>(sizeof(RefineMisc)) + 1024;
   }
+  static_assert(kBins >= 256 + 128, "radix histogram and bitmap fit a member's histogram words");
 };
 
-// Linear bin of an order key over [lo, ...) with `scale` bins per key unit,
-// clamped to [0, 511].  Every step is non-decreasing in the key.
-__device__ __forceinline__ int key_bin(uint32_t key, uint32_t lo, float scale) {
-  const uint32_t dl = key > lo ? key - lo : 0u;
-  const uint32_t b = __float2uint_rz(__uint2float_rn(dl) * scale);
-  return static_cast<int>(min(b, static_cast<uint32_t>(kRefBins - 1)));
-}
-
-// Linear bin of a score, round(s * scale + off) clamped to [0, 511], with
+// Linear bin of a score, round(s * scale + off) clamped to [0, kBins-1], with
 // offm = off + 2^23 (as a float): the fma rounds s*scale + offm to an integer
-// in [2^23, 2^23 + 511] after the clamps, and the bin is its low mantissa
+// in [2^23, 2^23 + kBins-1] after the clamps, and the bin is its low mantissa
 // bits.  One rounding of a function increasing in s, then monotone clamps, so
-// the bins are ordered like the scores, and -0 and +0 share a bin.  Scores of
-// real data spread evenly over such bins, while the order keys of scores on
-// both sides of zero crowd into a few of the key-linear ones.
+// the bins are ordered like the scores, and -0 and +0 share a bin.
 __device__ __forceinline__ int value_bin(float s, float scale, float offm) {
-  const float t = fminf(fmaxf(__fmaf_rn(s, scale, offm), kMagic), kMagic + static_cast<float>(kRefBins - 1));
-  return static_cast<int>(__float_as_uint(t) & static_cast<uint32_t>(kRefBins - 1));
+  const float t = fminf(fmaxf(__fmaf_rn(s, scale, offm), kMagic), kMagic + static_cast<float>(kBins - 1));
+  return static_cast<int>(__float_as_uint(t) & static_cast<uint32_t>(kBins - 1));
 }
 
-// Bin of an order key under either bin function; key patterns beyond the
-// infinities (no score has them) clamp to the infinities.
-__device__ __forceinline__ int bin_of_key(uint32_t key, uint32_t lo, float scale, float off, bool vmode) {
-  if (!vmode) return key_bin(key, lo, scale);
+// Bin of an order key; key patterns beyond the infinities (no score has them)
+// clamp to the infinities.
+__device__ __forceinline__ int bin_of_key(uint32_t key, float scale, float offm) {
   const uint32_t kc = min(max(key, 0x007FFFFFu), 0xFF800000u);
-  return value_bin(key_score(kc), scale, off);
+  return value_bin(key_score(kc), scale, offm);
 }
 
-// Smallest key whose bin is >= b (1 <= b <= 511), found by the whole warp;
-// false when no key reaches bin b.  A 32-key probe around the bin's nominal
-// edge usually brackets it; otherwise a 32-way search over all keys does.
-__device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float scale, float off, bool vmode,
-                                                      int lane, uint32_t* out) {
-  if (bin_of_key(0xFFFFFFFFu, lo, scale, off, vmode) < b) return false;
-  uint32_t guess;
-  if (vmode) {
-    // the score where round(s * scale + offm) reaches 2^23 + b
-    guess = score_key(static_cast<float>((static_cast<double>(kMagic) + b - 0.5 - static_cast<double>(off)) /
-                                         static_cast<double>(scale)));
-  } else {
-    const float dk = __fdiv_rn(static_cast<float>(b), scale);
-    guess = dk >= 4294967040.0f ? 0xFFFFFFFFu : lo + min(__float2uint_rz(dk), 0xFFFFFFFFu - lo);
-  }
+// Smallest order key whose bin is >= b (1 <= b <= kBins-1), found by the whole
+// warp (every key reaches the top bin at +inf).  A 32-key probe around the
+// bin's nominal edge usually brackets it; otherwise a 32-way search over all
+// keys does.
+__device__ __forceinline__ uint32_t warp_first_key_of_bin(int b, float scale, float offm, int lane) {
+  // the score where round(s * scale + offm) reaches 2^23 + b
+  const uint32_t guess = score_key(static_cast<float>(
+      (static_cast<double>(kMagic) + b - 0.5 - static_cast<double>(offm)) / static_cast<double>(scale)));
   const long long p0 = static_cast<long long>(guess) - 16;
   const long long pk = min(max(p0 + lane, 0ll), 4294967295ll);
-  const unsigned ge =
-      __ballot_sync(0xffffffffu, bin_of_key(static_cast<uint32_t>(pk), lo, scale, off, vmode) >= b);
-  if ((ge & 1u) == 0u && (ge >> 31) != 0u && p0 >= 0 && p0 + 31 <= 4294967295ll) {
-    *out = static_cast<uint32_t>(p0 + __ffs(ge) - 1);
-    return true;
-  }
+  const unsigned ge = __ballot_sync(0xffffffffu, bin_of_key(static_cast<uint32_t>(pk), scale, offm) >= b);
+  if ((ge & 1u) == 0u && (ge >> 31) != 0u && p0 >= 0 && p0 + 31 <= 4294967295ll)
+    return static_cast<uint32_t>(p0 + __ffs(ge) - 1);
   unsigned long long base = 0, span = 1ull << 32;
   while (span > 1) {
     const unsigned long long stride = (span + 31) / 32;
@@ -202,15 +179,48 @@ __device__ __forceinline__ bool warp_first_key_of_bin(int b, uint32_t lo, float 
     bool g = true;  // empty sub-ranges count as "beyond"
     if (first < base + span) {
       const unsigned long long last = min(first + stride, base + span) - 1;
-      g = bin_of_key(static_cast<uint32_t>(last), lo, scale, off, vmode) >= b;
+      g = bin_of_key(static_cast<uint32_t>(last), scale, offm) >= b;
     }
     const int j = __ffs(__ballot_sync(0xffffffffu, g)) - 1;
     const unsigned long long nb = base + static_cast<unsigned long long>(j) * stride;
     span = min(stride, base + span - nb);
     base = nb;
   }
-  *out = static_cast<uint32_t>(base);
-  return true;
+  return static_cast<uint32_t>(base);
+}
+
+// The bin that holds the r-th largest of the counts in h[0..nbins) (1 <= r <=
+// total), found by the whole warp: the largest b with sum(h[b..]) >= r.  Lane
+// l sums the nbins/32 bins just below nbins - (nbins/32)*l.  *above receives
+// sum(h[b+1..]).
+template <int NBINS>
+__device__ __forceinline__ int warp_rank_bin(const uint32_t* h, int r, int lane, int* above) {
+  constexpr int PER = NBINS / 32;
+  const int b0 = NBINS - PER * (lane + 1);
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) s += static_cast<int>(h[b0 + i]);
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, incl >= r);
+  const int L = hit ? __ffs(hit) - 1 : 31;
+  int cum = __shfl_sync(0xffffffffu, incl - s, L);
+  int bin = NBINS - PER * L - PER;  // (the counts always reach r)
+  const int bL = NBINS - PER * (L + 1);
+  for (int i = PER - 1; i >= 0; --i) {
+    const int c = static_cast<int>(h[bL + i]);
+    if (cum + c >= r) {
+      bin = bL + i;
+      break;
+    }
+    cum += c;
+  }
+  *above = cum;
+  return bin;
 }
 
 // One work item: a unit's batch of up to 16 members.
@@ -273,11 +283,11 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   const uint32_t sB = sbase + C::OFF_B;
   const int NCH = C::nch_max(p.Kc);
   const int CW = C::cidx_words(p.Kc);
-  const int BMW = C::bm_words(p.Kc);
   int32_t* cidx0 = reinterpret_cast<int32_t*>(smem + C::OFF_C);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::OFF_C + 2 * CW * 4);
-  uint32_t* bmap = hist + C::HIST_BYTES / 4;          // [16][2][BMW]
-  RefineMisc* M = reinterpret_cast<RefineMisc*>(bmap + 16 * 2 * BMW);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::off_hist(p.Kc));
+  uint32_t* lkeys = hist + C::HIST_BYTES / 4;                                   // [16][kCap]
+  uint16_t* lslot = reinterpret_cast<uint16_t*>(lkeys + C::LK_BYTES / 4);       // [16][kCap]
+  RefineMisc* M = reinterpret_cast<RefineMisc*>(lslot + C::LT_BYTES / 2);
   volatile int* abort_flag = &M->abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -429,12 +439,13 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
     __syncwarp();
   } else {
     // ======================================================== select
-    const int sw = warp - C::SEL_WARP0;   // 0..15: also the member whose bins this warp scans
+    const int sw = warp - C::SEL_WARP0;   // 0..15: also the member whose list this warp ranks
     const int grp = sw >> 2;              // member group: members 4grp..4grp+3
     const int quarter = warp & 3;         // TMEM lane quarter
     const int r = quarter * 32 + lane;    // this thread's candidate block
     const int stid = sw * 32 + lane;      // 0..511
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 4 * grp;
+    const float kInf = __int_as_float(0x7f800000);
     auto sel_sync = [&]() { named_barrier(2, C::NSEL); };
     int kk = 0;
     bool ok = true;
@@ -463,159 +474,164 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         const int K = min(p.top_k, nv);
         S.nv = nv;
         S.K = K;
-        S.mode = K == 0 ? kMNone : (K == nv ? kMAll : kMSel);
-        S.active = S.mode == kMSel;
-        S.need = K;
-        S.cnt = nv;
+        S.mode = K == 0 ? kMNone : (K == nv ? kMAll : (nv <= kCap ? kMList : kMBand));
         S.nlist = 0;
-        S.bmin = 0xFFFFFFFFu;
-        S.bmax = 0u;
-        S.need_eq = 0;
-        S.tk = 0;
-        S.vmode = 0;
-        S.off = 0.f;
+        S.nabove = 0;
+        S.nsamp = 0;
+        S.lo = -kInf;
+        S.hi = kInf;
+        S.kmin = 0xFFFFFFFFu;
+        S.kmax = 0u;
+        S.tk = 0u;
+        S.tmask = 0u;
+        S.need_eq = 0x7FFFFFFF;
       }
       for (int i = stid; i < C::HIST_BYTES / 16; i += C::NSEL) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
-      for (int i = stid; i < 16 * 2 * BMW / 4; i += C::NSEL) reinterpret_cast<uint4*>(bmap)[i] = make_uint4(0, 0, 0, 0);
       if (named_barrier_or(2, C::NSEL, !ok)) break;
 
       // this thread's view of its four members (member 4*grp + i)
       uint32_t um[4];       // usable chunks of this thread's block (a low-bit prefix)
-      uint32_t hm = 0;      // members counted in the round-0 histogram (uniform in the group)
+      uint32_t bandm = 0;   // this group's members with a sampled interval
+      bool anyb = false;    // the item has such a member (uniform)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const MemberSel& S = M->ms[4 * grp + i];
         const int nvt = min(max(S.nv - r * nch, 0), nch);
         um[i] = nvt >= 32 ? 0xFFFFFFFFu : ((1u << nvt) - 1u);
-        hm |= (S.mode == kMSel ? 1u : 0u) << i;
+        bandm |= (S.mode == kMBand ? 1u : 0u) << i;
       }
-      uint32_t ob4[4];    // score-linear bins: the offset's bits; key-linear: the origin
-      float sc4[4];
-      uint32_t vm4 = 0;   // members whose round-0 bins are linear in the score
+      for (int m = 0; m < 16; ++m) anyb |= M->ms[m].mode == kMBand;
+      const int s_ch = min(nch, kSample);
 
-      auto sample_range = [&]() {
-        uint32_t v[4];
-        tmem_ld_32x32b_x4(tl, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          reg_fence(v[i]);
-          const bool use = ((hm >> i) & um[i] & 1u) != 0u;
-          const uint32_t key = score_key(__uint_as_float(v[i]));
-          const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
-          const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
-          if (lane == 0) {
-            M->pmin[quarter][4 * grp + i] = mn;
-            M->pmax[quarter][4 * grp + i] = mx;
-          }
-        }
-      };
-      auto set_range = [&]() {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = 4 * grp + i;
-          uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            mn = min(mn, M->pmin[qq][m]);
-            mx = max(mx, M->pmax[qq][m]);
-          }
-          const float vmin = key_score(mn), vmax = key_score(mx);
-          const float vsc = static_cast<float>(kRefBins) / __fsub_rn(vmax, vmin);
-          const float voff = __fadd_rn(__fmul_rn(-vmin, vsc), kMagic);   // offset + 2^23
-          const bool vm = mn < mx && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f && isfinite(voff);
-          if (vm) {
-            ob4[i] = __float_as_uint(voff);
-            sc4[i] = vsc;
-            vm4 |= 1u << i;
-          } else if (mn > mx) {
-            ob4[i] = 0u;
-            sc4[i] = 0.f;
-          } else {
-            ob4[i] = mn;
-            sc4[i] = static_cast<float>(kRefBins) / (__uint2float_rn(mx - mn) + 1.0f);
-          }
-          if (quarter == 0 && lane == 0) {
-            M->ms[m].lo = vm ? 0u : ob4[i];
-            M->ms[m].off = vm ? voff : 0.f;
-            M->ms[m].scale = sc4[i];
-            M->ms[m].vmode = vm ? 1 : 0;
-          }
-        }
-      };
-      // shared-memory address of this thread's members' histograms
-      uint32_t hrow[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) hrow[i] = smem_u32(hist + (4 * grp + i) * kRefBins);
-      // chunks where all four members count every score of this thread's block
-      uint32_t allc = 0;
-      auto hist_chunk = [&](int c) {
-        uint32_t v[4];
-        tmem_ld_32x32b_x4(tl + c * 16, v);
-        tmem_ld_wait();
-        if ((allc >> c) & 1u) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            reg_fence(v[i]);
-            const int b = value_bin(__uint_as_float(v[i]), sc4[i], __uint_as_float(ob4[i]));
-            red_shared_add(hrow[i] + 4u * b, 1u);
-          }
-        } else if (vm4 == hm) {  // every counted member has score-linear bins (the rule)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            reg_fence(v[i]);
-            const bool cnt = ((hm >> i) & (um[i] >> c) & 1u) != 0u;
-            const int b = value_bin(__uint_as_float(v[i]), sc4[i], __uint_as_float(ob4[i]));
-            if (cnt) red_shared_add(hrow[i] + 4u * b, 1u);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            reg_fence(v[i]);
-            if (((hm >> i) & (um[i] >> c) & 1u) != 0u) {
-              const float f = __uint_as_float(v[i]);
-              const int b = ((vm4 >> i) & 1u) ? value_bin(f, sc4[i], __uint_as_float(ob4[i]))
-                                              : key_bin(score_key(f), ob4[i], sc4[i]);
-              red_shared_add(hrow[i] + 4u * b, 1u);
-            }
-          }
-        }
-      };
-
-      // ---- round 0, chunk by chunk as the MMAs finish
-      for (int c = 0; c < nch; ++c) {
-        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+      // ---- sample: chunk 0's score range, then a histogram of the first s_ch chunks
+      if (anyb) {
+        if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status, 64);
         ok = __all_sync(0xffffffffu, ok);
-        if (ok && hm != 0) {
+        if (ok && bandm != 0u) {
           tc_fence_after();
-          if (c == 0) {
-            sample_range();
-          } else {
-            if (c == 1) {
-              set_range();
-              allc = (hm == 0xFu && vm4 == 0xFu) ? (um[0] & um[1] & um[2] & um[3]) : 0u;
-              hist_chunk(0);
+          uint32_t v[4];
+          tmem_ld_32x32b_x4(tl, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            reg_fence(v[i]);
+            const bool use = ((bandm >> i) & um[i] & 1u) != 0u;
+            const uint32_t key = score_key(__uint_as_float(v[i]));
+            const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
+            if (lane == 0 && ((bandm >> i) & 1u)) {
+              red_shared_min(smem_u32(&M->ms[4 * grp + i].kmin), mn);
+              red_shared_max(smem_u32(&M->ms[4 * grp + i].kmax), mx);
             }
-            hist_chunk(c);
           }
         }
-        if (c == 0) sel_sync();  // the sample ranges are visible
+        sel_sync();
+        // bins linear in the score over chunk 0's range (every thread for its
+        // members, the same values in all warps of a group)
+        float sc4[4], of4[4];
+        uint32_t vm = 0;   // members with a usable score range
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const MemberSel& S = M->ms[4 * grp + i];
+          const float vmin = key_score(S.kmin), vmax = key_score(S.kmax);
+          sc4[i] = __fdiv_rn(static_cast<float>(kBins), __fsub_rn(vmax, vmin));
+          of4[i] = __fadd_rn(__fmul_rn(-vmin, sc4[i]), kMagic);
+          const bool good = ((bandm >> i) & 1u) && S.kmin < S.kmax && isfinite(vmin) && isfinite(vmax) &&
+                            isfinite(sc4[i]) && sc4[i] > 0.f && isfinite(of4[i]);
+          vm |= (good ? 1u : 0u) << i;
+        }
+        uint32_t hrow[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hrow[i] = smem_u32(hist + (4 * grp + i) * kBins);
+        int ns[4] = {0, 0, 0, 0};
+        for (int c = 0; c < s_ch; ++c) {
+          if (c > 0) {
+            if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+            ok = __all_sync(0xffffffffu, ok);
+          }
+          if (ok && vm != 0u) {
+            tc_fence_after();
+            uint32_t v[4];
+            tmem_ld_32x32b_x4(tl + c * 16, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              reg_fence(v[i]);
+              if (((vm >> i) & (um[i] >> c) & 1u) != 0u) {
+                red_shared_add(hrow[i] + 4u * value_bin(__uint_as_float(v[i]), sc4[i], of4[i]), 1u);
+                ++ns[i];
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if ((vm >> i) & 1u) {
+            const int s = __reduce_add_sync(0xffffffffu, ns[i]);
+            if (lane == 0) atom_shared_add(smem_u32(&M->ms[4 * grp + i].nsamp), static_cast<uint32_t>(s));
+          }
+        }
+        if (named_barrier_or(2, C::NSEL, !ok)) break;
+        // warp sw: member sw's interval from its sample -- sample ranks kZ
+        // standard deviations either side of the expected rank of the k-th
+        // score (hypergeometric: the sample is drawn without replacement)
+        if (sw < nb && M->ms[sw].mode == kMBand) {
+          MemberSel& S = M->ms[sw];
+          const float vmin = key_score(S.kmin), vmax = key_score(S.kmax);
+          const float vsc = __fdiv_rn(static_cast<float>(kBins), __fsub_rn(vmax, vmin));
+          const float voff = __fadd_rn(__fmul_rn(-vmin, vsc), kMagic);
+          const bool good = S.kmin < S.kmax && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f &&
+                            isfinite(voff);
+          if (!good) {
+            if (lane == 0) S.mode = kMMiss;
+          } else {
+            const int n_s = S.nsamp;
+            const float pk = static_cast<float>(S.K) / static_cast<float>(S.nv);
+            const float e = pk * static_cast<float>(n_s);
+            const float fpc = fmaxf(0.f, 1.f - static_cast<float>(n_s) / static_cast<float>(S.nv));
+            const float dlt = kZ * sqrtf(static_cast<float>(n_s) * pk * (1.f - pk) * fpc) + 2.f;
+            const int r_hi = static_cast<int>(floorf(e - dlt));
+            const int r_lo = static_cast<int>(ceilf(e + dlt));
+            const uint32_t* hm = hist + sw * kBins;
+            float hi = kInf, lo = -kInf;
+            int ab;
+            if (r_hi >= 1) {
+              // above = bins over the one holding the r_hi-th largest sample
+              const int b = warp_rank_bin<kBins>(hm, r_hi, lane, &ab);
+              if (b < kBins - 1) hi = key_score(warp_first_key_of_bin(b + 1, vsc, voff, lane));
+            }
+            if (r_lo <= n_s) {
+              // list = down to the bin holding the r_lo-th largest sample
+              const int b = warp_rank_bin<kBins>(hm, r_lo, lane, &ab);
+              if (b > 0) lo = key_score(warp_first_key_of_bin(b, vsc, voff, lane));
+            }
+            if (lane == 0) {
+              S.lo = lo;
+              S.hi = hi;
+            }
+          }
+          __syncwarp();
+        }
+        sel_sync();
       }
-      if (ok && nch == 1 && hm != 0) {
-        set_range();
-        allc = (hm == 0xFu && vm4 == 0xFu) ? (um[0] & um[1] & um[2] & um[3]) : 0u;
-        hist_chunk(0);
-      }
-      if (named_barrier_or(2, C::NSEL, !ok)) break;
 
-      // ---- selection rounds
-      uint32_t gt[4], bnd[4];
+      // ---- one pass: candidates >= hi to the per-thread masks, [lo, hi) to
+      //      the member's list; each batch of chunks is given back at once
+      //      (unless the scores are written out, which reads them again)
+      const bool keep_tmem = p.out_scores != nullptr;
+      float th4[4], tl4[4];
+      uint32_t cm[4];            // chunks to classify, per member
+      uint32_t gt[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        gt[i] = M->ms[4 * grp + i].mode == kMAll ? um[i] : 0u;
-        bnd[i] = 0u;
+        const MemberSel& S = M->ms[4 * grp + i];
+        cm[i] = (S.mode == kMList || S.mode == kMBand) ? um[i] : 0u;
+        th4[i] = S.hi;
+        tl4[i] = S.lo;
       }
-      int released = 0;   // chunks whose TMEM columns this warp has given back
+      const uint32_t anyc = __reduce_or_sync(0xffffffffu, cm[0] | cm[1] | cm[2] | cm[3]);
+      const int waited = anyb ? s_ch : 0;   // chunks whose "scored" barrier the sample already took
+      int released = 0;                     // chunks whose TMEM columns this warp has given back
       auto release_upto = [&](int upto) {
         if (upto <= released) return;
         tc_fence_before();
@@ -625,359 +641,214 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         released = upto;
       };
 #pragma unroll 1
-      for (int round = 0;; ++round) {
-        if (round == kMaxRounds) {
-          if (stid == 0) atomicOr(p.status, kStNoConverge);
-          break;
+      for (int cb = 0; cb < nch; cb += 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = cb + j;
+          if (c < nch && c >= waited && ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
         }
-        // (a) warp sw: boundary bin and key thresholds of member sw
-        if (sw < nb && M->ms[sw].active) {
-          MemberSel& S = M->ms[sw];
-          const uint32_t* hw = hist + sw * kRefBins;
-          const int need = S.need;
-          // lane l owns bins [512 - 16(l+1), 512 - 16l), in descending order by lane
-          const int b0 = kRefBins - 16 * (lane + 1);
-          int s = 0;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (((anyc >> cb) & 15u) != 0u) {
+          tc_fence_after();
+          uint32_t v[4][4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 x = reinterpret_cast<const uint4*>(hw + b0)[(i + lane) & 3];
-            s += static_cast<int>(x.x + x.y + x.z + x.w);
-          }
-          int incl = s;
+          for (int j = 0; j < 4; ++j)
+            if (cb + j < nch) tmem_ld_32x32b_x4(tl + (cb + j) * 16, v[j]);
+          tmem_ld_wait();
+          uint32_t lb[4] = {0u, 0u, 0u, 0u};   // this batch's list entries (bit j: chunk cb + j)
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          // (the counts always reach need; the clamps only keep indices in range)
-          const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
-          const int L = hit ? __ffs(hit) - 1 : 31;
-          const int exclL = __shfl_sync(0xffffffffu, incl - s, L);
-          // lane i < 16: bin 512 - 16L - 1 - i
-          const int cb = lane < 16 ? static_cast<int>(hw[kRefBins - 16 * L - 1 - lane]) : 0;
-          int incl2 = cb;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl2, o);
-            if (lane >= o) incl2 += y;
-          }
-          const unsigned hit2 = __ballot_sync(0xffffffffu, exclL + incl2 >= need);
-          const int i2 = hit2 ? __ffs(hit2) - 1 : 15;
-          const int above = __shfl_sync(0xffffffffu, exclL + incl2 - cb, i2);
-          const int cntb = __shfl_sync(0xffffffffu, cb, i2);
-          const int bstar = kRefBins - 16 * L - 1 - i2;
-          const uint32_t lo = S.lo;
-          const float sc = S.scale, off = S.off;
-          const bool vm = S.vmode != 0;
-          uint32_t kl = 0, kh = 0;
-          bool has_kl = true, has_kh = false;
-          if (bstar > 0) has_kl = warp_first_key_of_bin(bstar, lo, sc, off, vm, lane, &kl);
-          if (bstar < kRefBins - 1) has_kh = warp_first_key_of_bin(bstar + 1, lo, sc, off, vm, lane, &kh);
-          if (lane == 0) {
-            const int need2 = need - above;
-            S.need = need2;
-            S.cnt = cntb;
-            S.kl = has_kl ? kl : 0u;
-            S.kh = kh;
-            S.kh_inf = has_kh ? 0 : 1;
-            S.mode = (cntb == need2) ? kMWhole : (cntb <= kListCap ? kMList : kMNarrow);
-            S.nlist = 0;
-            S.bmin = 0xFFFFFFFFu;
-            S.bmax = 0u;
-          }
-          __syncwarp();
-        }
-        sel_sync();
-
-        // (b) one pass over the scores: above / boundary, boundary lists.  In
-        //     round 0 the columns are given back chunk by chunk unless a
-        //     boundary needs more rounds or the scores are written out.
-        //     key >= K  <=>  score >= key_score(K) (the key order is the score
-        //     order, -0 folded onto +0), so the pass compares scores; no upper
-        //     edge compares against NaN (never true), no lower edge against -inf.
-        bool keep_tmem = p.out_scores != nullptr;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) keep_tmem |= M->ms[m].active && M->ms[m].mode == kMNarrow;
-        uint32_t lst = 0, nar = 0;
-        float th4[4], tl4[4];
-        uint32_t cand4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const MemberSel& S = M->ms[4 * grp + i];
-          const bool a = S.active != 0;
-          lst |= (a && S.mode == kMList ? 1u : 0u) << i;
-          nar |= (a && S.mode == kMNarrow ? 1u : 0u) << i;
-          th4[i] = S.kh_inf ? __int_as_float(0x7fc00000) : key_score(S.kh);
-          tl4[i] = S.kl == 0u ? -__int_as_float(0x7f800000) : key_score(S.kl);
-          cand4[i] = a ? (round == 0 ? um[i] : bnd[i]) : 0u;
-          if (a) bnd[i] = 0u;
-        }
-        const uint32_t anyc = __reduce_or_sync(0xffffffffu, cand4[0] | cand4[1] | cand4[2] | cand4[3]);
-        // common case: every candidate of every lane's block counts for all
-        // four members, so the pass needs no per-key candidate test
-        const uint32_t fullm = nch >= 32 ? 0xFFFFFFFFu : ((1u << nch) - 1u);
-        const bool dense4 = __all_sync(0xffffffffu, (cand4[0] & cand4[1] & cand4[2] & cand4[3]) == fullm);
-#pragma unroll 1
-        for (int cb = 0; cb < nch; cb += 4) {
-          if (((anyc >> cb) & 15u) != 0u) {
-            uint32_t v[4][4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (cb + j < nch) tmem_ld_32x32b_x4(tl + (cb + j) * 16, v[j]);
-            tmem_ld_wait();
-            if (dense4 && cb + 4 <= nch) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t bit = 1u << (cb + j);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  reg_fence(v[j][i]);
-                  const float f = __uint_as_float(v[j][i]);
-                  if (f >= th4[i]) gt[i] |= bit;
-                  else if (f >= tl4[i]) bnd[i] |= bit;
-                }
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int c = cb + j;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  reg_fence(v[j][i]);
-                  const float f = __uint_as_float(v[j][i]);
-                  const uint32_t in = c < nch ? (cand4[i] >> c) & 1u : 0u;
-                  const uint32_t hi = f >= th4[i] ? in : 0u;
-                  const uint32_t lo = f >= tl4[i] ? in : 0u;
-                  gt[i] |= hi << c;
-                  bnd[i] |= (lo & ~hi) << c;
-                }
-              }
-            }
-            // this batch's boundary keys join their member's list, one
-            // shared-memory atomic per warp and member (boundaries are small)
+          for (int j = 0; j < 4; ++j) {
+            const int c = cb + j;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const uint32_t mine = ((lst >> i) & 1u) ? (bnd[i] >> cb) & 15u : 0u;
-              if (mine != 0u) {
-                const int m = 4 * grp + i;
-                int at = static_cast<int>(atom_shared_add(smem_u32(&M->ms[m].nlist), static_cast<uint32_t>(__popc(mine))));
+              reg_fence(v[j][i]);
+              const float f = __uint_as_float(v[j][i]);
+              const uint32_t in = c < nch ? (cm[i] >> c) & 1u : 0u;
+              const uint32_t above = f >= th4[i] ? in : 0u;
+              const uint32_t inlist = f >= tl4[i] ? in : 0u;
+              gt[i] |= above << c;
+              lb[i] |= (inlist & ~above) << j;
+            }
+          }
+          // append to the lists: one shared atomic per warp and member
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  if ((mine >> j) & 1u) {
-                    if (at < kListCap) {
-                      hist[m * 2 * kListCap + at] = score_key(__uint_as_float(v[j][i]));
-                      hist[m * 2 * kListCap + kListCap + at] = static_cast<uint32_t>(r * nch + cb + j);
-                    }
-                    ++at;
+          for (int i = 0; i < 4; ++i) {
+            if (__any_sync(0xffffffffu, lb[i] != 0u)) {
+              const int m = 4 * grp + i;
+              const int cnt = __popc(lb[i]);
+              int incl = cnt;
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+              }
+              int base = 0;
+              if (lane == 31) base = static_cast<int>(atom_shared_add(smem_u32(&M->ms[m].nlist), static_cast<uint32_t>(incl)));
+              base = __shfl_sync(0xffffffffu, base, 31);
+              int at = base + incl - cnt;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if ((lb[i] >> j) & 1u) {
+                  if (at < kCap) {
+                    lkeys[m * kCap + at] = score_key(__uint_as_float(v[j][i]));
+                    lslot[m * kCap + at] = static_cast<uint16_t>(r * nch + cb + j);
                   }
+                  ++at;
                 }
               }
             }
           }
-          if (round == 0 && !keep_tmem) release_upto(min(cb + 4, nch));
         }
-        // key ranges of the boundaries that need another round (rare)
-        if (nar != 0) {
-#pragma unroll 1
-          for (int c = 0; c < nch; ++c) {
-            uint32_t v[4];
-            tmem_ld_32x32b_x4(tl + c * 16, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              reg_fence(v[i]);
-              const bool in = ((nar >> i) & (bnd[i] >> c) & 1u) != 0u;
-              const uint32_t key = score_key(__uint_as_float(v[i]));
-              const uint32_t mn = __reduce_min_sync(0xffffffffu, in ? key : 0xFFFFFFFFu);
-              const uint32_t mx = __reduce_max_sync(0xffffffffu, in ? key : 0u);
-              if (lane == 0 && ((nar >> i) & 1u)) {
-                red_shared_min(smem_u32(&M->ms[4 * grp + i].bmin), mn);
-                red_shared_max(smem_u32(&M->ms[4 * grp + i].bmax), mx);
-              }
-            }
-          }
-        }
-        if (stid == 0) M->more = 0;
-        sel_sync();
-
-        // (c) warp sw closes member sw's round: rank the list, or detect equal
-        //     keys, or set up the next round over the boundary's key range
-        if (sw < nb && M->ms[sw].active) {
-          MemberSel& S = M->ms[sw];
-          const int m = sw;
-          const int mode = S.mode;
-          const int need = S.need;
-          if (mode == kMWhole) {
-            if (lane == 0) {
-              S.need_eq = 0x7FFFFFFF;
-              S.active = 0;
-            }
-          } else if (mode == kMList) {
-            const int n = min(S.nlist, kListCap);
-            const uint32_t* lk = hist + m * 2 * kListCap;
-            // the need-th largest key (with multiplicity) and how many of its
-            // copies are taken
-            for (int e = lane; e < n; e += 32) {
-              const uint32_t ke = lk[e];
-              int ngt = 0, neq = 0;
-              for (int f = 0; f < n; ++f) {
-                const uint32_t kf = lk[f];
-                ngt += kf > ke ? 1 : 0;
-                neq += kf == ke ? 1 : 0;
-              }
-              if (ngt < need && need <= ngt + neq) {
-                S.tk = ke;             // every such lane writes the same values
-                S.need_eq = need - ngt;
-              }
-            }
-            __syncwarp();
-            // the list's decisions, as bitmaps over candidates
-            const uint32_t tk = S.tk;
-            uint32_t* bgt = bmap + (m * 2) * BMW;
-            uint32_t* beq = bgt + BMW;
-            for (int e = lane; e < n; e += 32) {
-              const uint32_t ke = lk[e];
-              const uint32_t te = lk[kListCap + e];
-              if (ke > tk) red_shared_or(smem_u32(&bgt[te >> 5]), 1u << (te & 31));
-              else if (ke == tk) red_shared_or(smem_u32(&beq[te >> 5]), 1u << (te & 31));
-            }
-            if (lane == 0) S.active = 0;
-          } else {  // kMNarrow
-            if (lane == 0) {
-              const uint32_t mn = S.bmin, mx = S.bmax;
-              if (mn == mx) {
-                S.mode = kMTies;
-                S.tk = mn;
-                S.need_eq = need;
-                S.active = 0;
-              } else {
-                S.lo = mn;
-                S.scale = static_cast<float>(kRefBins) / (__uint2float_rn(mx - mn) + 1.0f);
-                S.off = 0.f;
-                S.vmode = 0;
-                S.mode = kMSel;
-                M->more = 1;
-              }
-            }
-          }
-          __syncwarp();
-        }
-        sel_sync();
-        if (!M->more) break;
-
-        // (d) another histogram round over the open boundaries (rare: more
-        //     than kListCap keys in one bin with distinct values)
-        for (int i = stid; i < C::HIST_BYTES / 16; i += C::NSEL)
-          reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
-        sel_sync();
-        {
-          uint32_t c4[4], lo_[4];
-          float sc_[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const MemberSel& S = M->ms[4 * grp + i];
-            c4[i] = S.active ? bnd[i] : 0u;
-            lo_[i] = S.lo;
-            sc_[i] = S.scale;
-          }
-          const uint32_t anyb = __reduce_or_sync(0xffffffffu, c4[0] | c4[1] | c4[2] | c4[3]);
-#pragma unroll 1
-          for (int c = 0; c < nch; ++c) {
-            if (((anyb >> c) & 1u) == 0u) continue;
-            uint32_t v[4];
-            tmem_ld_32x32b_x4(tl + c * 16, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              reg_fence(v[i]);
-              if ((c4[i] >> c) & 1u) {
-                const int b = key_bin(score_key(__uint_as_float(v[i])), lo_[i], sc_[i]);
-                red_shared_add(hrow[i] + 4u * b, 1u);
-              }
-            }
-          }
-        }
-        sel_sync();
+        if (!keep_tmem) release_upto(min(cb + 4, nch));
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = __reduce_add_sync(0xffffffffu, __popc(gt[i]));
+        if (lane == 0 && n > 0) atom_shared_add(smem_u32(&M->ms[4 * grp + i].nabove), static_cast<uint32_t>(n));
+      }
+      if (named_barrier_or(2, C::NSEL, !ok)) break;
 
-      // ---- final rule per member: gt, plus the first need_eq of eq in order
-      uint32_t eq[4];
-      const int t0 = r * nch;
+      // ---- warp sw ranks member sw's list exactly: the need-th largest key
+      //      (radix select from the highest bit that varies) and how many of
+      //      its copies are taken; decisions to the member's bitmap
+      if (sw < nb) {
+        MemberSel& S = M->ms[sw];
+        int mode = S.mode;
+        if (mode == kMList || mode == kMBand) {
+          const int n = S.nlist, need = S.K - S.nabove;
+          if (n > kCap || need < 1 || need > n) {
+            mode = kMMiss;   // the k-th score fell outside the interval, or the list overflowed
+          } else {
+            const uint32_t* lk = lkeys + sw * kCap;
+            const uint16_t* ls = lslot + sw * kCap;
+            uint32_t* rh = hist + sw * kBins;   // radix histogram (256 words)
+            uint32_t* bs = rh + 256;            // decision bitmap (one bit per candidate slot)
+            for (int w = lane; w < 128; w += 32) bs[w] = 0u;
+            uint32_t tk = 0u, tmask = 0u;
+            int need_eq = 0x7FFFFFFF;
+            if (need < n) {
+              const uint32_t k0 = lk[0];
+              uint32_t diff = 0u;
+              for (int e = lane; e < n; e += 32) diff |= lk[e] ^ k0;
+              diff = __reduce_or_sync(0xffffffffu, diff);
+              int sh = 32 - __clz(diff);   // bits [sh, 32) are common to every key
+              tmask = sh >= 32 ? 0u : (0xFFFFFFFFu << sh);
+              tk = k0 & tmask;
+              int rank = need;             // keys matching tk on tmask still to take
+              bool whole = false;
+#pragma unroll 1
+              while (sh > 0) {
+                const int width = min(8, sh);
+                sh -= width;
+                const uint32_t nbm = (1u << width) - 1u;
+                for (int b = lane; b < 256; b += 32) rh[b] = 0u;
+                __syncwarp();
+                for (int e = lane; e < n; e += 32) {
+                  const uint32_t key = lk[e];
+                  if ((key & tmask) == tk) red_shared_add(smem_u32(&rh[(key >> sh) & nbm]), 1u);
+                }
+                __syncwarp();
+                int above;
+                const int b = warp_rank_bin<256>(rh, rank, lane, &above);
+                const int cntb = static_cast<int>(rh[b]);
+                __syncwarp();
+                tk |= static_cast<uint32_t>(b) << sh;
+                tmask |= nbm << sh;
+                rank -= above;
+                if (cntb == rank) {
+                  whole = true;   // every key of the boundary bin is taken
+                  break;
+                }
+              }
+              need_eq = whole ? 0x7FFFFFFF : rank;   // else: equal keys, the first `rank` in slot order
+            }
+            for (int e = lane; e < n; e += 32) {
+              const uint32_t mk = lk[e] & tmask;
+              bool take = mk > tk;
+              if (!take && mk == tk) {
+                take = true;
+                if (need_eq != 0x7FFFFFFF) {
+                  const int t = ls[e];
+                  int before = 0;
+                  for (int f = 0; f < n; ++f) before += ((lk[f] & tmask) == tk && ls[f] < t) ? 1 : 0;
+                  take = before < need_eq;
+                }
+              }
+              if (take) {
+                const int t = ls[e];
+                red_shared_or(smem_u32(&bs[t >> 5]), 1u << (t & 31));
+              }
+            }
+          }
+        }
+        if (mode == kMMiss && lane == 0) {
+          S.mode = kMMiss;
+          const int at = atomicAdd(p.miss_count, 1);
+          if (at < p.miss_cap) p.miss_list[at] = make_int2(item, sw);
+          else atomicOr(p.status, kStNoConverge);
+        }
+        __syncwarp();
+      }
+      sel_sync();
+
+      // ---- rows: each member's taken candidates in ascending order
       auto my_bits = [&](const uint32_t* bm) -> uint32_t {
         if (nch == 0) return 0u;
+        const int t0 = r * nch;
         const int w = t0 >> 5, o = t0 & 31;
         uint32_t x = bm[w] >> o;
-        if (o != 0 && w + 1 < BMW) x |= bm[w + 1] << (32 - o);
+        if (o != 0 && w + 1 < 128) x |= bm[w + 1] << (32 - o);
         return nch >= 32 ? x : (x & ((1u << nch) - 1u));
       };
+      uint32_t selm[4];
+      int mode4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = 4 * grp + i;
-        const int mode = M->ms[m].mode;
-        eq[i] = 0u;
-        if (mode == kMWhole || mode == kMTies) {
-          eq[i] = bnd[i];
-        } else if (mode == kMList) {
-          gt[i] |= my_bits(bmap + (m * 2) * BMW);
-          eq[i] = my_bits(bmap + (m * 2 + 1) * BMW);
-        }
+        mode4[i] = M->ms[m].mode;
+        selm[i] = 0u;
+        if (mode4[i] == kMAll) selm[i] = um[i];
+        else if (mode4[i] == kMList || mode4[i] == kMBand) selm[i] = gt[i] | my_bits(hist + m * kBins + 256);
       }
-      sel_sync();  // every warp has read its bitmaps: their bytes become staging
-      // group scan (thread order = candidate order) of (|gt|, |eq|) for the four members
-      int ex[8];
+      // group scan (thread order = candidate order) of the four members' counts
+      int ex[4];
       {
-        int incl[8], own[8];
+        int incl[4], own[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          own[i] = __popc(gt[i]);
-          own[4 + i] = __popc(eq[i]);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) incl[k] = own[k];
+        for (int i = 0; i < 4; ++i) incl[i] = own[i] = __popc(selm[i]);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int y = __shfl_up_sync(0xffffffffu, incl[k], o);
-            if (lane >= o) incl[k] += y;
+          for (int i = 0; i < 4; ++i) {
+            const int y = __shfl_up_sync(0xffffffffu, incl[i], o);
+            if (lane >= o) incl[i] += y;
           }
         }
         if (lane == 31) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) M->gscan[grp][quarter][k] = incl[k];
+          for (int i = 0; i < 4; ++i) M->gscan[grp][quarter][i] = incl[i];
         }
         named_barrier(3 + grp, 128);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int i = 0; i < 4; ++i) {
           int off = 0;
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) off += (qq < quarter) ? M->gscan[grp][qq][k] : 0;
-          ex[k] = off + incl[k] - own[k];
+          for (int qq = 0; qq < 4; ++qq) off += (qq < quarter) ? M->gscan[grp][qq][i] : 0;
+          ex[i] = off + incl[i] - own[i];
         }
       }
-      // the histogram and bitmap bytes become per-warp output staging (STGE
-      // entries a warp); a warp's slice of a row goes out in STGE-entry parts
-      const int STGE = C::stg_entries(p.Kc);
-      uint32_t* stg = hist + sw * STGE;
+      // the ranked lists' bytes become per-warp output staging (STGE entries
+      // a warp); a warp's slice of a row goes out in STGE-entry parts
+      constexpr int STGE = C::STGE;
+      uint32_t* stg = lkeys + sw * STGE;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = 4 * grp + i;
-        if (m >= nb) continue;
-        const int K = M->ms[m].K, need_eq = M->ms[m].need_eq;
-        const int eqb = ex[4 + i];
-        const int neq = __popc(eq[i]);
-        const int take = min(max(need_eq - eqb, 0), neq);
-        uint32_t sel = gt[i];
-        if (take == neq) {
-          sel |= eq[i];
-        } else {
-          uint32_t e = eq[i];
-          for (int k = 0; k < take; ++k) {
-            sel |= e & (0u - e);  // lowest remaining equal key
-            e &= e - 1;
-          }
-        }
-        const int slot = ex[i] + min(eqb, need_eq);
+        if (m >= nb || mode4[i] == kMMiss) continue;   // a miss is written by refine_fallback_kernel
+        const int K = M->ms[m].K;
+        const uint32_t sel = selm[i];
+        const int slot = ex[i];
         const int wb = __shfl_sync(0xffffffffu, slot, 0);
         // (the selection takes exactly K; the bound only guards the row)
         const int wc = min(__shfl_sync(0xffffffffu, slot + __popc(sel), 31), K) - wb;
@@ -1044,7 +915,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
       ok = __all_sync(0xffffffffu, ok);
       // this item's TMEM columns and candidate list are free
-      release_upto(NCH);
+      if (ok) release_upto(NCH);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&M->cfree[buf]));
       ++kk;
@@ -1057,6 +928,87 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+constexpr int kRfbNT = 512;
+
+// Exact path for the members the one-pass select could not settle: re-score
+// the member's usable candidates on CUDA cores (bf16 query times bf16 keys,
+// fp32 accumulation) and select from all of them.  Dynamic shared memory:
+// 2 * cand_row_words(Kc) + 2 * top_k words.
+template <int D>
+__global__ void __launch_bounds__(kRfbNT) refine_fallback_kernel(RefineParams p) {
+  __shared__ SelectSmem<kRfbNT> sm;
+  __shared__ float qv[D];
+  __shared__ int nv_s;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int KW = cand_row_words(p.Kc);
+  int32_t* cl = reinterpret_cast<int32_t*>(smem_raw);     // candidates, ascending
+  uint32_t* sc = reinterpret_cast<uint32_t*>(cl + KW);     // their scores as order keys
+  int32_t* sel = reinterpret_cast<int32_t*>(sc + KW);
+  uint32_t* selk = reinterpret_cast<uint32_t*>(sel + p.top_k);
+  const int total = min(*p.miss_count, p.miss_cap);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && total > 0) atomicOr(p.status, kStFallback);
+  const long long rowstride = static_cast<long long>(p.H) * D;
+  for (int w = blockIdx.x; w < total; w += gridDim.x) {
+    const int2 e = p.miss_list[w];
+    const RefineItem it = refine_item(p, e.x);
+    const int m = it.mb + e.y;
+    const int pos = it.pos0 + m;
+    const int32_t* row = p.cand + (static_cast<long long>(it.h) * p.G + it.u) * KW;
+    const long long qrow = (it.qrow0 + m) * p.H + it.h;
+    __syncthreads();
+    for (int t = threadIdx.x; t < it.nc; t += kRfbNT) cl[t] = row[cand_word(t, it.nch)];
+    for (int c = threadIdx.x; c < D; c += kRfbNT) qv[c] = __uint_as_float(static_cast<uint32_t>(p.q[qrow * D + c]) << 16);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int lo = 0, hi = it.nc;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (cl[mid] < pos) lo = mid + 1;
+        else hi = mid;
+      }
+      nv_s = lo;
+    }
+    __syncthreads();
+    const int nv = nv_s;
+    const int K = min(p.top_k, nv);
+    const uint16_t* kb = p.keys + (it.key_row0 * p.H + it.h) * static_cast<long long>(D);
+    for (int t = threadIdx.x; t < nv; t += kRfbNT) {
+      const int j = cl[t];
+      float acc = 0.f;
+      if (j >= 0 && j < it.jlim) {
+        const uint4* kr = reinterpret_cast<const uint4*>(kb + j * rowstride);
+#pragma unroll 4
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          const uint4 u = kr[c8];
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            acc = fmaf(qv[c8 * 8 + 2 * k], __uint_as_float(w4[k] << 16), acc);
+            acc = fmaf(qv[c8 * 8 + 2 * k + 1], __uint_as_float(w4[k] & 0xFFFF0000u), acc);
+          }
+        }
+      }
+      sc[t] = score_key(acc);
+    }
+    __syncthreads();
+    block_select_emit<kRfbNT>(
+        nv, K, [&](int x) { return sc[x]; },
+        [&](int slot, int x) {
+          sel[slot] = cl[x];
+          selk[slot] = sc[x];
+        },
+        sm);
+    __syncthreads();
+    int32_t* orow = p.out + qrow * p.top_k;
+    for (int t = threadIdx.x; t < p.top_k; t += kRfbNT) orow[t] = t < K ? sel[t] : -1;
+    if (p.out_scores) {
+      float* srow = p.out_scores + qrow * p.top_k;
+      for (int t = threadIdx.x; t < p.top_k; t += kRfbNT)
+        srow[t] = t < K ? key_score(selk[t]) : __int_as_float(0x7fc00000);
+    }
   }
 }
 

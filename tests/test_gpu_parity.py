@@ -384,3 +384,25 @@ def test_decode_bad_lengths_are_skipped_and_reported(mode, entry):
     res = compare(o[0], r["out"].transpose(1, 0, 2), r["edge"].transpose(1, 0, 2), pos, cedge,
                   sc.cpu().numpy()[0], r["score"].transpose(1, 0, 2))
     assert_parity(res, f"bad-length batch, valid sequence, {mode} {entry}")
+
+
+def test_refine_select_ties_and_misses():
+    """Refine members with more than 512 usable candidates take the sampled
+    interval path.  Constant keys make every score of a member equal, so the
+    sample has no score range: the member goes to the exact refine fallback
+    (flag bit 4) and must still take the lowest indices.  Keys and queries of
+    small integers give many exact ties inside the ranked list, resolved in
+    candidate (index) order."""
+    L, H, d, g, top_k, Kc = 6000, 1, 64, 4, 700, 1500
+    rng = np.random.default_rng(31)
+    q = synthetic.bf16_from_f32(rng.standard_normal((L, H, d)).astype(np.float32))
+    k = synthetic.bf16_from_f32(np.ones((L, H, d), np.float32))
+    res, flags = check_full(q, k, g, top_k, Kc, oracle.REFINE)
+    assert flags & qg.FLAG_FALLBACK
+    assert res["exempt"] == 0
+    qi = synthetic.bf16_from_f32(rng.integers(-1, 2, size=(L, 2, d)).astype(np.float32))
+    ki = synthetic.bf16_from_f32(rng.integers(-1, 2, size=(L, 2, d)).astype(np.float32))
+    res, _ = check_full(qi, ki, g, top_k, Kc, oracle.REFINE)
+    assert res["exempt"] == 0
+    res, _ = check_full(qi, ki, 8, 300, 2000, oracle.REFINE)
+    assert res["exempt"] == 0
