@@ -55,27 +55,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete yet is suspended
+// in hardware (it takes no issue slots) until the phase completes or about
+// `hint_ns` nanoseconds have passed.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspension per poll of the bounded waits: long enough that a waiting warp
+// costs almost no issue slots, short enough that it sees another role's abort
+// promptly.
+constexpr uint32_t kSuspendNs = 20000;
+
 // Waits until the phase with the given parity of `bar` has completed.
 // Returns false (and sets *abort, raising kStTimeout) after kWaitNs, or
-// returns false at once when another role has already set *abort.  With
-// max_sleep_ns > 0 the waiting warp backs off between polls (doubling sleeps
-// up to that bound), leaving issue slots to the warps it is waiting for.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
-                                          unsigned max_sleep_ns = 0) {
+// returns false at once when another role has already set *abort.  Between
+// polls the warp is suspended on the barrier itself (mbar_try_wait_suspend),
+// so waiting warps leave the issue slots to the warps they wait for.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
-  unsigned sleep_ns = 32;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
     if (*abort) return false;
     if (global_timer_ns() - t0 > kWaitNs) {
       *abort = 1;
       atomicOr(status, kStTimeout);
       return false;
-    }
-    if (max_sleep_ns) {
-      __nanosleep(sleep_ns);
-      sleep_ns = min(2 * sleep_ns, max_sleep_ns);
     }
   }
 }

@@ -341,21 +341,21 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       // the list and B buffers of this parity are free once the select warps
       // are done with the item two back
       if (kk >= 2 && ok && warp == 0)
-        ok = mbar_wait(smem_u32(&M->cfree[buf]), ((kk >> 1) - 1) & 1, abort_flag, p.status, 256);
+        ok = mbar_wait(smem_u32(&M->cfree[buf]), ((kk >> 1) - 1) & 1, abort_flag, p.status);
       ok = !named_barrier_or(1, C::NPROD, !ok);
       if (ok && pt == 0) {
         const uint32_t bytes = static_cast<uint32_t>(it.nch) * 128u * 4u;
         mbar_arrive_expect_tx(cbar, bytes);
         if (bytes) bulk_copy_g2s(smem_u32(cx), p.cand + (static_cast<long long>(it.h) * p.G + it.u) * CW, bytes, cbar);
       }
-      if (ok) ok = mbar_wait(cbar, (kk >> 1) & 1, abort_flag, p.status, 128);
+      if (ok) ok = mbar_wait(cbar, (kk >> 1) & 1, abort_flag, p.status);
       const uint16_t* kbase = p.keys + (it.key_row0 * p.H + it.h) * static_cast<long long>(D) + p8 * 8;
       const uint32_t bB = sB + buf * C::B_BYTES;
       for (int c = 0; c < it.nch; ++c) {
         const int s = sseq % C::NS;
         // one warp watches the stage; the others sleep on the named barrier
         if (sseq >= C::NS && ok && warp == 0)
-          ok = mbar_wait(smem_u32(&M->empty[s]), ((sseq / C::NS) - 1) & 1, abort_flag, p.status, 256);
+          ok = mbar_wait(smem_u32(&M->empty[s]), ((sseq / C::NS) - 1) & 1, abort_flag, p.status);
         ok = !named_barrier_or(1, C::NPROD, !ok);
         if (ok) {
           const uint32_t dst0 = sA + s * C::STAGE;
@@ -404,11 +404,11 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       const uint32_t bB = sB + (kk & 1) * C::B_BYTES;
       for (int c = 0; c < NCH && ok; ++c) {
         // the previous item's select warps are done with these columns
-        if (kk >= 1) ok = mbar_wait(smem_u32(&M->tfree[c]), (kk - 1) & 1, abort_flag, p.status, 128);
+        if (kk >= 1) ok = mbar_wait(smem_u32(&M->tfree[c]), (kk - 1) & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (ok && c < it.nch) {
           const int s = sseq % C::NS;
-          ok = mbar_wait(smem_u32(&M->full[s]), (sseq / C::NS) & 1, abort_flag, p.status, 64);
+          ok = mbar_wait(smem_u32(&M->full[s]), (sseq / C::NS) & 1, abort_flag, p.status);
           ok = __all_sync(0xffffffffu, ok);
           if (ok && lane == 0) {
             tc_fence_after();
@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       const int buf = kk & 1;
       const int nch = it.nch, nb = it.nb;
       const int32_t* cx = cidx0 + buf * CW;
-      if (ok) ok = mbar_wait(smem_u32(&M->cready[buf]), (kk >> 1) & 1, abort_flag, p.status, 256);
+      if (ok) ok = mbar_wait(smem_u32(&M->cready[buf]), (kk >> 1) & 1, abort_flag, p.status);
       // ---- per-member usable counts (the candidate set is ascending) and modes
       if (stid < 16 && ok) {
         MemberSel& S = M->ms[stid];
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 
       // ---- sample: chunk 0's score range, then a histogram of the first s_ch chunks
       if (anyb) {
-        if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status, 64);
+        if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (ok && bandm != 0u) {
           tc_fence_after();
@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         int ns[4] = {0, 0, 0, 0};
         for (int c = 0; c < s_ch; ++c) {
           if (c > 0) {
-            if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+            if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
           }
           if (ok && vm != 0u) {
@@ -645,7 +645,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int c = cb + j;
-          if (c < nch && c >= waited && ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+          if (c < nch && c >= waited && ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
         }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -912,7 +912,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       // release then answers a commit of this item, and the MMA warp can never
       // find a chunk's "free" barrier two phases ahead of its wait.
       for (int c = nch; c < NCH; ++c)
-        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, 64);
+        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       // this item's TMEM columns and candidate list are free
       if (ok) release_upto(NCH);

@@ -419,7 +419,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
       if (q != e) return;
       advance(phase);
       // the whole warp decides together: tcgen05.ld below is warp-collective
-      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(e), use & 1, abort_flag, p.status, 256));
+      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(e), use & 1, abort_flag, p.status));
       ++use;
       if (!alive) return;
       tc_fence_after();
