@@ -41,13 +41,12 @@ constexpr int kFinNT = 512;
 constexpr int kFbNT = 512;
 
 // Copies the K selected key indices (staged in shared memory) to their
-// destination: a candidate row in the refine kernel's order (`stage` holds
-// cand_row_words(K) scratch words), or every member's index row, coalesced,
-// with -1 padding to `width`.
+// destination: a candidate row, or every member's index row, coalesced, with
+// -1 padding to `width`.
 __device__ __forceinline__ void write_rows(const FinalizeParams& p, int h, int i, const int32_t* sel,
-                                           const uint32_t* selk, int K, int32_t* stage) {
+                                           const uint32_t* selk, int K) {
   if (!p.broadcast) {
-    write_cand_row(p.cand + (static_cast<long long>(h) * p.G + i) * p.width, sel, K, stage);
+    write_cand_row(p.cand + (static_cast<long long>(h) * p.G + i) * p.width, sel, K);
     return;
   }
   const int s = i * p.g, e = min(s + p.g, p.L);
@@ -104,29 +103,13 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
   __syncthreads();
   if (!p.broadcast) {
     // candidate row: each selected index goes straight to its word of the
-    // row in the refine kernel's read order (no staging, so the kernel needs
-    // only the entries' shared memory); a thread's slots arrive in ascending
-    // order, so their (r, c) position is stepped rather than divided out
+    // row (no staging, so the kernel needs only the entries' shared memory)
     int32_t* dst = p.cand + row_id * p.width;
-    const int nch = (K + 127) / 128;
-    int last = -2, rr = 0, cc = 0;
     block_select_emit<kFinNT>(
         nn, K, [&](int e) { return ent[e].x; },
-        [&](int slot, int e) {
-          if (slot == last + 1) {
-            if (++cc == nch) {
-              cc = 0;
-              ++rr;
-            }
-          } else {
-            rr = slot / nch;
-            cc = slot - rr * nch;
-          }
-          last = slot;
-          dst[cc * 128 + ((rr + cc) & 127)] = static_cast<int32_t>(ent[e].y);
-        },
-        sm);
-    for (int t = K + static_cast<int>(threadIdx.x); t < nch * 128; t += kFinNT) dst[cand_word(t, nch)] = -1;
+        [&](int slot, int e) { dst[slot] = static_cast<int32_t>(ent[e].y); }, sm);
+    const int words = (K + 127) / 128 * 128;
+    for (int t = K + static_cast<int>(threadIdx.x); t < words; t += kFinNT) dst[t] = -1;
     return;
   }
   block_select_emit<kFinNT>(
@@ -137,7 +120,7 @@ __global__ void __launch_bounds__(kFinNT) finalize_kernel(FinalizeParams p) {
       },
       sm);
   __syncthreads();
-  write_rows(p, h, i, sel, selk, K, reinterpret_cast<int32_t*>(ent));  // the entries are no longer needed
+  write_rows(p, h, i, sel, selk, K);
 }
 
 // Exact path for rows the filter could not settle: recompute the row's scores
@@ -149,7 +132,6 @@ __global__ void __launch_bounds__(kFbNT) fallback_kernel(FinalizeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   int32_t* sel = reinterpret_cast<int32_t*>(smem_raw);
   uint32_t* selk = reinterpret_cast<uint32_t*>(sel + p.K_sel);
-  int32_t* stage = reinterpret_cast<int32_t*>(selk + p.K_sel);   // cand_row_words(K_sel) words
   uint32_t* sc = p.fb_scratch + static_cast<long long>(blockIdx.x) * p.L;
   const int total = *p.fb_count;
   if (blockIdx.x == 0 && threadIdx.x == 0 && total > 0) atomicOr(p.status, kStFallback);
@@ -189,7 +171,7 @@ __global__ void __launch_bounds__(kFbNT) fallback_kernel(FinalizeParams p) {
         },
         sm);
     __syncthreads();
-    write_rows(p, h, i, sel, selk, K, stage);
+    write_rows(p, h, i, sel, selk, K);
   }
 }
 

@@ -288,8 +288,8 @@ int launch_refine(RefineParams rp, int units, int sms, uint8_t* miss, cudaStream
 }
 
 // Shared prefill driver (PIVOT Refine/Reuse, and dense when `dense`).
-// Copies candidate rows from the refine kernel's read order ([H][G][CW]) to
-// the plain layout out[unit][h][Kc]: ascending key indices, -1 padding.  Row
+// Copies candidate rows ([H][G][CW]) to the layout out[unit][h][Kc]:
+// ascending key indices, -1 padding.  Row
 // (h, u) holds n = min(Kc, bound) candidates; bound is the Refine scan bound
 // (prefill: the group's last position; decode: n_b + g - 1, or no candidates
 // for a sequence the decode scan skipped).
@@ -304,10 +304,9 @@ __global__ void cand_export_kernel(const int32_t* __restrict__ cand, int32_t* __
     bound = (len > max_seqlen || len < g) ? 0 : len - 1;
   }
   const int n = min(Kc, max(bound, 0));
-  const int nch = (n + 127) / 128;
   const int32_t* row = cand + (static_cast<long long>(h) * G + u) * cand_row_words(Kc);
   int32_t* dst = out + (static_cast<long long>(u) * H + h) * Kc;
-  for (int t = threadIdx.x; t < Kc; t += blockDim.x) dst[t] = t < n ? row[cand_word(t, nch)] : -1;
+  for (int t = threadIdx.x; t < Kc; t += blockDim.x) dst[t] = t < n ? row[t] : -1;
 }
 
 int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int top_k, int Kc, int mode_bits,
@@ -411,7 +410,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
       finalize_kernel<<<static_cast<unsigned>(nh * pl.G), kFinNT, fin_smem, st>>>(fp);
     }
     CUDA_TRY(cudaGetLastError());
-    const int fb_smem = pl.K_sel * 8 + cand_row_words(pl.K_sel) * 4;
+    const int fb_smem = pl.K_sel * 8;
     CUDA_TRY(cudaFuncSetAttribute(fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fb_smem));
     {
       TraceScope tr("fallback", st);
@@ -524,7 +523,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     decode_scan_kernel<64><<<grid, kDecNT, 0, st>>>(dp);
   }
   CUDA_TRY(cudaGetLastError());
-  const int sel_smem = dp.K_sel * 8 + cand_row_words(dp.K_sel) * 4;
+  const int sel_smem = dp.K_sel * 8;
   CUDA_TRY(cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem));
   {
     TraceScope tr("decode_select", st);

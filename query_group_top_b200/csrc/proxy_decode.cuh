@@ -197,9 +197,7 @@ __global__ void __launch_bounds__(kDecSelNT) decode_select_kernel(DecodeParams p
       sm);
   __syncthreads();
   if (p.mode == 0) {
-    // stage: the cand_row_words(K_sel) words after sel and selk
-    write_cand_row(p.cand + (static_cast<long long>(h) * p.B + b) * cand_row_words(p.K_sel), sel, K,
-                   reinterpret_cast<int32_t*>(selk + p.K_sel));
+    write_cand_row(p.cand + (static_cast<long long>(h) * p.B + b) * cand_row_words(p.K_sel), sel, K);
   } else {
     for (int m = 0; m < p.g; ++m) {
       int32_t* dst = p.out + ((static_cast<long long>(b) * p.g + m) * p.H + h) * p.width;

@@ -270,27 +270,17 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 }
 
 // ------------------------------------------------------------------ candidate rows
-// Candidate rows are stored in the order the refine kernel reads them.  A row
-// of n candidates (ascending key indices) has nch = ceil(n / 128) chunks;
-// candidate t = r*nch + c (r < 128, c < nch) sits at word c*128 + ((r+c) & 127)
-// of the row, so that both a chunk (fixed c) and a thread's block (fixed r)
-// are free of shared-memory bank conflicts.  Words of slots t >= n hold -1.
-// A row's stride is cand_row_words(Kc).
+// A candidate row holds a group's candidate key indices in ascending order in
+// words [0, n), then -1 up to the next multiple of 128 (the refine kernel
+// reads a row in whole chunks of 128 candidates).  A row's stride is
+// cand_row_words(Kc).
 __host__ __device__ inline int cand_row_words(int Kc) { return (Kc + 127) / 128 * 128; }
-__host__ __device__ inline int cand_word(int t, int nch) {
-  const int r = t / nch, c = t - r * nch;
-  return c * 128 + ((r + c) & 127);
-}
-// Writes the n selected key indices sel[0..n) as a candidate row at dst,
-// staging the reordering in shared memory `stage` (cand_row_words(n) words);
-// the whole block calls it.
-__device__ inline void write_cand_row(int32_t* __restrict__ dst, const int32_t* sel, int n, int32_t* stage) {
+// Writes the n selected key indices sel[0..n) as a candidate row at dst; the
+// whole block calls it.
+__device__ inline void write_cand_row(int32_t* __restrict__ dst, const int32_t* sel, int n) {
   if (n <= 0) return;
-  const int nch = (n + 127) / 128, words = nch * 128;
-  __syncthreads();
-  for (int t = threadIdx.x; t < words; t += blockDim.x) stage[cand_word(t, nch)] = t < n ? sel[t] : -1;
-  __syncthreads();
-  for (int w = threadIdx.x; w < words; w += blockDim.x) dst[w] = stage[w];
+  const int words = (n + 127) / 128 * 128;
+  for (int t = threadIdx.x; t < words; t += blockDim.x) dst[t] = t < n ? sel[t] : -1;
 }
 
 // ------------------------------------------------------------------ score keys

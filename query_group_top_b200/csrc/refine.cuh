@@ -17,32 +17,38 @@
 //  * the MMA warp (warp 3) issues tcgen05.mma with M = 128 candidate rows,
 //    N = 16 member queries, K = d, into TMEM columns [16c, 16c+16) for chunk
 //    c, and signals "chunk c scored" on a per-chunk mbarrier;
-//  * the select warps (4-19, four per TMEM lane quarter; group grp of four
-//    warps owns members 4grp..4grp+3) select every member's exact top-k and
-//    write the rows.
-// Chunk c's MMA row r holds candidate t = r*nch + c, so TMEM lane r owns the
-// contiguous, ascending candidates [r*nch, r*nch + nch).  With Kc <= 4096 a
-// unit's scores (4096 x 16 fp32 = 256 KB) fill TMEM; the select warps read
-// each chunk's columns once and give them back at once, so the MMA warp can
-// write the next unit into them while this unit is still being selected.
+//  * the select warps (4-19) select every member's exact top-k and write the
+//    rows.
+// Chunk c holds candidates c*128 .. c*128+127 (MMA row r = candidate
+// c*128 + r), so TMEM lane quarter q of chunk c holds 32 consecutive
+// candidates.  Chunks are scored in the order 0, 2, 4, ..., then 1, 3, 5, ...,
+// so that the first ones spread over the whole candidate set.  With
+// Kc <= 4096 a unit's scores (4096 x 16 fp32 = 256 KB) fill TMEM; the select
+// warps read each chunk's columns once and give them back at once, so the
+// MMA warp can write the next unit into them while this unit is still being
+// selected.
 //
 // Selection (exact, on 32-bit order keys, ties to the lower index), in one
-// pass over the scores:
+// pass over the scores.  Select warp w = 4s + q reads TMEM lane quarter q of
+// the chunks at scoring positions s, s+4, s+8, ... (all 16 members of 32
+// candidates per load) and later ranks member w's list and writes member w's
+// rows:
 //  * a member with at most kCap usable candidates sends all of them to its
 //    boundary list;
-//  * otherwise the first kSample chunks (a stride sample of the candidate
-//    set, since chunk c holds every nch-th candidate) give an interval
-//    [lo, hi) that holds the member's k-th score with overwhelming
-//    probability: a histogram linear in the score over chunk 0's range, and
-//    sample ranks kZ standard deviations on either side of the expected one;
-//  * one pass over all chunks marks candidates >= hi in per-thread bit masks
-//    and appends those in [lo, hi) to the member's list, and gives each
-//    chunk's TMEM columns back as soon as it is read;
+//  * otherwise the first kSample chunks give an interval [lo, hi) that holds
+//    the member's k-th score with overwhelming probability: a histogram
+//    linear in the score over chunk 0's range, and sample ranks kZ standard
+//    deviations on either side of the expected one;
+//  * one pass over all chunks classifies 32 candidates of a member with two
+//    warp votes: the ">= hi" mask goes straight into the member's selection
+//    bitmap (bit t = candidate t), the "[lo, hi)" lanes append their scores
+//    to the member's list; each chunk's TMEM columns are given back as soon
+//    as they are loaded;
 //  * the list is ranked exactly (a warp radix select: the need-th largest key
 //    and how many of its copies are taken, ties in candidate order), and its
-//    decisions go to a per-member bitmap;
-//  * one group scan gives every thread its output slots; each warp stages its
-//    slice of an output row in shared memory and writes it coalesced.
+//    decisions are OR-ed into the bitmap;
+//  * the member's warp walks the bitmap in candidate order: each 32-bit word
+//    gives one coalesced store of its selected key indices.
 // A member whose k-th score fell outside its interval, whose list overflowed,
 // or whose sample had no score range is not written here: it is recorded in a
 // miss list and refine_fallback_kernel redoes it exactly afterwards.
@@ -80,7 +86,7 @@ enum : int {
   kMMiss = 4,   // redone by refine_fallback_kernel
 };
 
-constexpr int kBins = 512;          // sample histogram bins per member
+constexpr int kBins = 256;          // sample histogram bins per member
 // 2^23: a float in [2^23, 2^24) is an integer, held in its low mantissa bits
 constexpr float kMagic = 8388608.0f;
 constexpr int kCap = 512;           // boundary list entries per member
@@ -92,17 +98,13 @@ struct MemberSel {
   int K;            // min(top_k, nv)
   int mode;
   int nlist;        // list entries appended (may exceed kCap: overflow)
-  int nabove;       // candidates >= hi
-  int nsamp;        // usable sampled scores
   float lo, hi;     // list interval [lo, hi); hi = +inf: no "above" region
+  float scale, offm;    // sample histogram bins: value_bin(s, scale, offm)
   uint32_t kmin, kmax;  // chunk 0's usable score range as order keys
-  uint32_t tk, tmask;   // list rule: (key & tmask) > tk, or == tk and among the first need_eq
-  int need_eq;
 };
 
 struct RefineMisc {
   MemberSel ms[16];
-  int gscan[4][4][4];
   uint64_t full[4], empty[4], cready[2], cfree[2], drain;
   uint64_t tready[32], tfree[32];
   uint32_t tmem_slot;
@@ -125,21 +127,21 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
   static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
-  // per member kBins 32-bit words: the sample histogram; later the list's
-  // 256-bin radix histogram (words 0..255) and the decision bitmap (words
-  // 256..383, one bit per candidate)
+  // per member kBins 32-bit words: the sample histogram, later the list's
+  // 256-bin radix histogram, and with the scores written out the selection's
+  // per-word prefix counts
   static constexpr int HIST_BYTES = 16 * kBins * 4;
-  static constexpr int LK_BYTES = 16 * kCap * 4;        // list keys
+  static constexpr int BMP_BYTES = 16 * 128 * 4;        // selection bitmaps: one bit per candidate slot
+  static constexpr int LK_BYTES = 16 * kCap * 4;        // list scores (fp32 bits, then order keys)
   static constexpr int LT_BYTES = 16 * kCap * 2;        // list candidate slots
-  // output staging entries per select warp: the list bytes, once ranked
-  static constexpr int STGE = (LK_BYTES + LT_BYTES) / 4 / 16;
   __host__ __device__ static int nch_max(int Kc) { return (Kc + 127) / 128; }
   __host__ __device__ static int cidx_words(int Kc) { return nch_max(Kc) * 128; }
   __host__ __device__ static int off_hist(int Kc) { return OFF_C + 2 * cidx_words(Kc) * 4; }
   static int smem_bytes(int Kc) {
-    return off_hist(Kc) + HIST_BYTES + LK_BYTES + LT_BYTES + static_cast<int>(sizeof(RefineMisc)) + 1024;
+    return off_hist(Kc) + HIST_BYTES + BMP_BYTES + LK_BYTES + LT_BYTES + static_cast<int>(sizeof(RefineMisc)) +
+           1024;
   }
-  static_assert(kBins >= 256 + 128, "radix histogram and bitmap fit a member's histogram words");
+  static_assert(kBins == 256, "the radix histogram reuses a member's histogram words");
 };
 
 // Linear bin of a score, round(s * scale + off) clamped to [0, kBins-1], with
@@ -269,9 +271,18 @@ __device__ __forceinline__ RefineItem refine_item(const RefineParams& p, int ite
   return it;
 }
 
-// candidate t = r*nch + c of a list lives at word c*128 + ((r + c) & 127):
-// conflict-free both along a chunk (fixed c) and along a thread's block (fixed r)
-__device__ __forceinline__ int cidx_pos(int c, int r) { return c * 128 + ((r + c) & 127); }
+// The chunk scored at position i of a unit with nch chunks: even chunks
+// first, then odd ones; positions past nch (chunks the unit does not use)
+// map to themselves.
+__device__ __forceinline__ int chunk_at(int i, int nch) {
+  const int ne = (nch + 1) >> 1;
+  return i < nch ? (i < ne ? 2 * i : 2 * (i - ne) + 1) : i;
+}
+// The scoring position of chunk c (the inverse of chunk_at).
+__device__ __forceinline__ int chunk_pos(int c, int nch) {
+  const int ne = (nch + 1) >> 1;
+  return c < nch ? ((c & 1) ? ne + (c >> 1) : (c >> 1)) : c;
+}
 
 template <int D>
 __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
@@ -284,8 +295,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   const int NCH = C::nch_max(p.Kc);
   const int CW = C::cidx_words(p.Kc);
   int32_t* cidx0 = reinterpret_cast<int32_t*>(smem + C::OFF_C);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::off_hist(p.Kc));
-  uint32_t* lkeys = hist + C::HIST_BYTES / 4;                                   // [16][kCap]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::off_hist(p.Kc));      // [16][kBins]
+  uint32_t* bmp = hist + C::HIST_BYTES / 4;                                     // [16][128]
+  uint32_t* lkeys = bmp + C::BMP_BYTES / 4;                                     // [16][kCap]
   uint16_t* lslot = reinterpret_cast<uint16_t*>(lkeys + C::LK_BYTES / 4);       // [16][kCap]
   RefineMisc* M = reinterpret_cast<RefineMisc*>(lslot + C::LT_BYTES / 2);
   volatile int* abort_flag = &M->abort_flag;
@@ -302,7 +314,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
     }
     for (int c = 0; c < 32; ++c) {
       mbar_init(smem_u32(&M->tready[c]), 1);
-      mbar_init(smem_u32(&M->tfree[c]), C::NSEL / 32);
+      mbar_init(smem_u32(&M->tfree[c]), 4);   // the four lane-quarter warps that read chunk c
     }
     mbar_init(smem_u32(&M->drain), 1);
     *abort_flag = 0;
@@ -319,8 +331,8 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 
   if (warp < C::MMA_WARP) {
     // ======================================================== producers
-    // Thread 0 fetches each unit's candidate row (stored in this kernel's
-    // read order) with one bulk copy; then all 96 producer threads gather the
+    // Thread 0 fetches each unit's candidate row with one bulk copy; then all
+    // 96 producer threads gather the
     // candidate key rows of each chunk with 16-byte cp.async into the
     // 128-byte-swizzled K-major layout, and each thread's arrival on the
     // stage's "full" barrier fires once its own copies have landed, so no
@@ -351,7 +363,8 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       if (ok) ok = mbar_wait(cbar, (kk >> 1) & 1, abort_flag, p.status);
       const uint16_t* kbase = p.keys + (it.key_row0 * p.H + it.h) * static_cast<long long>(D) + p8 * 8;
       const uint32_t bB = sB + buf * C::B_BYTES;
-      for (int c = 0; c < it.nch; ++c) {
+      for (int ci = 0; ci < it.nch; ++ci) {
+        const int c = chunk_at(ci, it.nch);
         const int s = sseq % C::NS;
         // one warp watches the stage; the others sleep on the named barrier
         if (sseq >= C::NS && ok && warp == 0)
@@ -361,7 +374,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           const uint32_t dst0 = sA + s * C::STAGE;
           const int32_t* cxc = cx + c * 128;
           for (int rr = rr0; rr < 128; rr += RSTEP) {
-            const int j = cxc[(rr + c) & 127];
+            const int j = cxc[rr];
             // a missing candidate (-1 padding) reads as zeros; so would an
             // index outside the scan's bound, which no candidate row holds
             const bool in = j >= 0 && j < it.jlim;
@@ -371,7 +384,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 #pragma unroll
             for (int a = 0; a < C::KATOMS; ++a) cp_async_16(dst + a * C::ATOM_A, src + a * 64, nbytes);
           }
-          if (c == 0) {
+          if (ci == 0) {
             // member queries of this batch -> B operand, zero rows past nb
             for (int id = pt; id < 16 * (D / 8); id += C::NPROD) {
               const int rr = id / (D / 8), piece = id % (D / 8);
@@ -402,7 +415,8 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       const RefineItem it = refine_item(p, item);
       if (it.nb <= 0) continue;
       const uint32_t bB = sB + (kk & 1) * C::B_BYTES;
-      for (int c = 0; c < NCH && ok; ++c) {
+      for (int ci = 0; ci < NCH && ok; ++ci) {
+        const int c = chunk_at(ci, it.nch);
         // the previous item's select warps are done with these columns
         if (kk >= 1) ok = mbar_wait(smem_u32(&M->tfree[c]), (kk - 1) & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
@@ -439,14 +453,20 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
     __syncwarp();
   } else {
     // ======================================================== select
-    const int sw = warp - C::SEL_WARP0;   // 0..15: also the member whose list this warp ranks
-    const int grp = sw >> 2;              // member group: members 4grp..4grp+3
-    const int quarter = warp & 3;         // TMEM lane quarter
-    const int r = quarter * 32 + lane;    // this thread's candidate block
+    const int sw = warp - C::SEL_WARP0;   // 0..15: the member whose list and rows this warp handles
+    const int q = warp & 3;               // TMEM lane quarter: candidates 32q .. 32q+31 of a chunk
+    const int st = sw >> 2;               // chunk stream: the chunks at scoring positions st, st+4, ...
     const int stid = sw * 32 + lane;      // 0..511
-    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 4 * grp;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t ltmask = (1u << lane) - 1u;
     const float kInf = __int_as_float(0x7f800000);
     auto sel_sync = [&]() { named_barrier(2, C::NSEL); };
+    // gives chunk c's columns back (this warp has its scores in registers)
+    auto release = [&](int c) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&M->tfree[c]));
+    };
     int kk = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
@@ -465,8 +485,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           int lo = 0, hi = it.nc;
           while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            const int rr = mid / nch;
-            if (cx[cidx_pos(mid - rr * nch, rr)] < pos) lo = mid + 1;
+            if (cx[mid] < pos) lo = mid + 1;
             else hi = mid;
           }
           nv = lo;
@@ -476,257 +495,210 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         S.K = K;
         S.mode = K == 0 ? kMNone : (K == nv ? kMAll : (nv <= kCap ? kMList : kMBand));
         S.nlist = 0;
-        S.nabove = 0;
-        S.nsamp = 0;
-        S.lo = -kInf;
+        S.lo = S.mode == kMList ? -kInf : kInf;   // None/All take no list; Band is set below
         S.hi = kInf;
         S.kmin = 0xFFFFFFFFu;
         S.kmax = 0u;
-        S.tk = 0u;
-        S.tmask = 0u;
-        S.need_eq = 0x7FFFFFFF;
       }
-      for (int i = stid; i < C::HIST_BYTES / 16; i += C::NSEL) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+      for (int i = stid; i < (C::HIST_BYTES + C::BMP_BYTES) / 16; i += C::NSEL)
+        reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
       if (named_barrier_or(2, C::NSEL, !ok)) break;
-
-      // this thread's view of its four members (member 4*grp + i)
-      uint32_t um[4];       // usable chunks of this thread's block (a low-bit prefix)
-      uint32_t bandm = 0;   // this group's members with a sampled interval
-      bool anyb = false;    // the item has such a member (uniform)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const MemberSel& S = M->ms[4 * grp + i];
-        const int nvt = min(max(S.nv - r * nch, 0), nch);
-        um[i] = nvt >= 32 ? 0xFFFFFFFFu : ((1u << nvt) - 1u);
-        bandm |= (S.mode == kMBand ? 1u : 0u) << i;
+      bool anyb = false;     // a member with a sampled interval (uniform)
+      int nvmin = 0x7FFFFFFF;  // fewest usable candidates of a classified member (uniform)
+      for (int m = 0; m < 16; ++m) {
+        const int md = M->ms[m].mode;
+        anyb |= md == kMBand;
+        if (md == kMList || md == kMBand) nvmin = min(nvmin, M->ms[m].nv);
       }
-      for (int m = 0; m < 16; ++m) anyb |= M->ms[m].mode == kMBand;
       const int s_ch = min(nch, kSample);
 
-      // ---- sample: chunk 0's score range, then a histogram of the first s_ch chunks
+      // ---- sample: chunk 0's score range, then a histogram of the first s_ch
+      //      chunks scored; then warp w derives member w's interval
       if (anyb) {
-        if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok && bandm != 0u) {
-          tc_fence_after();
-          uint32_t v[4];
-          tmem_ld_32x32b_x4(tl, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            reg_fence(v[i]);
-            const bool use = ((bandm >> i) & um[i] & 1u) != 0u;
-            const uint32_t key = score_key(__uint_as_float(v[i]));
-            const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
-            const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
-            if (lane == 0 && ((bandm >> i) & 1u)) {
-              red_shared_min(smem_u32(&M->ms[4 * grp + i].kmin), mn);
-              red_shared_max(smem_u32(&M->ms[4 * grp + i].kmax), mx);
-            }
-          }
-        }
-        sel_sync();
-        // bins linear in the score over chunk 0's range (every thread for its
-        // members, the same values in all warps of a group)
-        float sc4[4], of4[4];
-        uint32_t vm = 0;   // members with a usable score range
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const MemberSel& S = M->ms[4 * grp + i];
-          const float vmin = key_score(S.kmin), vmax = key_score(S.kmax);
-          sc4[i] = __fdiv_rn(static_cast<float>(kBins), __fsub_rn(vmax, vmin));
-          of4[i] = __fadd_rn(__fmul_rn(-vmin, sc4[i]), kMagic);
-          const bool good = ((bandm >> i) & 1u) && S.kmin < S.kmax && isfinite(vmin) && isfinite(vmax) &&
-                            isfinite(sc4[i]) && sc4[i] > 0.f && isfinite(of4[i]);
-          vm |= (good ? 1u : 0u) << i;
-        }
-        uint32_t hrow[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hrow[i] = smem_u32(hist + (4 * grp + i) * kBins);
-        int ns[4] = {0, 0, 0, 0};
-        for (int c = 0; c < s_ch; ++c) {
-          if (c > 0) {
-            if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
-            ok = __all_sync(0xffffffffu, ok);
-          }
-          if (ok && vm != 0u) {
+        if (st == 0) {
+          if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok) {
             tc_fence_after();
-            uint32_t v[4];
-            tmem_ld_32x32b_x4(tl + c * 16, v);
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tq, v);
             tmem_ld_wait();
+            const int t = q * 32 + lane;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              reg_fence(v[i]);
-              if (((vm >> i) & (um[i] >> c) & 1u) != 0u) {
-                red_shared_add(hrow[i] + 4u * value_bin(__uint_as_float(v[i]), sc4[i], of4[i]), 1u);
-                ++ns[i];
+            for (int j = 0; j < 16; ++j) {
+              reg_fence(v[j]);
+              if (M->ms[j].mode == kMBand) {
+                const bool use = t < M->ms[j].nv;
+                const uint32_t key = score_key(__uint_as_float(v[j]));
+                const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
+                const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
+                if (lane == 0) {
+                  red_shared_min(smem_u32(&M->ms[j].kmin), mn);
+                  red_shared_max(smem_u32(&M->ms[j].kmax), mx);
+                }
               }
             }
           }
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if ((vm >> i) & 1u) {
-            const int s = __reduce_add_sync(0xffffffffu, ns[i]);
-            if (lane == 0) atom_shared_add(smem_u32(&M->ms[4 * grp + i].nsamp), static_cast<uint32_t>(s));
-          }
-        }
         if (named_barrier_or(2, C::NSEL, !ok)) break;
-        // warp sw: member sw's interval from its sample -- sample ranks kZ
-        // standard deviations either side of the expected rank of the k-th
-        // score (hypergeometric: the sample is drawn without replacement)
-        if (sw < nb && M->ms[sw].mode == kMBand) {
+        // bins linear in the score over chunk 0's range; a member whose range
+        // is empty or not finite goes to the exact fallback
+        if (lane == 0 && M->ms[sw].mode == kMBand) {
           MemberSel& S = M->ms[sw];
           const float vmin = key_score(S.kmin), vmax = key_score(S.kmax);
           const float vsc = __fdiv_rn(static_cast<float>(kBins), __fsub_rn(vmax, vmin));
           const float voff = __fadd_rn(__fmul_rn(-vmin, vsc), kMagic);
-          const bool good = S.kmin < S.kmax && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f &&
-                            isfinite(voff);
-          if (!good) {
-            if (lane == 0) S.mode = kMMiss;
-          } else {
-            const int n_s = S.nsamp;
-            const float pk = static_cast<float>(S.K) / static_cast<float>(S.nv);
-            const float e = pk * static_cast<float>(n_s);
-            const float fpc = fmaxf(0.f, 1.f - static_cast<float>(n_s) / static_cast<float>(S.nv));
-            const float dlt = kZ * sqrtf(static_cast<float>(n_s) * pk * (1.f - pk) * fpc) + 2.f;
-            const int r_hi = static_cast<int>(floorf(e - dlt));
-            const int r_lo = static_cast<int>(ceilf(e + dlt));
-            const uint32_t* hm = hist + sw * kBins;
-            float hi = kInf, lo = -kInf;
-            int ab;
-            if (r_hi >= 1) {
-              // above = bins over the one holding the r_hi-th largest sample
-              const int b = warp_rank_bin<kBins>(hm, r_hi, lane, &ab);
-              if (b < kBins - 1) hi = key_score(warp_first_key_of_bin(b + 1, vsc, voff, lane));
-            }
-            if (r_lo <= n_s) {
-              // list = down to the bin holding the r_lo-th largest sample
-              const int b = warp_rank_bin<kBins>(hm, r_lo, lane, &ab);
-              if (b > 0) lo = key_score(warp_first_key_of_bin(b, vsc, voff, lane));
-            }
-            if (lane == 0) {
-              S.lo = lo;
-              S.hi = hi;
-            }
+          const bool good =
+              S.kmin < S.kmax && isfinite(vmin) && isfinite(vmax) && isfinite(vsc) && vsc > 0.f && isfinite(voff);
+          S.scale = vsc;
+          S.offm = voff;
+          if (!good) S.mode = kMMiss;
+        }
+        sel_sync();
+        for (int i = st; i < s_ch; i += 4) {
+          const int c = chunk_at(i, nch);
+          if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tq + 16 * c, v);
+          tmem_ld_wait();
+          const int t = c * 128 + q * 32 + lane;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            reg_fence(v[j]);
+            const MemberSel& S = M->ms[j];
+            if (S.mode == kMBand && t < S.nv)
+              red_shared_add(smem_u32(hist + j * kBins + value_bin(__uint_as_float(v[j]), S.scale, S.offm)), 1u);
+          }
+        }
+        if (named_barrier_or(2, C::NSEL, !ok)) break;
+        // member sw's interval: sample ranks kZ standard deviations either side
+        // of the expected rank of the k-th score (hypergeometric: the sample
+        // is drawn without replacement)
+        if (sw < nb && M->ms[sw].mode == kMBand) {
+          MemberSel& S = M->ms[sw];
+          const uint32_t* hm = hist + sw * kBins;
+          int n_s = 0;
+#pragma unroll
+          for (int b = 0; b < kBins / 32; ++b) n_s += static_cast<int>(hm[lane * (kBins / 32) + b]);
+          n_s = __reduce_add_sync(0xffffffffu, n_s);
+          const float pk = static_cast<float>(S.K) / static_cast<float>(S.nv);
+          const float e = pk * static_cast<float>(n_s);
+          const float fpc = fmaxf(0.f, 1.f - static_cast<float>(n_s) / static_cast<float>(S.nv));
+          const float dlt = kZ * sqrtf(static_cast<float>(n_s) * pk * (1.f - pk) * fpc) + 2.f;
+          const int r_hi = static_cast<int>(floorf(e - dlt));
+          const int r_lo = static_cast<int>(ceilf(e + dlt));
+          float hi = kInf, lo = -kInf;
+          int ab;
+          if (r_hi >= 1) {
+            // above = the bins over the one holding the r_hi-th largest sample
+            const int b = warp_rank_bin<kBins>(hm, r_hi, lane, &ab);
+            if (b < kBins - 1) hi = key_score(warp_first_key_of_bin(b + 1, S.scale, S.offm, lane));
+          }
+          if (r_lo <= n_s) {
+            // list = down to the bin holding the r_lo-th largest sample
+            const int b = warp_rank_bin<kBins>(hm, r_lo, lane, &ab);
+            if (b > 0) lo = key_score(warp_first_key_of_bin(b, S.scale, S.offm, lane));
+          }
+          if (lane == 0) {
+            S.lo = lo;
+            S.hi = hi;
           }
           __syncwarp();
         }
         sel_sync();
       }
 
-      // ---- one pass: candidates >= hi to the per-thread masks, [lo, hi) to
-      //      the member's list; each batch of chunks is given back at once
-      //      (unless the scores are written out, which reads them again)
+      // ---- one pass: per chunk, each member's ">= hi" lanes into its bitmap
+      //      and its "[lo, hi)" lanes onto its list; the chunk's TMEM columns
+      //      go back as soon as they are loaded (unless the scores are
+      //      written out, which reads them again)
       const bool keep_tmem = p.out_scores != nullptr;
-      float th4[4], tl4[4];
-      uint32_t cm[4];            // chunks to classify, per member
-      uint32_t gt[4] = {0u, 0u, 0u, 0u};
+      float th[16], tl[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const MemberSel& S = M->ms[4 * grp + i];
-        cm[i] = (S.mode == kMList || S.mode == kMBand) ? um[i] : 0u;
-        th4[i] = S.hi;
-        tl4[i] = S.lo;
+      for (int j = 0; j < 16; ++j) {
+        const MemberSel& S = M->ms[j];
+        const bool cls = S.mode == kMList || S.mode == kMBand;
+        th[j] = cls ? S.hi : kInf;
+        tl[j] = cls ? S.lo : kInf;
       }
-      const uint32_t anyc = __reduce_or_sync(0xffffffffu, cm[0] | cm[1] | cm[2] | cm[3]);
-      const int waited = anyb ? s_ch : 0;   // chunks whose "scored" barrier the sample already took
-      int released = 0;                     // chunks whose TMEM columns this warp has given back
-      auto release_upto = [&](int upto) {
-        if (upto <= released) return;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-          for (int c = released; c < upto; ++c) mbar_arrive(smem_u32(&M->tfree[c]));
-        released = upto;
-      };
 #pragma unroll 1
-      for (int cb = 0; cb < nch; cb += 4) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = cb + j;
-          if (c < nch && c >= waited && ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
-        }
+      for (int i = st; i < nch; i += 4) {
+        const int c = chunk_at(i, nch);
+        if (ok && (i >= s_ch || !anyb)) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        if (((anyc >> cb) & 15u) != 0u) {
-          tc_fence_after();
-          uint32_t v[4][4];
+        tc_fence_after();
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tq + 16 * c, v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (cb + j < nch) tmem_ld_32x32b_x4(tl + (cb + j) * 16, v[j]);
-          tmem_ld_wait();
-          uint32_t lb[4] = {0u, 0u, 0u, 0u};   // this batch's list entries (bit j: chunk cb + j)
+        for (int j = 0; j < 16; ++j) reg_fence(v[j]);
+        if (!keep_tmem) release(c);
+        const int base_t = c * 128 + q * 32;
+        const bool partial = base_t + 32 > nvmin;   // some classified member cannot use every lane
+        uint32_t lm[16];
+        uint32_t my_above = 0u, my_n = 0u;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int c = cb + j;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              reg_fence(v[j][i]);
-              const float f = __uint_as_float(v[j][i]);
-              const uint32_t in = c < nch ? (cm[i] >> c) & 1u : 0u;
-              const uint32_t above = f >= th4[i] ? in : 0u;
-              const uint32_t inlist = f >= tl4[i] ? in : 0u;
-              gt[i] |= above << c;
-              lb[i] |= (inlist & ~above) << j;
-            }
+        for (int j = 0; j < 16; ++j) {
+          const float f = __uint_as_float(v[j]);
+          uint32_t a = __ballot_sync(0xffffffffu, f >= th[j]);
+          uint32_t b = __ballot_sync(0xffffffffu, f >= tl[j]);
+          if (partial) {
+            const int u = M->ms[j].nv - base_t;
+            const uint32_t um = u >= 32 ? 0xFFFFFFFFu : (u <= 0 ? 0u : ((1u << u) - 1u));
+            a &= um;
+            b &= um;
           }
-          // append to the lists: one shared atomic per warp and member
+          lm[j] = b & ~a;
+          my_above = lane == j ? a : my_above;
+          my_n = lane == j ? static_cast<uint32_t>(__popc(lm[j])) : my_n;
+        }
+        // lane j < 16: member j's bitmap word and list reservation
+        if (lane < 16) bmp[lane * 128 + c * 4 + q] = my_above;
+        uint32_t base = 0u;
+        if (lane < 16 && my_n != 0u) base = atom_shared_add(smem_u32(&M->ms[lane].nlist), my_n);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (__any_sync(0xffffffffu, lb[i] != 0u)) {
-              const int m = 4 * grp + i;
-              const int cnt = __popc(lb[i]);
-              int incl = cnt;
-#pragma unroll
-              for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-              }
-              int base = 0;
-              if (lane == 31) base = static_cast<int>(atom_shared_add(smem_u32(&M->ms[m].nlist), static_cast<uint32_t>(incl)));
-              base = __shfl_sync(0xffffffffu, base, 31);
-              int at = base + incl - cnt;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                if ((lb[i] >> j) & 1u) {
-                  if (at < kCap) {
-                    lkeys[m * kCap + at] = score_key(__uint_as_float(v[j][i]));
-                    lslot[m * kCap + at] = static_cast<uint16_t>(r * nch + cb + j);
-                  }
-                  ++at;
-                }
+        for (int j = 0; j < 16; ++j) {
+          if (lm[j] != 0u) {
+            const uint32_t bj = __shfl_sync(0xffffffffu, base, j);
+            if ((lm[j] >> lane) & 1u) {
+              const uint32_t at = bj + static_cast<uint32_t>(__popc(lm[j] & ltmask));
+              if (at < static_cast<uint32_t>(kCap)) {
+                lkeys[j * kCap + at] = v[j];
+                lslot[j * kCap + at] = static_cast<uint16_t>(base_t + lane);
               }
             }
           }
         }
-        if (!keep_tmem) release_upto(min(cb + 4, nch));
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int n = __reduce_add_sync(0xffffffffu, __popc(gt[i]));
-        if (lane == 0 && n > 0) atom_shared_add(smem_u32(&M->ms[4 * grp + i].nabove), static_cast<uint32_t>(n));
       }
       if (named_barrier_or(2, C::NSEL, !ok)) break;
 
       // ---- warp sw ranks member sw's list exactly: the need-th largest key
       //      (radix select from the highest bit that varies) and how many of
-      //      its copies are taken; decisions to the member's bitmap
+      //      its copies are taken; decisions OR-ed into the member's bitmap
+      uint32_t* mb = bmp + sw * 128;
       if (sw < nb) {
         MemberSel& S = M->ms[sw];
         int mode = S.mode;
         if (mode == kMList || mode == kMBand) {
-          const int n = S.nlist, need = S.K - S.nabove;
+          int nabove = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) nabove += __popc(mb[lane + 32 * w]);
+          nabove = __reduce_add_sync(0xffffffffu, nabove);
+          const int n = S.nlist, need = S.K - nabove;
           if (n > kCap || need < 1 || need > n) {
             mode = kMMiss;   // the k-th score fell outside the interval, or the list overflowed
           } else {
-            const uint32_t* lk = lkeys + sw * kCap;
+            uint32_t* lk = lkeys + sw * kCap;
             const uint16_t* ls = lslot + sw * kCap;
-            uint32_t* rh = hist + sw * kBins;   // radix histogram (256 words)
-            uint32_t* bs = rh + 256;            // decision bitmap (one bit per candidate slot)
-            for (int w = lane; w < 128; w += 32) bs[w] = 0u;
+            uint32_t* rh = hist + sw * kBins;   // radix histogram
+            for (int e = lane; e < n; e += 32) lk[e] = score_key(__uint_as_float(lk[e]));
+            __syncwarp();
             uint32_t tk = 0u, tmask = 0u;
-            int need_eq = 0x7FFFFFFF;
+            int need_eq = 0x7FFFFFFF;   // the whole list, when need == n
             if (need < n) {
               const uint32_t k0 = lk[0];
               uint32_t diff = 0u;
@@ -777,7 +749,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               }
               if (take) {
                 const int t = ls[e];
-                red_shared_or(smem_u32(&bs[t >> 5]), 1u << (t & 31));
+                red_shared_or(smem_u32(&mb[t >> 5]), 1u << (t & 31));
               }
             }
           }
@@ -790,132 +762,74 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         }
         __syncwarp();
       }
-      sel_sync();
-
-      // ---- rows: each member's taken candidates in ascending order
-      auto my_bits = [&](const uint32_t* bm) -> uint32_t {
-        if (nch == 0) return 0u;
-        const int t0 = r * nch;
-        const int w = t0 >> 5, o = t0 & 31;
-        uint32_t x = bm[w] >> o;
-        if (o != 0 && w + 1 < 128) x |= bm[w + 1] << (32 - o);
-        return nch >= 32 ? x : (x & ((1u << nch) - 1u));
-      };
-      uint32_t selm[4];
-      int mode4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = 4 * grp + i;
-        mode4[i] = M->ms[m].mode;
-        selm[i] = 0u;
-        if (mode4[i] == kMAll) selm[i] = um[i];
-        else if (mode4[i] == kMList || mode4[i] == kMBand) selm[i] = gt[i] | my_bits(hist + m * kBins + 256);
-      }
-      // group scan (thread order = candidate order) of the four members' counts
-      int ex[4];
-      {
-        int incl[4], own[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) incl[i] = own[i] = __popc(selm[i]);
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int y = __shfl_up_sync(0xffffffffu, incl[i], o);
-            if (lane >= o) incl[i] += y;
-          }
-        }
-        if (lane == 31) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) M->gscan[grp][quarter][i] = incl[i];
-        }
-        named_barrier(3 + grp, 128);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int off = 0;
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) off += (qq < quarter) ? M->gscan[grp][qq][i] : 0;
-          ex[i] = off + incl[i] - own[i];
-        }
-      }
-      // the ranked lists' bytes become per-warp output staging (STGE entries
-      // a warp); a warp's slice of a row goes out in STGE-entry parts
-      constexpr int STGE = C::STGE;
-      uint32_t* stg = lkeys + sw * STGE;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = 4 * grp + i;
-        if (m >= nb || mode4[i] == kMMiss) continue;   // a miss is written by refine_fallback_kernel
-        const int K = M->ms[m].K;
-        const uint32_t sel = selm[i];
-        const int slot = ex[i];
-        const int wb = __shfl_sync(0xffffffffu, slot, 0);
-        // (the selection takes exactly K; the bound only guards the row)
-        const int wc = min(__shfl_sync(0xffffffffu, slot + __popc(sel), 31), K) - wb;
-        const long long orow_off = ((it.qrow0 + it.mb + m) * p.H + it.h) * static_cast<long long>(p.top_k);
+      // ---- warp sw writes member sw's row: its bitmap in candidate order,
+      //      one coalesced store per word (a miss is written by the fallback)
+      if (sw < nb) {
+        const MemberSel& S = M->ms[sw];
+        const int mode = S.mode, K = S.K;
+        const long long orow_off = ((it.qrow0 + it.mb + sw) * p.H + it.h) * static_cast<long long>(p.top_k);
         int32_t* orow = p.out + orow_off;
-        for (int part = 0; part * STGE < wc; ++part) {
-          const int plo = part * STGE;
-          // this lane's selected candidates that fall in the part [plo, plo + STGE)
-          const int o0 = slot - wb - plo;
-          uint32_t bits = sel;
-          if (o0 < 0) {  // skip the ones staged by an earlier part
-            for (int k = 0; k < -o0 && bits; ++k) bits &= bits - 1;
+        uint32_t* pre = hist + sw * kBins;   // per-word prefix counts, for the scores
+        if (mode == kMAll) {
+          for (int t = lane; t < K; t += 32) orow[t] = cx[t];
+        } else if (mode == kMList || mode == kMBand) {
+          int base = 0;
+#pragma unroll 1
+          for (int w = 0; w < nch * 4; w += 4) {
+            const uint4 wd = *reinterpret_cast<const uint4*>(mb + w);
+            const uint32_t ws[4] = {wd.x, wd.y, wd.z, wd.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              if (keep_tmem && lane == 0) pre[w + x] = static_cast<uint32_t>(base);
+              if ((ws[x] >> lane) & 1u) orow[base + __popc(ws[x] & ltmask)] = cx[(w + x) * 32 + lane];
+              base += __popc(ws[x]);
+            }
           }
-          // two entries an iteration: their index loads overlap
-          int o = max(o0, 0);
-          while (bits != 0u && o < STGE) {
-            const int c1 = __ffs(bits) - 1;
-            bits &= bits - 1;
-            const bool two = bits != 0u && o + 1 < STGE;
-            const int c2 = two ? __ffs(bits) - 1 : c1;
-            if (two) bits &= bits - 1;
-            const uint32_t v1 = static_cast<uint32_t>(cx[cidx_pos(c1, r)]);
-            const uint32_t v2 = static_cast<uint32_t>(cx[cidx_pos(c2, r)]);
-            stg[o] = v1;
-            if (two) stg[o + 1] = v2;
-            o += two ? 2 : 1;
-          }
-          __syncwarp();
-          const int n = min(wc - plo, STGE);
-#pragma unroll 4
-          for (int x = lane; x < n; x += 32) orow[wb + plo + x] = static_cast<int32_t>(stg[x]);
-          __syncwarp();
         }
-        if (p.out_scores) {
-          float* srow = p.out_scores + orow_off;
-          const uint32_t any = __reduce_or_sync(0xffffffffu, sel);
-          for (int part = 0; part * STGE < wc; ++part) {
-            const int plo = part * STGE;
-            int o = slot - wb - plo;
-            for (uint32_t a = any; a; a &= a - 1) {
-              const int c = __ffs(a) - 1;
-              uint32_t v;
-              tmem_ld_32x32b_x1(tl + c * 16 + i, v);
-              tmem_ld_wait();
-              if ((sel >> c) & 1u) {
-                if (o >= 0 && o < STGE) stg[o] = v;
-                ++o;
+        if (mode != kMMiss) {
+          for (int t = K + lane; t < p.top_k; t += 32) orow[t] = -1;
+          if (keep_tmem)
+            for (int t = K + lane; t < p.top_k; t += 32) p.out_scores[orow_off + t] = __int_as_float(0x7fc00000);
+        }
+      }
+      if (keep_tmem) {
+        // the selected scores, read again from TMEM, then the columns go back
+        sel_sync();
+        for (int i = st; i < nch; i += 4) {
+          const int c = chunk_at(i, nch);
+          tc_fence_after();
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tq + 16 * c, v);
+          tmem_ld_wait();
+          const int t = c * 128 + q * 32 + lane;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            reg_fence(v[j]);
+            if (j < nb) {
+              const int mode = M->ms[j].mode;
+              float* srow = p.out_scores + ((it.qrow0 + it.mb + j) * p.H + it.h) * static_cast<long long>(p.top_k);
+              if (mode == kMAll) {
+                if (t < M->ms[j].K) srow[t] = __uint_as_float(v[j]);
+              } else if (mode == kMList || mode == kMBand) {
+                const uint32_t word = bmp[j * 128 + c * 4 + q];
+                if ((word >> lane) & 1u)
+                  srow[hist[j * kBins + c * 4 + q] + __popc(word & ltmask)] = __uint_as_float(v[j]);
               }
             }
-            __syncwarp();
-            const int n = min(wc - plo, STGE);
-            for (int x = lane; x < n; x += 32) srow[wb + plo + x] = __uint_as_float(stg[x]);
-            __syncwarp();
           }
-          for (int x = K + r; x < p.top_k; x += 128) srow[x] = __int_as_float(0x7fc00000);
+          release(c);
         }
-        for (int x = K + r; x < p.top_k; x += 128) orow[x] = -1;
       }
-      // Chunks past this item's list got their "scored" commit without MMAs.
+      // Chunks past this item's list got their "scored" commit without MMAs;
+      // this warp's stream owns those at positions st, st+4, ... past nch.
       // Wait for those commits too before giving the chunks back: every
       // release then answers a commit of this item, and the MMA warp can never
       // find a chunk's "free" barrier two phases ahead of its wait.
-      for (int c = nch; c < NCH; ++c)
+      for (int c = nch + ((st - nch) & 3); c < NCH; c += 4) {
         if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
-      ok = __all_sync(0xffffffffu, ok);
-      // this item's TMEM columns and candidate list are free
-      if (ok) release_upto(NCH);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) release(c);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&M->cfree[buf]));
       ++kk;
@@ -959,7 +873,7 @@ __global__ void __launch_bounds__(kRfbNT) refine_fallback_kernel(RefineParams p)
     const int32_t* row = p.cand + (static_cast<long long>(it.h) * p.G + it.u) * KW;
     const long long qrow = (it.qrow0 + m) * p.H + it.h;
     __syncthreads();
-    for (int t = threadIdx.x; t < it.nc; t += kRfbNT) cl[t] = row[cand_word(t, it.nch)];
+    for (int t = threadIdx.x; t < it.nc; t += kRfbNT) cl[t] = row[t];
     for (int c = threadIdx.x; c < D; c += kRfbNT) qv[c] = __uint_as_float(static_cast<uint32_t>(p.q[qrow * D + c]) << 16);
     __syncthreads();
     if (threadIdx.x == 0) {
