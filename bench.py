@@ -69,11 +69,91 @@ def algorithmic(c):
         "scan_filter": ("tensor", scan_flops),
         # a select must at least read Kc (key, index) pairs and write Kc indices per row
         "finalize": ("hbm", float(H * nC.sum() * (8 + 4))),
-        # output rows + candidate rows + member queries + every key once
-        "refine": ("hbm", float(L * H * k * 4 + H * nC.sum() * 4 + 2 * L * H * d * 2)),
+        # candidate rows + member queries + every key once + selection bitmaps (512 B a row) written
+        "refine": ("hbm", float(H * nC.sum() * 4 + 2 * L * H * d * 2 + L * H * 512)),
+        # bitmaps read + output rows written + candidate rows read once
+        "refine_expand": ("hbm", float(L * H * 512 + L * H * k * 4 + H * nC.sum() * 4)),
         "proxy": ("hbm", float(L * H * d * 2 + G * H * d * 2)),
         "fallback": ("hbm", 0.0),
+        "refine_fallback": ("hbm", 0.0),
     }
+
+
+def config_work(c):
+    """The method's own work per call on a prefill workload: compulsory HBM
+    bytes (q and k read once, the index rows written once, and for Refine the
+    candidate rows written and read once) and the scan's tensor-core flops
+    (Refine scans j < last of each group, Reuse j < group start, dense j < pos)."""
+    L, H, d, g, k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
+    G = (L + g - 1) // g
+    s = np.arange(G, dtype=np.int64) * g
+    last = np.minimum(s + g, L) - 1
+    qk = 2 * L * H * d * 2
+    out = L * H * k * 4
+    nC = np.minimum(Kc, last)
+    return {
+        "refine": {"bytes": float(qk + out + 2 * H * nC.sum() * 4), "flops": 2.0 * d * H * float(last.sum())},
+        "reuse": {"bytes": float(qk + out), "flops": 2.0 * d * H * float(s.sum())},
+        "dense": {"bytes": float(qk + out), "flops": 2.0 * d * H * float(np.arange(L, dtype=np.int64).sum())},
+    }
+
+
+def roofline_ms(work, pk):
+    """The slower of the HBM and the tensor-core bound, in ms (measured peaks)."""
+    return max(work["bytes"] / (pk["hbm"] * 1e9), work["flops"] / (pk["bf16"] * 1e12)) * 1e3
+
+
+def config_records(qg, torch, stream, pk, steps, names=("C0", "C1", "C2")):
+    """Refine, Reuse and dense on the smaller prefill workloads: ms per call,
+    query-heads/s, the fraction of each call's roofline, PIVOT's speedup over
+    the dense indexer and Recall@k against it (on a seeded sample of rows)."""
+    recs = {}
+    for name in names:
+        c = synthetic.CONFIGS[name]
+        q_np, k_np = synthetic.make_prefill(name)
+        q = torch.from_numpy(q_np.view(np.int16)).cuda().view(torch.bfloat16)
+        k = torch.from_numpy(k_np.view(np.int16)).cuda().view(torch.bfloat16)
+        L, H, d, g, top_k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
+        outs, ms = {}, {}
+        calls = {"refine": lambda o: qg.pivot_index(q, k, g, top_k, Kc, qg.REFINE, out=o),
+                 "reuse": lambda o: qg.pivot_index(q, k, g, top_k, Kc, qg.REUSE, out=o),
+                 "dense": lambda o: qg.dense_index(q, k, top_k, out=o)}
+        for mode, fn in calls.items():
+            o = torch.empty((L, H, top_k), dtype=torch.int32, device="cuda")
+            for _ in range(2):
+                fn(o)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn(o)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms[mode] = e0.elapsed_time(e1) / steps
+            outs[mode] = o
+        qg.sync_status()
+        rng = np.random.default_rng(11)
+        n = max(256, L * H // 100)
+        rows = torch.from_numpy(rng.integers(1, L, size=n)).cuda()
+        heads = torch.from_numpy(rng.integers(0, H, size=n)).cuda()
+        dn = outs["dense"][rows, heads].cpu().numpy()
+        rec = {}
+        for mode in ("refine", "reuse"):
+            pv = outs[mode][rows, heads].cpu().numpy()
+            rec[mode] = float(np.mean([np.intersect1d(a[a >= 0], b[b >= 0]).size / max(1, (b >= 0).sum())
+                                       for a, b in zip(pv, dn)]))
+        work = config_work(c)
+        recs[name] = {
+            "shape": f"L={L} H={H} d={d} g={g} top_k={top_k} Kc={Kc}",
+            "ms": ms,
+            "query_heads_per_s": {m: L * H / (v / 1000.0) for m, v in ms.items()},
+            "roofline_ms": {m: roofline_ms(work[m], pk) for m in ms},
+            "roofline_frac": {m: roofline_ms(work[m], pk) / ms[m] for m in ms},
+            "speedup_vs_dense": {"refine": ms["dense"] / ms["refine"], "reuse": ms["dense"] / ms["reuse"]},
+            "recall_at_k_vs_dense": rec, "recall_rows": int(n)}
+        del outs, q, k
+        torch.cuda.empty_cache()
+    return recs
 
 
 def measured_traffic(kernel, heads):
@@ -191,25 +271,59 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def cpu_baseline(c, q, k, budget_s=12.0, seed=0):
-    """The oracle, as it stands, on a seeded sample of (group, head) units."""
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def oracle_sample(c, q, k, budget_s, threads, seed):
+    """The oracle, as it stands, on seeded random (group, head) units of the
+    workload, one stream of units per host thread (the oracle is plain C called
+    through ctypes, which releases the GIL), until budget_s has passed.
+    Returns (query-heads indexed, units, wall seconds, summed per-unit seconds)."""
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     L, H, g = c["L"], c["H"], c["g"]
     G = (L + g - 1) // g
-    rng = np.random.default_rng(seed)
+
+    def worker(w):
+        rng = np.random.default_rng([seed, w])
+        t0 = time.perf_counter()
+        nq = nu = 0
+        busy = 0.0
+        while time.perf_counter() - t0 < budget_s:
+            gi = rng.integers(0, G, size=1).astype(np.int32)
+            hi = rng.integers(0, H, size=1).astype(np.int32)
+            a = time.perf_counter()
+            oracle.prefill_units(q, k, g, c["top_k"], c["Kc"], oracle.REFINE, gi, hi)
+            busy += time.perf_counter() - a
+            nq += min(int(gi[0]) * g + g, L) - int(gi[0]) * g
+            nu += 1
+        return nq, nu, busy
+
     t0 = time.perf_counter()
-    n_q = 0
-    n_units = 0
-    while time.perf_counter() - t0 < budget_s:
-        gi = rng.integers(0, G, size=4).astype(np.int32)
-        hi = rng.integers(0, H, size=4).astype(np.int32)
-        oracle.prefill_units(q, k, g, c["top_k"], c["Kc"], oracle.REFINE, gi, hi)
-        n_q += int(sum(min(i * g + g, L) - i * g for i in gi))
-        n_units += 4
-    dt = time.perf_counter() - t0
-    return {"value": n_q / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n_units} random (group, head) units of {WORKLOAD} ({n_q} query-heads), "
-                      f"single-threaded C, {dt:.1f} s"}
+    with ThreadPoolExecutor(threads) as ex:
+        res = list(ex.map(worker, range(threads)))
+    wall = time.perf_counter() - t0
+    return sum(r[0] for r in res), sum(r[1] for r in res), wall, sum(r[2] for r in res)
+
+
+def cpu_baseline(c, q, k, budget_s=12.0, seed=0):
+    """The oracle on all host cores, on a bounded sample of the workload, with
+    the full-workload time it implies (extrapolated: units are drawn uniformly,
+    so the mean unit time estimates the mean over all units)."""
+    cores = host_cores()
+    nq, nu, wall, busy = oracle_sample(c, q, k, budget_s, cores, seed)
+    L, H, g = c["L"], c["H"], c["g"]
+    units = ((L + g - 1) // g) * H
+    full_s = busy / max(nu, 1) * units / cores
+    return {"value": nq / wall, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{nu} random (group, head) units of {WORKLOAD} ({nq} query-heads) on {cores} threads, "
+                      f"single-threaded C oracle per unit, {wall:.1f} s",
+            "single_thread_value": nq / busy if busy > 0 else None,
+            "full_workload_s_extrapolated": full_s}
 
 
 def run_reference(args, rank):
@@ -220,32 +334,26 @@ def run_reference(args, rank):
     oracle.build()
     c = synthetic.CONFIGS[WORKLOAD]
     q, k = synthetic.make_prefill(WORKLOAD)
-    L, H, g = c["L"], c["H"], c["g"]
-    G = (L + g - 1) // g
-    rng = np.random.default_rng(1234)
-    units = 48
-
-    def step():
-        gi = rng.integers(0, G, size=units).astype(np.int32)
-        hi = rng.integers(0, H, size=units).astype(np.int32)
-        t0 = time.perf_counter()
-        oracle.prefill_units(q, k, g, c["top_k"], c["Kc"], oracle.REFINE, gi, hi)
-        return time.perf_counter() - t0, int(sum(min(i * g + g, L) - i * g for i in gi))
-
-    for _ in range(args.warmup):
-        step()
-    tot_t, tot_q = 0.0, 0
-    for _ in range(args.steps):
-        t, n = step()
-        tot_t += t
-        tot_q += n
+    cores = host_cores()
+    # each step: every host thread indexes random (group, head) units for a
+    # bounded time (the whole run stays within a few minutes)
+    step_s = max(0.5, min(4.0, 120.0 / max(1, args.steps + args.warmup)))
+    for w in range(args.warmup):
+        oracle_sample(c, q, k, step_s, cores, seed=1000 + w)
+    tot_t, tot_q, tot_u = 0.0, 0, 0
+    for s_ in range(args.steps):
+        nq, nu, wall, _ = oracle_sample(c, q, k, step_s, cores, seed=2000 + s_)
+        tot_t += wall
+        tot_q += nq
+        tot_u += nu
     value = tot_q / tot_t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(c),
-            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": 1,
-                             "sample": f"{units} random (group, head) units of {WORKLOAD} per step"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": cores,
+                             "sample": f"{tot_u} random (group, head) units of {WORKLOAD} over {args.steps} steps "
+                                       f"of {step_s:.1f} s on {cores} threads"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -259,6 +367,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the Reuse/dense comparison runs")
     ap.add_argument("--e2e-steps", type=int, default=2, help="0 skips the end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--no-configs", action="store_true", help="skip the records of the smaller prefill workloads")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: index only this many heads of the workload (0 = all)")
     args = ap.parse_args()
@@ -441,10 +550,20 @@ def main():
                   "key_bytes": key_bytes}
         del dq, dk, dcu, dout
         torch.cuda.empty_cache()
+        w3 = config_work(c)
         extras = {"refine_ms": ms, "reuse_ms": reuse_ms, "dense_ms": dense_ms, "decode": decode,
                   "speedup_refine_vs_dense": dense_ms / ms, "speedup_reuse_vs_dense": dense_ms / reuse_ms,
-                  "recall_at_k_vs_dense": rec, "recall_rows": int(rows.numel())}
+                  "recall_at_k_vs_dense": rec, "recall_rows": int(rows.numel()),
+                  "roofline_ms": {"refine": roofline_ms(w3["refine"], pk), "reuse": roofline_ms(w3["reuse"], pk),
+                                  "dense": roofline_ms(w3["dense"], pk)},
+                  "roofline_frac": {"refine": roofline_ms(w3["refine"], pk) / ms,
+                                    "reuse": roofline_ms(w3["reuse"], pk) / reuse_ms,
+                                    "dense": roofline_ms(w3["dense"], pk) / dense_ms}}
         del out_reuse
+        if not args.no_configs:
+            del out
+            torch.cuda.empty_cache()
+            extras["configs"] = config_records(qg, torch, stream, pk, max(3, args.steps))
 
     if rank == 0:
         import oracle

@@ -239,6 +239,22 @@ __device__ __forceinline__ void red_shared_min(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void red_shared_max(uint32_t addr, uint32_t v) {
   asm volatile("red.shared.max.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+// Shared-memory reductions and stores without a compiler memory barrier, for
+// hot loops whose results are read only after a thread barrier (which orders
+// them): the compiler may then keep independent loads and arithmetic of
+// neighbouring iterations in flight around them.
+__device__ __forceinline__ void red_shared_add_nb(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+__device__ __forceinline__ void red_shared_or_nb(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+__device__ __forceinline__ void st_shared_u32_nb(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+__device__ __forceinline__ void st_shared_u16_nb(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v));
+}
 __device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
 }

@@ -47,8 +47,9 @@
 //  * the list is ranked exactly (a warp radix select: the need-th largest key
 //    and how many of its copies are taken, ties in candidate order), and its
 //    decisions are OR-ed into the bitmap;
-//  * the member's warp walks the bitmap in candidate order: each 32-bit word
-//    gives one coalesced store of its selected key indices.
+//  * the member's warp writes the bitmap out (512 bytes); refine_expand_kernel
+//    turns every bitmap into its index row afterwards, so the row writes
+//    (4 bytes per index) do not take issue slots from this kernel.
 // A member whose k-th score fell outside its interval, whose list overflowed,
 // or whose sample had no score range is not written here: it is recorded in a
 // miss list and refine_fallback_kernel redoes it exactly afterwards.
@@ -64,6 +65,7 @@ struct RefineParams {
   const uint16_t* keys;   // prefill [L][H][d]; decode packed cache [rows][H][d]
   const int32_t* cand;    // [H][G][cand_row_words(Kc)] candidate rows in read order (ptx.cuh)
   int32_t* out;           // prefill [L][H][top_k]; decode [B][g][H][top_k]
+  uint32_t* sel;          // selection bitmaps, 128 words per output row (bit t: candidate t taken)
   float* out_scores;      // same shape as out, or null
   const int32_t* cu;      // decode: [B+1] cache row offsets; null for prefill
   int G, L, H, g, top_k, Kc, d;
@@ -86,7 +88,7 @@ enum : int {
   kMMiss = 4,   // redone by refine_fallback_kernel
 };
 
-constexpr int kBins = 256;          // sample histogram bins per member
+constexpr int kBins = 1024;         // sample histogram bins per member
 // 2^23: a float in [2^23, 2^24) is an integer, held in its low mantissa bits
 constexpr float kMagic = 8388608.0f;
 constexpr int kCap = 512;           // boundary list entries per member
@@ -127,21 +129,23 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
   static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
-  // per member kBins 32-bit words: the sample histogram, later the list's
-  // 256-bin radix histogram, and with the scores written out the selection's
-  // per-word prefix counts
-  static constexpr int HIST_BYTES = 16 * kBins * 4;
-  static constexpr int BMP_BYTES = 16 * 128 * 4;        // selection bitmaps: one bit per candidate slot
+  // selection bitmaps: one bit per candidate slot
+  static constexpr int BMP_BYTES = 16 * 128 * 4;
+  // per member 256 32-bit words: the list's radix histogram, and with the
+  // scores written out the selection's per-word prefix counts
+  static constexpr int HIST_BYTES = 16 * 256 * 4;
   static constexpr int LK_BYTES = 16 * kCap * 4;        // list scores (fp32 bits, then order keys)
   static constexpr int LT_BYTES = 16 * kCap * 2;        // list candidate slots
+  // the sample histograms ([16][kBins] words) span the histogram and list
+  // bytes, which are not in use before the pass that fills the lists
+  static_assert(16 * kBins * 4 == HIST_BYTES + LK_BYTES + LT_BYTES, "sample histograms span hist + lists");
   __host__ __device__ static int nch_max(int Kc) { return (Kc + 127) / 128; }
   __host__ __device__ static int cidx_words(int Kc) { return nch_max(Kc) * 128; }
-  __host__ __device__ static int off_hist(int Kc) { return OFF_C + 2 * cidx_words(Kc) * 4; }
+  __host__ __device__ static int off_bmp(int Kc) { return OFF_C + 2 * cidx_words(Kc) * 4; }
   static int smem_bytes(int Kc) {
-    return off_hist(Kc) + HIST_BYTES + BMP_BYTES + LK_BYTES + LT_BYTES + static_cast<int>(sizeof(RefineMisc)) +
+    return off_bmp(Kc) + BMP_BYTES + HIST_BYTES + LK_BYTES + LT_BYTES + static_cast<int>(sizeof(RefineMisc)) +
            1024;
   }
-  static_assert(kBins == 256, "the radix histogram reuses a member's histogram words");
 };
 
 // Linear bin of a score, round(s * scale + off) clamped to [0, kBins-1], with
@@ -295,9 +299,10 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   const int NCH = C::nch_max(p.Kc);
   const int CW = C::cidx_words(p.Kc);
   int32_t* cidx0 = reinterpret_cast<int32_t*>(smem + C::OFF_C);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::off_hist(p.Kc));      // [16][kBins]
-  uint32_t* bmp = hist + C::HIST_BYTES / 4;                                     // [16][128]
-  uint32_t* lkeys = bmp + C::BMP_BYTES / 4;                                     // [16][kCap]
+  uint32_t* bmp = reinterpret_cast<uint32_t*>(smem + C::off_bmp(p.Kc));       // [16][128]
+  uint32_t* hist = bmp + C::BMP_BYTES / 4;                                      // [16][256]
+  uint32_t* shist = hist;                                                       // [16][kBins], phase A only
+  uint32_t* lkeys = hist + C::HIST_BYTES / 4;                                   // [16][kCap]
   uint16_t* lslot = reinterpret_cast<uint16_t*>(lkeys + C::LK_BYTES / 4);       // [16][kCap]
   RefineMisc* M = reinterpret_cast<RefineMisc*>(lslot + C::LT_BYTES / 2);
   volatile int* abort_flag = &M->abort_flag;
@@ -500,8 +505,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         S.kmin = 0xFFFFFFFFu;
         S.kmax = 0u;
       }
-      for (int i = stid; i < (C::HIST_BYTES + C::BMP_BYTES) / 16; i += C::NSEL)
-        reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+      // bitmaps and sample histograms start at zero
+      for (int i = stid; i < (C::BMP_BYTES + 16 * kBins * 4) / 16; i += C::NSEL)
+        reinterpret_cast<uint4*>(bmp)[i] = make_uint4(0, 0, 0, 0);
       if (named_barrier_or(2, C::NSEL, !ok)) break;
       bool anyb = false;     // a member with a sampled interval (uniform)
       int nvmin = 0x7FFFFFFF;  // fewest usable candidates of a classified member (uniform)
@@ -570,7 +576,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             reg_fence(v[j]);
             const MemberSel& S = M->ms[j];
             if (S.mode == kMBand && t < S.nv)
-              red_shared_add(smem_u32(hist + j * kBins + value_bin(__uint_as_float(v[j]), S.scale, S.offm)), 1u);
+              red_shared_add_nb(smem_u32(shist + j * kBins + value_bin(__uint_as_float(v[j]), S.scale, S.offm)), 1u);
           }
         }
         if (named_barrier_or(2, C::NSEL, !ok)) break;
@@ -579,7 +585,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         // is drawn without replacement)
         if (sw < nb && M->ms[sw].mode == kMBand) {
           MemberSel& S = M->ms[sw];
-          const uint32_t* hm = hist + sw * kBins;
+          const uint32_t* hm = shist + sw * kBins;
           int n_s = 0;
 #pragma unroll
           for (int b = 0; b < kBins / 32; ++b) n_s += static_cast<int>(hm[lane * (kBins / 32) + b]);
@@ -616,6 +622,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       //      go back as soon as they are loaded (unless the scores are
       //      written out, which reads them again)
       const bool keep_tmem = p.out_scores != nullptr;
+      const uint32_t lk_s = smem_u32(lkeys), ls_s = smem_u32(lslot);
       float th[16], tl[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -660,17 +667,15 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         if (lane < 16) bmp[lane * 128 + c * 4 + q] = my_above;
         uint32_t base = 0u;
         if (lane < 16 && my_n != 0u) base = atom_shared_add(smem_u32(&M->ms[lane].nlist), my_n);
+        // every member's slots at once: no branch keeps one member's shuffle
+        // and stores from overlapping the next member's
+        const uint16_t slot = static_cast<uint16_t>(base_t + lane);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          if (lm[j] != 0u) {
-            const uint32_t bj = __shfl_sync(0xffffffffu, base, j);
-            if ((lm[j] >> lane) & 1u) {
-              const uint32_t at = bj + static_cast<uint32_t>(__popc(lm[j] & ltmask));
-              if (at < static_cast<uint32_t>(kCap)) {
-                lkeys[j * kCap + at] = v[j];
-                lslot[j * kCap + at] = static_cast<uint16_t>(base_t + lane);
-              }
-            }
+          const uint32_t at = __shfl_sync(0xffffffffu, base, j) + static_cast<uint32_t>(__popc(lm[j] & ltmask));
+          if (((lm[j] >> lane) & 1u) && at < static_cast<uint32_t>(kCap)) {
+            st_shared_u32_nb(lk_s + 4u * (j * kCap + at), v[j]);
+            st_shared_u16_nb(ls_s + 2u * (j * kCap + at), slot);
           }
         }
       }
@@ -694,7 +699,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           } else {
             uint32_t* lk = lkeys + sw * kCap;
             const uint16_t* ls = lslot + sw * kCap;
-            uint32_t* rh = hist + sw * kBins;   // radix histogram
+            uint32_t* rh = hist + sw * 256;   // radix histogram
             for (int e = lane; e < n; e += 32) lk[e] = score_key(__uint_as_float(lk[e]));
             __syncwarp();
             uint32_t tk = 0u, tmask = 0u;
@@ -718,7 +723,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
                 __syncwarp();
                 for (int e = lane; e < n; e += 32) {
                   const uint32_t key = lk[e];
-                  if ((key & tmask) == tk) red_shared_add(smem_u32(&rh[(key >> sh) & nbm]), 1u);
+                  if ((key & tmask) == tk) red_shared_add_nb(smem_u32(&rh[(key >> sh) & nbm]), 1u);
                 }
                 __syncwarp();
                 int above;
@@ -749,7 +754,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               }
               if (take) {
                 const int t = ls[e];
-                red_shared_or(smem_u32(&mb[t >> 5]), 1u << (t & 31));
+                red_shared_or_nb(smem_u32(&mb[t >> 5]), 1u << (t & 31));
               }
             }
           }
@@ -762,34 +767,44 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         }
         __syncwarp();
       }
-      // ---- warp sw writes member sw's row: its bitmap in candidate order,
-      //      one coalesced store per word (a miss is written by the fallback)
+      // ---- warp sw writes member sw's selection bitmap (refine_expand_kernel
+      //      makes the index row; a miss's row is redone by the fallback)
       if (sw < nb) {
         const MemberSel& S = M->ms[sw];
         const int mode = S.mode, K = S.K;
-        const long long orow_off = ((it.qrow0 + it.mb + sw) * p.H + it.h) * static_cast<long long>(p.top_k);
-        int32_t* orow = p.out + orow_off;
-        uint32_t* pre = hist + sw * kBins;   // per-word prefix counts, for the scores
-        if (mode == kMAll) {
-          for (int t = lane; t < K; t += 32) orow[t] = cx[t];
-        } else if (mode == kMList || mode == kMBand) {
-          int base = 0;
-#pragma unroll 1
-          for (int w = 0; w < nch * 4; w += 4) {
-            const uint4 wd = *reinterpret_cast<const uint4*>(mb + w);
-            const uint32_t ws[4] = {wd.x, wd.y, wd.z, wd.w};
+        const long long orow = (it.qrow0 + it.mb + sw) * p.H + it.h;
+        uint32_t wds[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              if (keep_tmem && lane == 0) pre[w + x] = static_cast<uint32_t>(base);
-              if ((ws[x] >> lane) & 1u) orow[base + __popc(ws[x] & ltmask)] = cx[(w + x) * 32 + lane];
-              base += __popc(ws[x]);
-            }
+        for (int x = 0; x < 4; ++x) {
+          const int w = 4 * lane + x;
+          if (mode == kMAll) {
+            const int u = K - 32 * w;
+            wds[x] = u >= 32 ? 0xFFFFFFFFu : (u <= 0 ? 0u : ((1u << u) - 1u));
+          } else if (mode == kMList || mode == kMBand) {
+            wds[x] = mb[w];
+          } else {
+            wds[x] = 0u;
           }
         }
-        if (mode != kMMiss) {
-          for (int t = K + lane; t < p.top_k; t += 32) orow[t] = -1;
-          if (keep_tmem)
-            for (int t = K + lane; t < p.top_k; t += 32) p.out_scores[orow_off + t] = __int_as_float(0x7fc00000);
+        reinterpret_cast<uint4*>(p.sel + orow * 128)[lane] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+        if (keep_tmem) {
+          // per-word prefix counts of the selection, for the scores' slots
+          const int own = __popc(wds[0]) + __popc(wds[1]) + __popc(wds[2]) + __popc(wds[3]);
+          int incl = own;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          uint32_t* pre = hist + sw * 256;
+          int at = incl - own;
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            pre[4 * lane + x] = static_cast<uint32_t>(at);
+            at += __popc(wds[x]);
+          }
+          if (mode != kMMiss)
+            for (int t = K + lane; t < p.top_k; t += 32) p.out_scores[orow * p.top_k + t] = __int_as_float(0x7fc00000);
         }
       }
       if (keep_tmem) {
@@ -813,7 +828,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               } else if (mode == kMList || mode == kMBand) {
                 const uint32_t word = bmp[j * 128 + c * 4 + q];
                 if ((word >> lane) & 1u)
-                  srow[hist[j * kBins + c * 4 + q] + __popc(word & ltmask)] = __uint_as_float(v[j]);
+                  srow[hist[j * 256 + c * 4 + q] + __popc(word & ltmask)] = __uint_as_float(v[j]);
               }
             }
           }
@@ -842,6 +857,43 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+constexpr int kExpNT = 256;
+
+// Index rows from the selection bitmaps: one warp per output row walks the
+// row's 128 bitmap words in candidate order; each word gives one coalesced
+// store of its selected key indices (the candidates of the row's group,
+// ascending); the row is padded with -1 after its popcount.
+__global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, long long nrows) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t ltmask = (1u << lane) - 1u;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (kExpNT / 32);
+  const int CWd = cand_row_words(p.Kc);
+  for (long long row = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; row < nrows; row += nwarps) {
+    const int h = static_cast<int>(row % p.H);
+    const long long qr = row / p.H;   // prefill: the position; decode: b * g + i
+    const int u = static_cast<int>(qr / p.g);
+    const int32_t* crow = p.cand + (static_cast<long long>(h) * p.G + u) * CWd;
+    const uint32_t* srow = p.sel + row * 128;
+    int32_t* orow = p.out + row * p.top_k;
+    const int nw = min(128, CWd / 32);
+    int base = 0;
+#pragma unroll 1
+    for (int w = 0; w < nw; w += 4) {
+      const uint4 wd = *reinterpret_cast<const uint4*>(srow + w);   // the same 16 bytes for every lane
+      const uint32_t ws[4] = {wd.x, wd.y, wd.z, wd.w};
+      int32_t val[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) val[x] = ws[x] ? crow[(w + x) * 32 + lane] : 0;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        if ((ws[x] >> lane) & 1u) orow[base + __popc(ws[x] & ltmask)] = val[x];
+        base += __popc(ws[x]);
+      }
+    }
+    for (int t = base + lane; t < p.top_k; t += 32) orow[t] = -1;
   }
 }
 
