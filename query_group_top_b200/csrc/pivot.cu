@@ -282,7 +282,8 @@ int launch_refine(RefineParams rp, int units, long long rows, int sms, uint8_t* 
   CUDA_TRY(cudaGetLastError());
   {
     TraceScope tr("refine_expand", st);
-    const long long blocks = std::min<long long>((rows + kExpNT / 32 - 1) / (kExpNT / 32), 32ll * std::max(1, sms));
+    const long long units_w = static_cast<long long>(units);   // one warp per unit
+    const long long blocks = std::min<long long>((units_w + kExpNT / 32 - 1) / (kExpNT / 32), 32ll * std::max(1, sms));
     refine_expand_kernel<<<static_cast<unsigned>(std::max<long long>(1, blocks)), kExpNT, 0, st>>>(rp, rows);
   }
   CUDA_TRY(cudaGetLastError());

@@ -153,9 +153,10 @@ struct RefineCfg {
 // in [2^23, 2^23 + kBins-1] after the clamps, and the bin is its low mantissa
 // bits.  One rounding of a function increasing in s, then monotone clamps, so
 // the bins are ordered like the scores, and -0 and +0 share a bin.
+template <int NB = kBins>
 __device__ __forceinline__ int value_bin(float s, float scale, float offm) {
-  const float t = fminf(fmaxf(__fmaf_rn(s, scale, offm), kMagic), kMagic + static_cast<float>(kBins - 1));
-  return static_cast<int>(__float_as_uint(t) & static_cast<uint32_t>(kBins - 1));
+  const float t = fminf(fmaxf(__fmaf_rn(s, scale, offm), kMagic), kMagic + static_cast<float>(NB - 1));
+  return static_cast<int>(__float_as_uint(t) & static_cast<uint32_t>(NB - 1));
 }
 
 // Bin of an order key; key patterns beyond the infinities (no score has them)
@@ -202,10 +203,14 @@ __device__ __forceinline__ uint32_t warp_first_key_of_bin(int b, float scale, fl
 template <int NBINS>
 __device__ __forceinline__ int warp_rank_bin(const uint32_t* h, int r, int lane, int* above) {
   constexpr int PER = NBINS / 32;
+  static_assert(PER % 4 == 0, "bins are read four at a time");
   const int b0 = NBINS - PER * (lane + 1);
   int s = 0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) s += static_cast<int>(h[b0 + i]);
+  for (int i = 0; i < PER / 4; ++i) {
+    const uint4 x = reinterpret_cast<const uint4*>(h + b0)[i];
+    s += static_cast<int>(x.x + x.y + x.z + x.w);
+  }
   int incl = s;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -586,10 +591,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         if (sw < nb && M->ms[sw].mode == kMBand) {
           MemberSel& S = M->ms[sw];
           const uint32_t* hm = shist + sw * kBins;
+          // the usable candidates among the sampled chunks
           int n_s = 0;
-#pragma unroll
-          for (int b = 0; b < kBins / 32; ++b) n_s += static_cast<int>(hm[lane * (kBins / 32) + b]);
-          n_s = __reduce_add_sync(0xffffffffu, n_s);
+          for (int i = 0; i < s_ch; ++i) n_s += min(max(S.nv - 128 * chunk_at(i, nch), 0), 128);
           const float pk = static_cast<float>(S.K) / static_cast<float>(S.nv);
           const float e = pk * static_cast<float>(n_s);
           const float fpc = fmaxf(0.f, 1.f - static_cast<float>(n_s) / static_cast<float>(S.nv));
@@ -704,7 +708,68 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             __syncwarp();
             uint32_t tk = 0u, tmask = 0u;
             int need_eq = 0x7FFFFFFF;   // the whole list, when need == n
+            bool ranked = false;        // decisions already in the bitmap
             if (need < n) {
+              // bins linear in the score over the list's own range spread its
+              // keys evenly; the need-th largest lies in bin b, and the few
+              // keys of bin b are ranked exactly against each other
+              uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+              for (int e = lane; e < n; e += 32) {
+                kmn = min(kmn, lk[e]);
+                kmx = max(kmx, lk[e]);
+              }
+              kmn = __reduce_min_sync(0xffffffffu, kmn);
+              kmx = __reduce_max_sync(0xffffffffu, kmx);
+              const float vmin = key_score(kmn), vmax = key_score(kmx);
+              const float lsc = __fdiv_rn(256.f, __fsub_rn(vmax, vmin));
+              const float lof = __fadd_rn(__fmul_rn(-vmin, lsc), kMagic);
+              if (kmn < kmx && isfinite(vmin) && isfinite(vmax) && isfinite(lsc) && lsc > 0.f && isfinite(lof)) {
+                for (int b = lane; b < 256; b += 32) rh[b] = 0u;
+                __syncwarp();
+                for (int e = lane; e < n; e += 32)
+                  red_shared_add_nb(smem_u32(&rh[value_bin<256>(key_score(lk[e]), lsc, lof)]), 1u);
+                __syncwarp();
+                int above;
+                const int bb = warp_rank_bin<256>(rh, need, lane, &above);
+                const int cntb = static_cast<int>(rh[bb]);
+                const int r2 = need - above;   // keys of bin bb to take
+                __syncwarp();
+                if (cntb <= 64) {
+                  // bin bb's keys and slots to rh[0..63] and rh[64..127]
+                  int base = 0;
+                  for (int e0 = 0; e0 < n; e0 += 32) {
+                    const int e = e0 + lane;
+                    const uint32_t key = e < n ? lk[e] : 0u;
+                    const int bin = e < n ? value_bin<256>(key_score(key), lsc, lof) : -1;
+                    const unsigned m = __ballot_sync(0xffffffffu, bin == bb);
+                    if (bin == bb) {
+                      const int at = base + __popc(m & ltmask);
+                      rh[at] = key;
+                      rh[64 + at] = ls[e];
+                    }
+                    if (bin > bb) red_shared_or_nb(smem_u32(&mb[ls[e] >> 5]), 1u << (ls[e] & 31));
+                    base += __popc(m);
+                  }
+                  __syncwarp();
+                  // a key is taken when fewer than r2 keys of the bin beat it
+                  // (larger, or equal with a lower slot)
+                  for (int x = lane; x < cntb; x += 32) {
+                    const uint32_t kx = rh[x], sx = rh[64 + x];
+                    int beat = 0;
+                    for (int y = 0; y < cntb; ++y) {
+                      const uint32_t ky = rh[y], sy = rh[64 + y];
+                      beat += (ky > kx || (ky == kx && sy < sx)) ? 1 : 0;
+                    }
+                    if (beat < r2) red_shared_or_nb(smem_u32(&mb[sx >> 5]), 1u << (sx & 31));
+                  }
+                  __syncwarp();
+                  ranked = true;
+                }
+              }
+            }
+            if (need < n && !ranked) {
+              // many keys in one bin (ties, or a crowded bin): radix select on
+              // the order keys from the highest bit that varies
               const uint32_t k0 = lk[0];
               uint32_t diff = 0u;
               for (int e = lane; e < n; e += 32) diff |= lk[e] ^ k0;
@@ -740,7 +805,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               }
               need_eq = whole ? 0x7FFFFFFF : rank;   // else: equal keys, the first `rank` in slot order
             }
-            for (int e = lane; e < n; e += 32) {
+            for (int e = lane; e < n && !ranked; e += 32) {
               const uint32_t mk = lk[e] & tmask;
               bool take = mk > tk;
               if (!take && mk == tk) {
@@ -862,38 +927,56 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 
 constexpr int kExpNT = 256;
 
-// Index rows from the selection bitmaps: one warp per output row walks the
-// row's 128 bitmap words in candidate order; each word gives one coalesced
-// store of its selected key indices (the candidates of the row's group,
-// ascending); the row is padded with -1 after its popcount.
+// Index rows from the selection bitmaps.  One warp per unit (group, head)
+// writes its members' rows one after the other, so the unit's candidate row
+// is read from L1 after the first member.  A row's 128 bitmap words are loaded
+// at once (four a lane) with their prefix counts; then each word gives one
+// coalesced store of its selected key indices (the candidates loaded eight
+// words ahead); the row is padded with -1 after its popcount.
 __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, long long nrows) {
+  (void)nrows;
   const int lane = threadIdx.x & 31;
   const uint32_t ltmask = (1u << lane) - 1u;
   const long long nwarps = static_cast<long long>(gridDim.x) * (kExpNT / 32);
   const int CWd = cand_row_words(p.Kc);
-  for (long long row = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; row < nrows; row += nwarps) {
-    const int h = static_cast<int>(row % p.H);
-    const long long qr = row / p.H;   // prefill: the position; decode: b * g + i
-    const int u = static_cast<int>(qr / p.g);
-    const int32_t* crow = p.cand + (static_cast<long long>(h) * p.G + u) * CWd;
-    const uint32_t* srow = p.sel + row * 128;
-    int32_t* orow = p.out + row * p.top_k;
-    const int nw = min(128, CWd / 32);
-    int base = 0;
-#pragma unroll 1
-    for (int w = 0; w < nw; w += 4) {
-      const uint4 wd = *reinterpret_cast<const uint4*>(srow + w);   // the same 16 bytes for every lane
-      const uint32_t ws[4] = {wd.x, wd.y, wd.z, wd.w};
-      int32_t val[4];
+  const int nw = min(128, CWd / 32);
+  const long long units = static_cast<long long>(p.H) * p.G;
+  for (long long ui = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; ui < units; ui += nwarps) {
+    const int h = static_cast<int>(ui / p.G), u = static_cast<int>(ui % p.G);
+    const int32_t* crow = p.cand + ui * CWd;
+    const int nm = p.cu ? p.g : min(u * p.g + p.g, p.L) - u * p.g;
+    for (int i = 0; i < nm; ++i) {
+      const long long row = (static_cast<long long>(u) * p.g + i) * p.H + h;
+      const uint32_t* srow = p.sel + row * 128;
+      int32_t* orow = p.out + row * p.top_k;
+      const uint4 w4 = reinterpret_cast<const uint4*>(srow)[lane];
+      const uint32_t wl[4] = {w4.x, w4.y, w4.z, w4.w};
+      const int own = __popc(wl[0]) + __popc(wl[1]) + __popc(wl[2]) + __popc(wl[3]);
+      int incl = own;
 #pragma unroll
-      for (int x = 0; x < 4; ++x) val[x] = ws[x] ? crow[(w + x) * 32 + lane] : 0;
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        if ((ws[x] >> lane) & 1u) orow[base + __popc(ws[x] & ltmask)] = val[x];
-        base += __popc(ws[x]);
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
+      int pre[4];
+      pre[0] = incl - own;
+#pragma unroll
+      for (int x = 1; x < 4; ++x) pre[x] = pre[x - 1] + __popc(wl[x - 1]);
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll 1
+      for (int w0 = 0; w0 < nw; w0 += 8) {
+        int32_t val[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) val[x] = w0 + x < nw ? crow[(w0 + x) * 32 + lane] : 0;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const uint32_t word = __shfl_sync(0xffffffffu, wl[x & 3], (w0 + x) >> 2);
+          const int bw = __shfl_sync(0xffffffffu, pre[x & 3], (w0 + x) >> 2);
+          if ((word >> lane) & 1u) orow[bw + __popc(word & ltmask)] = val[x];
+        }
+      }
+      for (int t = total + lane; t < p.top_k; t += 32) orow[t] = -1;
     }
-    for (int t = base + lane; t < p.top_k; t += 32) orow[t] = -1;
   }
 }
 
