@@ -930,16 +930,20 @@ constexpr int kExpNT = 256;
 // Index rows from the selection bitmaps.  One warp per unit (group, head)
 // writes its members' rows one after the other, so the unit's candidate row
 // is read from L1 after the first member.  A row's 128 bitmap words are loaded
-// at once (four a lane) with their prefix counts; then each word gives one
-// coalesced store of its selected key indices (the candidates loaded eight
-// words ahead); the row is padded with -1 after its popcount.
+// at once (four a lane) with their prefix counts; each word's selected key
+// indices (the candidates of the row's group, ascending) go to the warp's
+// staging row in shared memory, and the row, padded with -1, leaves in 16-byte
+// stores.  Dynamic shared memory: kExpNT / 32 rows of top_k words.
 __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, long long nrows) {
   (void)nrows;
-  const int lane = threadIdx.x & 31;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const uint32_t ltmask = (1u << lane) - 1u;
+  int32_t* stg = reinterpret_cast<int32_t*>(smem_raw) + wib * p.top_k;
   const long long nwarps = static_cast<long long>(gridDim.x) * (kExpNT / 32);
   const int CWd = cand_row_words(p.Kc);
   const int nw = min(128, CWd / 32);
+  const bool vec = (p.top_k & 3) == 0;   // rows are 16-byte aligned
   const long long units = static_cast<long long>(p.H) * p.G;
   for (long long ui = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; ui < units; ui += nwarps) {
     const int h = static_cast<int>(ui / p.G), u = static_cast<int>(ui % p.G);
@@ -962,7 +966,7 @@ __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, l
       pre[0] = incl - own;
 #pragma unroll
       for (int x = 1; x < 4; ++x) pre[x] = pre[x - 1] + __popc(wl[x - 1]);
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
 #pragma unroll 1
       for (int w0 = 0; w0 < nw; w0 += 8) {
         int32_t val[8];
@@ -972,10 +976,19 @@ __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, l
         for (int x = 0; x < 8; ++x) {
           const uint32_t word = __shfl_sync(0xffffffffu, wl[x & 3], (w0 + x) >> 2);
           const int bw = __shfl_sync(0xffffffffu, pre[x & 3], (w0 + x) >> 2);
-          if ((word >> lane) & 1u) orow[bw + __popc(word & ltmask)] = val[x];
+          const int at = bw + __popc(word & ltmask);
+          if (((word >> lane) & 1u) && at < p.top_k) stg[at] = val[x];
         }
       }
-      for (int t = total + lane; t < p.top_k; t += 32) orow[t] = -1;
+      for (int t = total + lane; t < p.top_k; t += 32) stg[t] = -1;
+      __syncwarp();
+      if (vec) {
+        for (int t = 4 * lane; t < p.top_k; t += 128)
+          *reinterpret_cast<int4*>(orow + t) = *reinterpret_cast<const int4*>(stg + t);
+      } else {
+        for (int t = lane; t < p.top_k; t += 32) orow[t] = stg[t];
+      }
+      __syncwarp();
     }
   }
 }
