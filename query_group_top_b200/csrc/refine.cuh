@@ -129,7 +129,8 @@ struct RefineCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = NS * STAGE;              // two B buffers (item parity)
   static constexpr int OFF_C = OFF_B + 2 * B_BYTES;     // two candidate lists
-  // selection bitmaps: one bit per candidate slot
+  // selection bitmaps: one bit per candidate slot, word w of member m at
+  // word 16w + m (the 16 members' words of a 32-candidate slice are adjacent)
   static constexpr int BMP_BYTES = 16 * 128 * 4;
   // per member 256 32-bit words: the list's radix histogram, and with the
   // scores written out the selection's per-word prefix counts
@@ -668,7 +669,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           my_n = lane == j ? static_cast<uint32_t>(__popc(lm[j])) : my_n;
         }
         // lane j < 16: member j's bitmap word and list reservation
-        if (lane < 16) bmp[lane * 128 + c * 4 + q] = my_above;
+        if (lane < 16) bmp[(c * 4 + q) * 16 + lane] = my_above;
         uint32_t base = 0u;
         if (lane < 16 && my_n != 0u) base = atom_shared_add(smem_u32(&M->ms[lane].nlist), my_n);
         // every member's slots at once: no branch keeps one member's shuffle
@@ -676,8 +677,10 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         const uint16_t slot = static_cast<uint16_t>(base_t + lane);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const uint32_t at = __shfl_sync(0xffffffffu, base, j) + static_cast<uint32_t>(__popc(lm[j] & ltmask));
-          if (((lm[j] >> lane) & 1u) && at < static_cast<uint32_t>(kCap)) {
+          // (a list that overflows is a miss; its last slot just takes the rest)
+          const uint32_t at = min(__shfl_sync(0xffffffffu, base, j) + static_cast<uint32_t>(__popc(lm[j] & ltmask)),
+                                  static_cast<uint32_t>(kCap - 1));
+          if ((lm[j] >> lane) & 1u) {
             st_shared_u32_nb(lk_s + 4u * (j * kCap + at), v[j]);
             st_shared_u16_nb(ls_s + 2u * (j * kCap + at), slot);
           }
@@ -688,14 +691,14 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       // ---- warp sw ranks member sw's list exactly: the need-th largest key
       //      (radix select from the highest bit that varies) and how many of
       //      its copies are taken; decisions OR-ed into the member's bitmap
-      uint32_t* mb = bmp + sw * 128;
+      uint32_t* mb = bmp + sw;   // member sw's word w is mb[16 * w]
       if (sw < nb) {
         MemberSel& S = M->ms[sw];
         int mode = S.mode;
         if (mode == kMList || mode == kMBand) {
           int nabove = 0;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) nabove += __popc(mb[lane + 32 * w]);
+          for (int w = 0; w < 4; ++w) nabove += __popc(mb[16 * (lane + 32 * w)]);
           nabove = __reduce_add_sync(0xffffffffu, nabove);
           const int n = S.nlist, need = S.K - nabove;
           if (n > kCap || need < 1 || need > n) {
@@ -747,7 +750,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
                       rh[at] = key;
                       rh[64 + at] = ls[e];
                     }
-                    if (bin > bb) red_shared_or_nb(smem_u32(&mb[ls[e] >> 5]), 1u << (ls[e] & 31));
+                    if (bin > bb) red_shared_or_nb(smem_u32(&mb[16 * (ls[e] >> 5)]), 1u << (ls[e] & 31));
                     base += __popc(m);
                   }
                   __syncwarp();
@@ -760,7 +763,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
                       const uint32_t ky = rh[y], sy = rh[64 + y];
                       beat += (ky > kx || (ky == kx && sy < sx)) ? 1 : 0;
                     }
-                    if (beat < r2) red_shared_or_nb(smem_u32(&mb[sx >> 5]), 1u << (sx & 31));
+                    if (beat < r2) red_shared_or_nb(smem_u32(&mb[16 * (sx >> 5)]), 1u << (sx & 31));
                   }
                   __syncwarp();
                   ranked = true;
@@ -819,7 +822,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               }
               if (take) {
                 const int t = ls[e];
-                red_shared_or_nb(smem_u32(&mb[t >> 5]), 1u << (t & 31));
+                red_shared_or_nb(smem_u32(&mb[16 * (t >> 5)]), 1u << (t & 31));
               }
             }
           }
@@ -846,7 +849,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             const int u = K - 32 * w;
             wds[x] = u >= 32 ? 0xFFFFFFFFu : (u <= 0 ? 0u : ((1u << u) - 1u));
           } else if (mode == kMList || mode == kMBand) {
-            wds[x] = mb[w];
+            wds[x] = mb[16 * w];
           } else {
             wds[x] = 0u;
           }
@@ -891,7 +894,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               if (mode == kMAll) {
                 if (t < M->ms[j].K) srow[t] = __uint_as_float(v[j]);
               } else if (mode == kMList || mode == kMBand) {
-                const uint32_t word = bmp[j * 128 + c * 4 + q];
+                const uint32_t word = bmp[(c * 4 + q) * 16 + j];
                 if ((word >> lane) & 1u)
                   srow[hist[j * 256 + c * 4 + q] + __popc(word & ltmask)] = __uint_as_float(v[j]);
               }
@@ -926,6 +929,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 }
 
 constexpr int kExpNT = 256;
+// Per-warp shared memory of refine_expand_kernel, in 8-byte units: 128
+// (word, prefix) pairs and a staging row of top_k words rounded up to 16 bytes.
+__host__ __device__ inline int expand_warp_u2(int top_k) { return 128 + 2 * ((top_k + 3) / 4); }
 
 // Index rows from the selection bitmaps.  One warp per unit (group, head)
 // writes its members' rows one after the other, so the unit's candidate row
@@ -939,7 +945,10 @@ __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, l
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const uint32_t ltmask = (1u << lane) - 1u;
-  int32_t* stg = reinterpret_cast<int32_t*>(smem_raw) + wib * p.top_k;
+  // per warp: the row's (word, prefix) pairs, then its staging row (a
+  // multiple of 16 bytes, so that every warp's row stays 16-byte aligned)
+  uint2* wp = reinterpret_cast<uint2*>(smem_raw) + wib * expand_warp_u2(p.top_k);
+  int32_t* stg = reinterpret_cast<int32_t*>(wp + 128);
   const long long nwarps = static_cast<long long>(gridDim.x) * (kExpNT / 32);
   const int CWd = cand_row_words(p.Kc);
   const int nw = min(128, CWd / 32);
@@ -962,11 +971,16 @@ __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, l
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      int pre[4];
-      pre[0] = incl - own;
+      {
+        uint32_t pre = static_cast<uint32_t>(incl - own);
 #pragma unroll
-      for (int x = 1; x < 4; ++x) pre[x] = pre[x - 1] + __popc(wl[x - 1]);
+        for (int x = 0; x < 4; ++x) {
+          wp[4 * lane + x] = make_uint2(wl[x], pre);
+          pre += __popc(wl[x]);
+        }
+      }
       const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
+      __syncwarp();
 #pragma unroll 1
       for (int w0 = 0; w0 < nw; w0 += 8) {
         int32_t val[8];
@@ -974,10 +988,10 @@ __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, l
         for (int x = 0; x < 8; ++x) val[x] = w0 + x < nw ? crow[(w0 + x) * 32 + lane] : 0;
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          const uint32_t word = __shfl_sync(0xffffffffu, wl[x & 3], (w0 + x) >> 2);
-          const int bw = __shfl_sync(0xffffffffu, pre[x & 3], (w0 + x) >> 2);
-          const int at = bw + __popc(word & ltmask);
-          if (((word >> lane) & 1u) && at < p.top_k) stg[at] = val[x];
+          if (w0 + x < nw) {
+            const uint2 e = wp[w0 + x];   // the same 8 bytes for every lane
+            if ((e.x >> lane) & 1u) stg[e.y + __popc(e.x & ltmask)] = val[x];
+          }
         }
       }
       for (int t = total + lane; t < p.top_k; t += 32) stg[t] = -1;
