@@ -28,31 +28,30 @@
 // MMA warp can write the next unit into them while this unit is still being
 // selected.
 //
-// Selection (exact, on 32-bit order keys, ties to the lower index), in one
-// pass over the scores.  Select warp w = 4s + q reads TMEM lane quarter q of
-// the chunks at scoring positions s, s+4, s+8, ... (all 16 members of 32
-// candidates per load) and later ranks member w's list and writes member w's
-// rows:
-//  * a member with at most kCap usable candidates sends all of them to its
-//    boundary list;
-//  * otherwise the first kSample chunks give an interval [lo, hi) that holds
-//    the member's k-th score with overwhelming probability: a histogram
-//    linear in the score over chunk 0's range, and sample ranks kZ standard
-//    deviations on either side of the expected one;
+// Selection (exact, on 32-bit order keys, ties to the lower index).  Select
+// warp w = 4s + q reads TMEM lane quarter q of the chunks at scoring positions
+// s, s+4, s+8, ... (all 16 members of 32 candidates per load) and later ranks
+// member w's list and writes member w's bitmap:
+//  * chunk 0's score range sets, per member, kBins bins linear in the score;
+//    every usable score is counted into its member's histogram as soon as its
+//    chunk's MMAs finish, so the counting overlaps the gather;
+//  * the bin holding the member's k-th largest score is found exactly: keys
+//    in higher bins are taken, the bin's own keys (a few on real scores) form
+//    the member's list;
 //  * one pass over all chunks classifies 32 candidates of a member with two
 //    warp votes: the ">= hi" mask goes straight into the member's selection
-//    bitmap (bit t = candidate t), the "[lo, hi)" lanes append their scores
+//    bitmap (bit t = candidate t), the boundary-bin lanes append their scores
 //    to the member's list; each chunk's TMEM columns are given back as soon
-//    as they are loaded;
-//  * the list is ranked exactly (a warp radix select: the need-th largest key
-//    and how many of its copies are taken, ties in candidate order), and its
-//    decisions are OR-ed into the bitmap;
+//    as they are loaded, so the next unit's MMAs follow this pass closely;
+//  * the list is ranked exactly (pairwise when short, else by value bins or
+//    a radix select; ties in candidate order) and its decisions are OR-ed into
+//    the bitmap;
 //  * the member's warp writes the bitmap out (512 bytes); refine_expand_kernel
 //    turns every bitmap into its index row afterwards, so the row writes
 //    (4 bytes per index) do not take issue slots from this kernel.
-// A member whose k-th score fell outside its interval, whose list overflowed,
-// or whose sample had no score range is not written here: it is recorded in a
-// miss list and refine_fallback_kernel redoes it exactly afterwards.
+// A member whose chunk-0 range is empty, or whose boundary bin holds more than
+// kCap keys (ties), is not written here: it is recorded in a miss list and
+// refine_fallback_kernel redoes it exactly afterwards.
 #pragma once
 
 #include "ptx.cuh"
@@ -83,8 +82,7 @@ struct RefineParams {
 enum : int {
   kMNone = 0,   // takes nothing (no usable candidate)
   kMAll = 1,    // takes every usable candidate (top_k >= usable count)
-  kMList = 2,   // few usable candidates: all of them go to the list
-  kMBand = 3,   // sampled interval: >= hi taken, [lo, hi) to the list
+  kMBand = 3,   // a selection: >= hi taken, the boundary bin [lo, hi) ranked
   kMMiss = 4,   // redone by refine_fallback_kernel
 };
 
@@ -92,8 +90,6 @@ constexpr int kBins = 1024;         // sample histogram bins per member
 // 2^23: a float in [2^23, 2^24) is an integer, held in its low mantissa bits
 constexpr float kMagic = 8388608.0f;
 constexpr int kCap = 512;           // boundary list entries per member
-constexpr int kSample = 16;         // sampled chunks
-constexpr float kZ = 4.0f;          // interval half-width, in standard deviations of the sample rank
 
 struct MemberSel {
   int nv;           // usable candidates: the ascending prefix with j < pos
@@ -103,6 +99,7 @@ struct MemberSel {
   float lo, hi;     // list interval [lo, hi); hi = +inf: no "above" region
   float scale, offm;    // sample histogram bins: value_bin(s, scale, offm)
   uint32_t kmin, kmax;  // chunk 0's usable score range as order keys
+  int need;             // keys of the list (the boundary bin) to take
 };
 
 struct RefineMisc {
@@ -504,29 +501,29 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         const int K = min(p.top_k, nv);
         S.nv = nv;
         S.K = K;
-        S.mode = K == 0 ? kMNone : (K == nv ? kMAll : (nv <= kCap ? kMList : kMBand));
+        S.mode = K == 0 ? kMNone : (K == nv ? kMAll : kMBand);
         S.nlist = 0;
-        S.lo = S.mode == kMList ? -kInf : kInf;   // None/All take no list; Band is set below
+        S.need = 0;
+        S.lo = kInf;   // None and All take no list; Band is set below
         S.hi = kInf;
         S.kmin = 0xFFFFFFFFu;
         S.kmax = 0u;
       }
-      // bitmaps and sample histograms start at zero
+      // bitmaps and histograms start at zero
       for (int i = stid; i < (C::BMP_BYTES + 16 * kBins * 4) / 16; i += C::NSEL)
         reinterpret_cast<uint4*>(bmp)[i] = make_uint4(0, 0, 0, 0);
       if (named_barrier_or(2, C::NSEL, !ok)) break;
-      bool anyb = false;     // a member with a sampled interval (uniform)
-      int nvmin = 0x7FFFFFFF;  // fewest usable candidates of a classified member (uniform)
+      bool anyb = false;       // a member that needs a selection (uniform)
+      int nvmin = 0x7FFFFFFF;  // fewest usable candidates of such a member (uniform)
       for (int m = 0; m < 16; ++m) {
-        const int md = M->ms[m].mode;
-        anyb |= md == kMBand;
-        if (md == kMList || md == kMBand) nvmin = min(nvmin, M->ms[m].nv);
+        if (M->ms[m].mode == kMBand) {
+          anyb = true;
+          nvmin = min(nvmin, M->ms[m].nv);
+        }
       }
-      const int s_ch = min(nch, kSample);
 
-      // ---- sample: chunk 0's score range, then a histogram of the first s_ch
-      //      chunks scored; then warp w derives member w's interval
       if (anyb) {
+        // ---- chunk 0's score range sets each member's histogram bins
         if (st == 0) {
           if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status);
           ok = __all_sync(0xffffffffu, ok);
@@ -553,8 +550,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           }
         }
         if (named_barrier_or(2, C::NSEL, !ok)) break;
-        // bins linear in the score over chunk 0's range; a member whose range
-        // is empty or not finite goes to the exact fallback
+        // bins linear in the score over chunk 0's range (scores outside it
+        // clamp to the end bins); a member whose range is empty or not finite
+        // goes to the exact fallback
         if (lane == 0 && M->ms[sw].mode == kMBand) {
           MemberSel& S = M->ms[sw];
           const float vmin = key_score(S.kmin), vmax = key_score(S.kmax);
@@ -567,7 +565,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           if (!good) S.mode = kMMiss;
         }
         sel_sync();
-        for (int i = st; i < s_ch; i += 4) {
+        // ---- the histogram of every usable score, chunk by chunk as the MMAs
+        //      finish (the columns stay in TMEM for the pass below)
+        for (int i = st; i < nch; i += 4) {
           const int c = chunk_at(i, nch);
           if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
           ok = __all_sync(0xffffffffu, ok);
@@ -586,36 +586,23 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           }
         }
         if (named_barrier_or(2, C::NSEL, !ok)) break;
-        // member sw's interval: sample ranks kZ standard deviations either side
-        // of the expected rank of the k-th score (hypergeometric: the sample
-        // is drawn without replacement)
+        // ---- warp sw: member sw's boundary bin, the one that holds its k-th
+        //      largest score: keys in higher bins are taken, the bin's own keys
+        //      (its list) are ranked exactly
         if (sw < nb && M->ms[sw].mode == kMBand) {
           MemberSel& S = M->ms[sw];
           const uint32_t* hm = shist + sw * kBins;
-          // the usable candidates among the sampled chunks
-          int n_s = 0;
-          for (int i = 0; i < s_ch; ++i) n_s += min(max(S.nv - 128 * chunk_at(i, nch), 0), 128);
-          const float pk = static_cast<float>(S.K) / static_cast<float>(S.nv);
-          const float e = pk * static_cast<float>(n_s);
-          const float fpc = fmaxf(0.f, 1.f - static_cast<float>(n_s) / static_cast<float>(S.nv));
-          const float dlt = kZ * sqrtf(static_cast<float>(n_s) * pk * (1.f - pk) * fpc) + 2.f;
-          const int r_hi = static_cast<int>(floorf(e - dlt));
-          const int r_lo = static_cast<int>(ceilf(e + dlt));
+          int above;
+          const int b = warp_rank_bin<kBins>(hm, S.K, lane, &above);
+          const int cnt = static_cast<int>(hm[b]);
           float hi = kInf, lo = -kInf;
-          int ab;
-          if (r_hi >= 1) {
-            // above = the bins over the one holding the r_hi-th largest sample
-            const int b = warp_rank_bin<kBins>(hm, r_hi, lane, &ab);
-            if (b < kBins - 1) hi = key_score(warp_first_key_of_bin(b + 1, S.scale, S.offm, lane));
-          }
-          if (r_lo <= n_s) {
-            // list = down to the bin holding the r_lo-th largest sample
-            const int b = warp_rank_bin<kBins>(hm, r_lo, lane, &ab);
-            if (b > 0) lo = key_score(warp_first_key_of_bin(b, S.scale, S.offm, lane));
-          }
+          if (b < kBins - 1) hi = key_score(warp_first_key_of_bin(b + 1, S.scale, S.offm, lane));
+          if (b > 0) lo = key_score(warp_first_key_of_bin(b, S.scale, S.offm, lane));
           if (lane == 0) {
+            S.need = S.K - above;
             S.lo = lo;
             S.hi = hi;
+            if (cnt > kCap) S.mode = kMMiss;   // a bin crowded by ties: the exact fallback
           }
           __syncwarp();
         }
@@ -623,7 +610,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       }
 
       // ---- one pass: per chunk, each member's ">= hi" lanes into its bitmap
-      //      and its "[lo, hi)" lanes onto its list; the chunk's TMEM columns
+      //      and its boundary-bin lanes onto its list; the chunk's TMEM columns
       //      go back as soon as they are loaded (unless the scores are
       //      written out, which reads them again)
       const bool keep_tmem = p.out_scores != nullptr;
@@ -632,16 +619,20 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const MemberSel& S = M->ms[j];
-        const bool cls = S.mode == kMList || S.mode == kMBand;
+        const bool cls = S.mode == kMBand;
         th[j] = cls ? S.hi : kInf;
         tl[j] = cls ? S.lo : kInf;
       }
 #pragma unroll 1
       for (int i = st; i < nch; i += 4) {
         const int c = chunk_at(i, nch);
-        if (ok && (i >= s_ch || !anyb)) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
+        if (ok && !anyb) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
+        if (!anyb) {   // nothing to classify
+          if (!keep_tmem) release(c);
+          continue;
+        }
         tc_fence_after();
         uint32_t v[16];
         tmem_ld_32x32b_x16(tq + 16 * c, v);
@@ -670,19 +661,20 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         }
         // lane j < 16: member j's bitmap word and list reservation
         if (lane < 16) bmp[(c * 4 + q) * 16 + lane] = my_above;
-        uint32_t base = 0u;
-        if (lane < 16 && my_n != 0u) base = atom_shared_add(smem_u32(&M->ms[lane].nlist), my_n);
-        // every member's slots at once: no branch keeps one member's shuffle
-        // and stores from overlapping the next member's
-        const uint16_t slot = static_cast<uint16_t>(base_t + lane);
+        if (__any_sync(0xffffffffu, my_n != 0u)) {
+          uint32_t base = 0u;
+          if (lane < 16 && my_n != 0u) base = atom_shared_add(smem_u32(&M->ms[lane].nlist), my_n);
+          const uint16_t slot = static_cast<uint16_t>(base_t + lane);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          // (a list that overflows is a miss; its last slot just takes the rest)
-          const uint32_t at = min(__shfl_sync(0xffffffffu, base, j) + static_cast<uint32_t>(__popc(lm[j] & ltmask)),
-                                  static_cast<uint32_t>(kCap - 1));
-          if ((lm[j] >> lane) & 1u) {
-            st_shared_u32_nb(lk_s + 4u * (j * kCap + at), v[j]);
-            st_shared_u16_nb(ls_s + 2u * (j * kCap + at), slot);
+          for (int j = 0; j < 16; ++j) {
+            if (lm[j] != 0u) {   // the same for every lane: boundary keys are few
+              const uint32_t at = min(__shfl_sync(0xffffffffu, base, j) + static_cast<uint32_t>(__popc(lm[j] & ltmask)),
+                                      static_cast<uint32_t>(kCap - 1));
+              if ((lm[j] >> lane) & 1u) {
+                st_shared_u32_nb(lk_s + 4u * (j * kCap + at), v[j]);
+                st_shared_u16_nb(ls_s + 2u * (j * kCap + at), slot);
+              }
+            }
           }
         }
       }
@@ -695,14 +687,10 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       if (sw < nb) {
         MemberSel& S = M->ms[sw];
         int mode = S.mode;
-        if (mode == kMList || mode == kMBand) {
-          int nabove = 0;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) nabove += __popc(mb[16 * (lane + 32 * w)]);
-          nabove = __reduce_add_sync(0xffffffffu, nabove);
-          const int n = S.nlist, need = S.K - nabove;
+        if (mode == kMBand) {
+          const int n = S.nlist, need = S.need;
           if (n > kCap || need < 1 || need > n) {
-            mode = kMMiss;   // the k-th score fell outside the interval, or the list overflowed
+            mode = kMMiss;   // (cannot happen: the list is the boundary bin)
           } else {
             uint32_t* lk = lkeys + sw * kCap;
             const uint16_t* ls = lslot + sw * kCap;
@@ -712,7 +700,22 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             uint32_t tk = 0u, tmask = 0u;
             int need_eq = 0x7FFFFFFF;   // the whole list, when need == n
             bool ranked = false;        // decisions already in the bitmap
-            if (need < n) {
+            if (need < n && n <= 64) {
+              // a short list: a key is taken when fewer than `need` keys beat
+              // it (larger, or equal with a lower slot)
+              for (int x = lane; x < n; x += 32) {
+                const uint32_t kx = lk[x], sx = ls[x];
+                int beat = 0;
+                for (int y = 0; y < n; ++y) {
+                  const uint32_t ky = lk[y], sy = ls[y];
+                  beat += (ky > kx || (ky == kx && sy < sx)) ? 1 : 0;
+                }
+                if (beat < need) red_shared_or_nb(smem_u32(&mb[16 * (sx >> 5)]), 1u << (sx & 31));
+              }
+              __syncwarp();
+              ranked = true;
+            }
+            if (need < n && !ranked) {
               // bins linear in the score over the list's own range spread its
               // keys evenly; the need-th largest lies in bin b, and the few
               // keys of bin b are ranked exactly against each other
@@ -848,7 +851,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           if (mode == kMAll) {
             const int u = K - 32 * w;
             wds[x] = u >= 32 ? 0xFFFFFFFFu : (u <= 0 ? 0u : ((1u << u) - 1u));
-          } else if (mode == kMList || mode == kMBand) {
+          } else if (mode == kMBand) {
             wds[x] = mb[16 * w];
           } else {
             wds[x] = 0u;
@@ -893,7 +896,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
               float* srow = p.out_scores + ((it.qrow0 + it.mb + j) * p.H + it.h) * static_cast<long long>(p.top_k);
               if (mode == kMAll) {
                 if (t < M->ms[j].K) srow[t] = __uint_as_float(v[j]);
-              } else if (mode == kMList || mode == kMBand) {
+              } else if (mode == kMBand) {
                 const uint32_t word = bmp[(c * 4 + q) * 16 + j];
                 if ((word >> lane) & 1u)
                   srow[hist[j * 256 + c * 4 + q] + __popc(word & ltmask)] = __uint_as_float(v[j]);
