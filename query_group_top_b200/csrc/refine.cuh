@@ -566,7 +566,17 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         }
         sel_sync();
         // ---- the histogram of every usable score, chunk by chunk as the MMAs
-        //      finish (the columns stay in TMEM for the pass below)
+        //      finish (the columns stay in TMEM for the pass below).  A member
+        //      without a selection counts into its own, unused, histogram,
+        //      which keeps the loop free of branches
+        float sc4[16], of4[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const bool band = M->ms[j].mode == kMBand;
+          sc4[j] = band ? M->ms[j].scale : 0.f;
+          of4[j] = band ? M->ms[j].offm : kMagic;
+        }
+        const uint32_t sh0 = smem_u32(shist);
         for (int i = st; i < nch; i += 4) {
           const int c = chunk_at(i, nch);
           if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
@@ -577,12 +587,19 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           tmem_ld_32x32b_x16(tq + 16 * c, v);
           tmem_ld_wait();
           const int t = c * 128 + q * 32 + lane;
+          if (c * 128 + q * 32 + 32 <= nvmin) {   // every member can use every lane
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            reg_fence(v[j]);
-            const MemberSel& S = M->ms[j];
-            if (S.mode == kMBand && t < S.nv)
-              red_shared_add_nb(smem_u32(shist + j * kBins + value_bin(__uint_as_float(v[j]), S.scale, S.offm)), 1u);
+            for (int j = 0; j < 16; ++j) {
+              reg_fence(v[j]);
+              red_shared_add_nb(sh0 + 4u * (j * kBins + value_bin(__uint_as_float(v[j]), sc4[j], of4[j])), 1u);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              reg_fence(v[j]);
+              if (t < M->ms[j].nv)
+                red_shared_add_nb(sh0 + 4u * (j * kBins + value_bin(__uint_as_float(v[j]), sc4[j], of4[j])), 1u);
+            }
           }
         }
         if (named_barrier_or(2, C::NSEL, !ok)) break;
