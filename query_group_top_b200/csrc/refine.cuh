@@ -949,81 +949,59 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 }
 
 constexpr int kExpNT = 256;
-// Per-warp shared memory of refine_expand_kernel, in 8-byte units: 128
-// (word, prefix) pairs and a staging row of top_k words rounded up to 16 bytes.
-__host__ __device__ inline int expand_warp_u2(int top_k) { return 128 + 2 * ((top_k + 3) / 4); }
 
-// Index rows from the selection bitmaps.  One warp per unit (group, head)
-// writes its members' rows one after the other, so the unit's candidate row
-// is read from L1 after the first member.  A row's 128 bitmap words are loaded
-// at once (four a lane) with their prefix counts; each word's selected key
-// indices (the candidates of the row's group, ascending) go to the warp's
-// staging row in shared memory, and the row, padded with -1, leaves in 16-byte
-// stores.  Dynamic shared memory: kExpNT / 32 rows of top_k words.
+// Index rows from the selection bitmaps, one warp per output row.  Rows are
+// numbered member-fastest within a unit (group, head), so the members of a
+// unit run in neighbouring warps of a block and share its candidate row
+// through L1.  A row's 128 bitmap words are loaded at once (four a lane) with
+// their prefix counts; each word then gives one coalesced store of its
+// selected key indices (the candidates of the row's group, ascending), and
+// the row is padded with -1 after its popcount.
 __global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, long long nrows) {
   (void)nrows;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const uint32_t ltmask = (1u << lane) - 1u;
-  // per warp: the row's (word, prefix) pairs, then its staging row (a
-  // multiple of 16 bytes, so that every warp's row stays 16-byte aligned)
-  uint2* wp = reinterpret_cast<uint2*>(smem_raw) + wib * expand_warp_u2(p.top_k);
-  int32_t* stg = reinterpret_cast<int32_t*>(wp + 128);
   const long long nwarps = static_cast<long long>(gridDim.x) * (kExpNT / 32);
   const int CWd = cand_row_words(p.Kc);
-  const int nw = min(128, CWd / 32);
-  const bool vec = (p.top_k & 3) == 0;   // rows are 16-byte aligned
-  const long long units = static_cast<long long>(p.H) * p.G;
-  for (long long ui = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; ui < units; ui += nwarps) {
+  const int nw = min(128, CWd / 32);   // a multiple of 4
+  const long long slots = static_cast<long long>(p.H) * p.G * p.g;
+  for (long long f = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; f < slots; f += nwarps) {
+    const long long ui = f / p.g;
+    const int i = static_cast<int>(f - ui * p.g);
     const int h = static_cast<int>(ui / p.G), u = static_cast<int>(ui % p.G);
-    const int32_t* crow = p.cand + ui * CWd;
     const int nm = p.cu ? p.g : min(u * p.g + p.g, p.L) - u * p.g;
-    for (int i = 0; i < nm; ++i) {
-      const long long row = (static_cast<long long>(u) * p.g + i) * p.H + h;
-      const uint32_t* srow = p.sel + row * 128;
-      int32_t* orow = p.out + row * p.top_k;
-      const uint4 w4 = reinterpret_cast<const uint4*>(srow)[lane];
-      const uint32_t wl[4] = {w4.x, w4.y, w4.z, w4.w};
-      const int own = __popc(wl[0]) + __popc(wl[1]) + __popc(wl[2]) + __popc(wl[3]);
-      int incl = own;
+    if (i >= nm) continue;   // past a partial last group
+    const long long row = (static_cast<long long>(u) * p.g + i) * p.H + h;
+    const int32_t* crow = p.cand + ui * CWd;
+    int32_t* orow = p.out + row * p.top_k;
+    const uint4 w4 = reinterpret_cast<const uint4*>(p.sel + row * 128)[lane];
+    const uint32_t wl[4] = {w4.x, w4.y, w4.z, w4.w};
+    const int own = __popc(wl[0]) + __popc(wl[1]) + __popc(wl[2]) + __popc(wl[3]);
+    int incl = own;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      {
-        uint32_t pre = static_cast<uint32_t>(incl - own);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          wp[4 * lane + x] = make_uint2(wl[x], pre);
-          pre += __popc(wl[x]);
-        }
-      }
-      const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
-      __syncwarp();
-#pragma unroll 1
-      for (int w0 = 0; w0 < nw; w0 += 8) {
-        int32_t val[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) val[x] = w0 + x < nw ? crow[(w0 + x) * 32 + lane] : 0;
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          if (w0 + x < nw) {
-            const uint2 e = wp[w0 + x];   // the same 8 bytes for every lane
-            if ((e.x >> lane) & 1u) stg[e.y + __popc(e.x & ltmask)] = val[x];
-          }
-        }
-      }
-      for (int t = total + lane; t < p.top_k; t += 32) stg[t] = -1;
-      __syncwarp();
-      if (vec) {
-        for (int t = 4 * lane; t < p.top_k; t += 128)
-          *reinterpret_cast<int4*>(orow + t) = *reinterpret_cast<const int4*>(stg + t);
-      } else {
-        for (int t = lane; t < p.top_k; t += 32) orow[t] = stg[t];
-      }
-      __syncwarp();
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    int pre[4];
+    pre[0] = incl - own;
+#pragma unroll
+    for (int x = 1; x < 4; ++x) pre[x] = pre[x - 1] + __popc(wl[x - 1]);
+    const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
+#pragma unroll 2
+    for (int w0 = 0; w0 < nw; w0 += 4) {
+      int32_t val[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) val[x] = crow[(w0 + x) * 32 + lane];
+      const int owner = w0 >> 2;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const uint32_t word = __shfl_sync(0xffffffffu, wl[x], owner);
+        const int bw = __shfl_sync(0xffffffffu, pre[x], owner);
+        if ((word >> lane) & 1u) orow[bw + __popc(word & ltmask)] = val[x];
+      }
+    }
+    for (int t = total + lane; t < p.top_k; t += 32) orow[t] = -1;
   }
 }
 
