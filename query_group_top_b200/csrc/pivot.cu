@@ -282,9 +282,11 @@ int launch_refine(RefineParams rp, int units, long long rows, int sms, uint8_t* 
   CUDA_TRY(cudaGetLastError());
   {
     TraceScope tr("refine_expand", st);
-    const long long slots = static_cast<long long>(units) * rp.g;   // one warp per (unit, member)
-    const long long blocks = std::min<long long>((slots + kExpNT / 32 - 1) / (kExpNT / 32), 64ll * std::max(1, sms));
-    refine_expand_kernel<<<static_cast<unsigned>(std::max<long long>(1, blocks)), kExpNT, 0, st>>>(rp, rows);
+    // one block per unit (group, head), grid-stride
+    const long long blocks = std::min<long long>(units, 16ll * std::max(1, sms));
+    const int esmem = expand_smem_words(rp.Kc, rp.top_k) * 4;
+    CUDA_TRY(cudaFuncSetAttribute(refine_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, esmem));
+    refine_expand_kernel<<<static_cast<unsigned>(std::max<long long>(1, blocks)), kExpNT, esmem, st>>>(rp, rows);
   }
   CUDA_TRY(cudaGetLastError());
   const int fsmem = (2 * cand_row_words(rp.Kc) + 2 * rp.top_k) * 4;

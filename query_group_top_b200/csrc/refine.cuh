@@ -950,58 +950,66 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 
 constexpr int kExpNT = 256;
 
-// Index rows from the selection bitmaps, one warp per output row.  Rows are
-// numbered member-fastest within a unit (group, head), so the members of a
-// unit run in neighbouring warps of a block and share its candidate row
-// through L1.  A row's 128 bitmap words are loaded at once (four a lane) with
-// their prefix counts; each word then gives one coalesced store of its
-// selected key indices (the candidates of the row's group, ascending), and
-// the row is padded with -1 after its popcount.
-__global__ void __launch_bounds__(kExpNT) refine_expand_kernel(RefineParams p, long long nrows) {
+// Index rows from the selection bitmaps.  A block takes a unit (group, head):
+// its candidate row goes to shared memory, and each warp expands one member's
+// row at a time.  Lane l owns candidates 128l .. 128l+127 (bitmap words
+// 4l .. 4l+3): after a warp scan of the words' popcounts it walks its own set
+// bits and writes their key indices to the warp's staging row, which then
+// leaves in coalesced stores, padded with -1.  Both shared arrays are
+// XOR-swizzled within 32-word groups so that the lanes' scattered accesses
+// fall in different banks.  Dynamic shared memory: expand_smem_words(Kc, top_k).
+__host__ __device__ inline int expand_stage_words(int top_k) { return (top_k + 31) / 32 * 32; }
+__host__ __device__ inline int expand_smem_words(int Kc, int top_k) {
+  return cand_row_words(Kc) + (kExpNT / 32) * expand_stage_words(top_k);
+}
+__device__ __forceinline__ int cand_swz(int t) { return t ^ ((t >> 7) & 31); }
+__device__ __forceinline__ int stage_swz(int p) { return p ^ ((p >> 6) & 31); }
+
+__global__ void __launch_bounds__(kExpNT, 2) refine_expand_kernel(RefineParams p, long long nrows) {
   (void)nrows;
-  const int lane = threadIdx.x & 31;
-  const uint32_t ltmask = (1u << lane) - 1u;
-  const long long nwarps = static_cast<long long>(gridDim.x) * (kExpNT / 32);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int CWd = cand_row_words(p.Kc);
-  const int nw = min(128, CWd / 32);   // a multiple of 4
-  const long long slots = static_cast<long long>(p.H) * p.G * p.g;
-  for (long long f = (static_cast<long long>(blockIdx.x) * kExpNT + threadIdx.x) >> 5; f < slots; f += nwarps) {
-    const long long ui = f / p.g;
-    const int i = static_cast<int>(f - ui * p.g);
+  int32_t* cs = reinterpret_cast<int32_t*>(smem_raw);
+  int32_t* stg = cs + CWd + wib * expand_stage_words(p.top_k);
+  const long long units = static_cast<long long>(p.H) * p.G;
+  for (long long ui = blockIdx.x; ui < units; ui += gridDim.x) {
     const int h = static_cast<int>(ui / p.G), u = static_cast<int>(ui % p.G);
     const int nm = p.cu ? p.g : min(u * p.g + p.g, p.L) - u * p.g;
-    if (i >= nm) continue;   // past a partial last group
-    const long long row = (static_cast<long long>(u) * p.g + i) * p.H + h;
     const int32_t* crow = p.cand + ui * CWd;
-    int32_t* orow = p.out + row * p.top_k;
-    const uint4 w4 = reinterpret_cast<const uint4*>(p.sel + row * 128)[lane];
-    const uint32_t wl[4] = {w4.x, w4.y, w4.z, w4.w};
-    const int own = __popc(wl[0]) + __popc(wl[1]) + __popc(wl[2]) + __popc(wl[3]);
-    int incl = own;
+    __syncthreads();   // the previous unit's candidates are no longer read
+    for (int t = threadIdx.x; t < CWd; t += kExpNT) cs[cand_swz(t)] = crow[t];
+    __syncthreads();
+    for (int i = wib; i < nm; i += kExpNT / 32) {
+      const long long row = (static_cast<long long>(u) * p.g + i) * p.H + h;
+      const uint4 w4 = lane * 4 < CWd / 32 ? reinterpret_cast<const uint4*>(p.sel + row * 128)[lane]
+                                           : make_uint4(0, 0, 0, 0);
+      const uint32_t wl[4] = {w4.x, w4.y, w4.z, w4.w};
+      const int own = __popc(wl[0]) + __popc(wl[1]) + __popc(wl[2]) + __popc(wl[3]);
+      int incl = own;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pre[4];
-    pre[0] = incl - own;
-#pragma unroll
-    for (int x = 1; x < 4; ++x) pre[x] = pre[x - 1] + __popc(wl[x - 1]);
-    const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
-#pragma unroll 2
-    for (int w0 = 0; w0 < nw; w0 += 4) {
-      int32_t val[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) val[x] = crow[(w0 + x) * 32 + lane];
-      const int owner = w0 >> 2;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
+      int at = incl - own;
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
-        const uint32_t word = __shfl_sync(0xffffffffu, wl[x], owner);
-        const int bw = __shfl_sync(0xffffffffu, pre[x], owner);
-        if ((word >> lane) & 1u) orow[bw + __popc(word & ltmask)] = val[x];
+        uint32_t bits = wl[x];
+        const int t0 = lane * 128 + x * 32;
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1;
+          if (at < p.top_k) stg[stage_swz(at)] = cs[cand_swz(t0 + b)];
+          ++at;
+        }
       }
+      __syncwarp();
+      int32_t* orow = p.out + row * p.top_k;
+      for (int t = lane; t < p.top_k; t += 32) orow[t] = t < total ? stg[stage_swz(t)] : -1;
+      __syncwarp();
     }
-    for (int t = total + lane; t < p.top_k; t += 32) orow[t] = -1;
   }
 }
 
