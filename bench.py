@@ -69,10 +69,8 @@ def algorithmic(c):
         "scan_filter": ("tensor", scan_flops),
         # a select must at least read Kc (key, index) pairs and write Kc indices per row
         "finalize": ("hbm", float(H * nC.sum() * (8 + 4))),
-        # candidate rows + member queries + every key once + selection bitmaps (512 B a row) written
-        "refine": ("hbm", float(H * nC.sum() * 4 + 2 * L * H * d * 2 + L * H * 512)),
-        # bitmaps read + output rows written + candidate rows read once
-        "refine_expand": ("hbm", float(L * H * 512 + L * H * k * 4 + H * nC.sum() * 4)),
+        # output rows + candidate rows + member queries + every key once
+        "refine": ("hbm", float(L * H * k * 4 + H * nC.sum() * 4 + 2 * L * H * d * 2)),
         "proxy": ("hbm", float(L * H * d * 2 + G * H * d * 2)),
         "fallback": ("hbm", 0.0),
         "refine_fallback": ("hbm", 0.0),

@@ -163,7 +163,7 @@ struct Plan {
   // sizes
   int G, cap, S, K_sel, heads_per_pass, nfb;
   // offsets
-  size_t off_proxy, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, off_miss, off_sel, total;
+  size_t off_proxy, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, off_miss, total;
 };
 
 // Sample stride and spill capacity for a select of K_sel keys per row over
@@ -212,8 +212,6 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(H) * p.G * cand_row_words(Kc) * sizeof(int32_t)) : 0;
   p.off_miss = o;
   o += (!dense && mode == PIVOT_REFINE) ? miss_bytes(static_cast<size_t>(H) * p.G, g) : 0;
-  p.off_sel = o;   // Refine's selection bitmaps: 512 bytes per output row
-  o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(L) * H * 512) : 0;
   p.total = o;
   return p;
 }
@@ -260,11 +258,10 @@ int launch_scan(const CUtensorMap& tmP, const CUtensorMap& tmK, const ScanParams
   return PIVOT_OK;
 }
 
-// Refine (selection bitmaps), the index rows from the bitmaps, then the exact
-// redo of the members the one-pass select missed.  `miss` points at the
-// workspace region sized by miss_bytes(units, g); rp.sel at rows * 512 bytes.
+// Refine, then the exact redo of the members its select could not settle.
+// `miss` points at the workspace region sized by miss_bytes(units, g).
 template <int D>
-int launch_refine(RefineParams rp, int units, long long rows, int sms, uint8_t* miss, cudaStream_t st) {
+int launch_refine(RefineParams rp, int units, int sms, uint8_t* miss, cudaStream_t st) {
   const int smem = RefineCfg<D>::smem_bytes(rp.Kc);
   CUDA_TRY(cudaFuncSetAttribute(refine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   rp.nbatch = (rp.g + 15) / 16;
@@ -278,15 +275,6 @@ int launch_refine(RefineParams rp, int units, long long rows, int sms, uint8_t* 
   {
     TraceScope tr("refine", st);
     refine_kernel<D><<<grid, RefineCfg<D>::NT, smem, st>>>(rp);
-  }
-  CUDA_TRY(cudaGetLastError());
-  {
-    TraceScope tr("refine_expand", st);
-    // one block per unit (group, head), grid-stride
-    const long long blocks = std::min<long long>(units, 16ll * std::max(1, sms));
-    const int esmem = expand_smem_words(rp.Kc, rp.top_k) * 4;
-    CUDA_TRY(cudaFuncSetAttribute(refine_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, esmem));
-    refine_expand_kernel<<<static_cast<unsigned>(std::max<long long>(1, blocks)), kExpNT, esmem, st>>>(rp, rows);
   }
   CUDA_TRY(cudaGetLastError());
   const int fsmem = (2 * cand_row_words(rp.Kc) + 2 * rp.top_k) * 4;
@@ -454,10 +442,8 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
       CUDA_TRY(cudaGetLastError());
     }
     uint8_t* miss = w + pl.off_miss;
-    rp.sel = reinterpret_cast<uint32_t*>(w + pl.off_sel);
-    const long long rows = static_cast<long long>(L) * H;
-    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, rows, dev->sms, miss, st)
-                        : launch_refine<64>(rp, H * pl.G, rows, dev->sms, miss, st);
+    int rc = (d == 128) ? launch_refine<128>(rp, H * pl.G, dev->sms, miss, st)
+                        : launch_refine<64>(rp, H * pl.G, dev->sms, miss, st);
     if (rc) return rc;
   }
   return PIVOT_OK;
@@ -469,7 +455,6 @@ size_t decode_ws_size(int B, int H, int d, int g, int Kc, int mode, int max_seql
   o += up(static_cast<size_t>(H) * B * max_seqlen * sizeof(uint32_t));       // order keys
   if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
   if (mode == PIVOT_REFINE) o += miss_bytes(static_cast<size_t>(H) * B, g);
-  if (mode == PIVOT_REFINE) o += up(static_cast<size_t>(B) * g * H * 512);   // selection bitmaps
   return o;
 }
 
@@ -568,10 +553,8 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
       CUDA_TRY(cudaGetLastError());
     }
     uint8_t* miss = reinterpret_cast<uint8_t*>(cand) + up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
-    rp.sel = reinterpret_cast<uint32_t*>(miss + miss_bytes(static_cast<size_t>(H) * B, g));
-    const long long rows = static_cast<long long>(B) * g * H;
-    int rc = (d == 128) ? launch_refine<128>(rp, H * B, rows, dev->sms, miss, st)
-                        : launch_refine<64>(rp, H * B, rows, dev->sms, miss, st);
+    int rc = (d == 128) ? launch_refine<128>(rp, H * B, dev->sms, miss, st)
+                        : launch_refine<64>(rp, H * B, dev->sms, miss, st);
     if (rc) return rc;
   }
   return PIVOT_OK;

@@ -46,9 +46,8 @@
 //  * the list is ranked exactly (pairwise when short, else by value bins or
 //    a radix select; ties in candidate order) and its decisions are OR-ed into
 //    the bitmap;
-//  * the member's warp writes the bitmap out (512 bytes); refine_expand_kernel
-//    turns every bitmap into its index row afterwards, so the row writes
-//    (4 bytes per index) do not take issue slots from this kernel.
+//  * the member's warp walks its bitmap in candidate order: each 32-bit word
+//    gives one coalesced store of its selected key indices.
 // A member whose chunk-0 range is empty, or whose boundary bin holds more than
 // kCap keys (ties), is not written here: it is recorded in a miss list and
 // refine_fallback_kernel redoes it exactly afterwards.
@@ -64,7 +63,6 @@ struct RefineParams {
   const uint16_t* keys;   // prefill [L][H][d]; decode packed cache [rows][H][d]
   const int32_t* cand;    // [H][G][cand_row_words(Kc)] candidate rows in read order (ptx.cuh)
   int32_t* out;           // prefill [L][H][top_k]; decode [B][g][H][top_k]
-  uint32_t* sel;          // selection bitmaps, 128 words per output row (bit t: candidate t taken)
   float* out_scores;      // same shape as out, or null
   const int32_t* cu;      // decode: [B+1] cache row offsets; null for prefill
   int G, L, H, g, top_k, Kc, d;
@@ -855,15 +853,39 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         }
         __syncwarp();
       }
-      // ---- warp sw writes member sw's selection bitmap (refine_expand_kernel
-      //      makes the index row; a miss's row is redone by the fallback)
+      // ---- warp sw writes member sw's row: its bitmap in candidate order, one
+      //      coalesced store per 32-candidate word (a miss's row is written by
+      //      the fallback)
       if (sw < nb) {
         const MemberSel& S = M->ms[sw];
         const int mode = S.mode, K = S.K;
         const long long orow = (it.qrow0 + it.mb + sw) * p.H + it.h;
+        int32_t* out_row = p.out + orow * p.top_k;
+        if (mode == kMAll) {
+          for (int t = lane; t < K; t += 32) out_row[t] = cx[t];
+        } else if (mode == kMBand) {
+          int base = 0;
+#pragma unroll 1
+          for (int w0 = 0; w0 < nch * 4; w0 += 4) {
+            uint32_t wd[4];
+            int32_t val[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              wd[x] = mb[16 * (w0 + x)];
+              val[x] = cx[(w0 + x) * 32 + lane];
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              if ((wd[x] >> lane) & 1u) out_row[base + __popc(wd[x] & ltmask)] = val[x];
+              base += __popc(wd[x]);
+            }
+          }
+        }
+        if (mode != kMMiss)
+          for (int t = K + lane; t < p.top_k; t += 32) out_row[t] = -1;
         uint32_t wds[4];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
+        for (int x = 0; x < 4 && keep_tmem; ++x) {
           const int w = 4 * lane + x;
           if (mode == kMAll) {
             const int u = K - 32 * w;
@@ -874,7 +896,6 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             wds[x] = 0u;
           }
         }
-        reinterpret_cast<uint4*>(p.sel + orow * 128)[lane] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
         if (keep_tmem) {
           // per-word prefix counts of the selection, for the scores' slots
           const int own = __popc(wds[0]) + __popc(wds[1]) + __popc(wds[2]) + __popc(wds[3]);
@@ -948,70 +969,6 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   }
 }
 
-constexpr int kExpNT = 256;
-
-// Index rows from the selection bitmaps.  A block takes a unit (group, head):
-// its candidate row goes to shared memory, and each warp expands one member's
-// row at a time.  Lane l owns candidates 128l .. 128l+127 (bitmap words
-// 4l .. 4l+3): after a warp scan of the words' popcounts it walks its own set
-// bits and writes their key indices to the warp's staging row, which then
-// leaves in coalesced stores, padded with -1.  Both shared arrays are
-// XOR-swizzled within 32-word groups so that the lanes' scattered accesses
-// fall in different banks.  Dynamic shared memory: expand_smem_words(Kc, top_k).
-__host__ __device__ inline int expand_stage_words(int top_k) { return (top_k + 31) / 32 * 32; }
-__host__ __device__ inline int expand_smem_words(int Kc, int top_k) {
-  return cand_row_words(Kc) + (kExpNT / 32) * expand_stage_words(top_k);
-}
-__device__ __forceinline__ int cand_swz(int t) { return t ^ ((t >> 7) & 31); }
-__device__ __forceinline__ int stage_swz(int p) { return p ^ ((p >> 6) & 31); }
-
-__global__ void __launch_bounds__(kExpNT, 2) refine_expand_kernel(RefineParams p, long long nrows) {
-  (void)nrows;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int CWd = cand_row_words(p.Kc);
-  int32_t* cs = reinterpret_cast<int32_t*>(smem_raw);
-  int32_t* stg = cs + CWd + wib * expand_stage_words(p.top_k);
-  const long long units = static_cast<long long>(p.H) * p.G;
-  for (long long ui = blockIdx.x; ui < units; ui += gridDim.x) {
-    const int h = static_cast<int>(ui / p.G), u = static_cast<int>(ui % p.G);
-    const int nm = p.cu ? p.g : min(u * p.g + p.g, p.L) - u * p.g;
-    const int32_t* crow = p.cand + ui * CWd;
-    __syncthreads();   // the previous unit's candidates are no longer read
-    for (int t = threadIdx.x; t < CWd; t += kExpNT) cs[cand_swz(t)] = crow[t];
-    __syncthreads();
-    for (int i = wib; i < nm; i += kExpNT / 32) {
-      const long long row = (static_cast<long long>(u) * p.g + i) * p.H + h;
-      const uint4 w4 = lane * 4 < CWd / 32 ? reinterpret_cast<const uint4*>(p.sel + row * 128)[lane]
-                                           : make_uint4(0, 0, 0, 0);
-      const uint32_t wl[4] = {w4.x, w4.y, w4.z, w4.w};
-      const int own = __popc(wl[0]) + __popc(wl[1]) + __popc(wl[2]) + __popc(wl[3]);
-      int incl = own;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int total = min(__shfl_sync(0xffffffffu, incl, 31), p.top_k);
-      int at = incl - own;
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        uint32_t bits = wl[x];
-        const int t0 = lane * 128 + x * 32;
-        while (bits) {
-          const int b = __ffs(bits) - 1;
-          bits &= bits - 1;
-          if (at < p.top_k) stg[stage_swz(at)] = cs[cand_swz(t0 + b)];
-          ++at;
-        }
-      }
-      __syncwarp();
-      int32_t* orow = p.out + row * p.top_k;
-      for (int t = lane; t < p.top_k; t += 32) orow[t] = t < total ? stg[stage_swz(t)] : -1;
-      __syncwarp();
-    }
-  }
-}
 
 constexpr int kRfbNT = 512;
 

@@ -26,11 +26,9 @@ def test_algorithmic_work_at_l131072():
     assert alg["scan_filter"] == ("tensor", 2.0 * d * H * float(last.sum()))
     assert abs(alg["scan_filter"][1] - 2.20e12) < 0.01e12
     n_cand = np.minimum(Kc, last)
-    want = H * n_cand.sum() * 4 + 2 * L * H * d * 2 + L * H * 512
+    want = L * H * k * 4 + H * n_cand.sum() * 4 + 2 * L * H * d * 2
     assert alg["refine"] == ("hbm", float(want))
-    # the index rows (17.2 GB) are written by the expand kernel from the bitmaps
-    assert alg["refine_expand"] == ("hbm", float(L * H * 512 + L * H * k * 4 + H * n_cand.sum() * 4))
-    assert abs(alg["refine_expand"][1] - 20.4e9) < 0.1e9
+    assert abs(alg["refine"][1] - 20.4e9) < 0.1e9
     assert alg["proxy"][0] == "hbm" and alg["fallback"] == ("hbm", 0.0)
 
 
