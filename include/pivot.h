@@ -201,6 +201,17 @@ int pivot_sync_status(void* stream, int* flags);
 int pivot_trace_enable(int on);
 int pivot_trace_collect(char* names, size_t names_len, float* ms, int* count, int max_items);
 
+/*
+ * Testing aid (the method has no counterpart).  Every wait of a kernel on
+ * another of its roles (an mbarrier phase) gives up after a limit, raises the
+ * status that pivot_sync_status() reports as PIVOT_ERR_TIMEOUT, drains what it
+ * had issued and returns; no kernel traps or spins for ever.  This sets that
+ * limit, in nanoseconds, for the calls that follow in this process (0 restores
+ * the default of 2 seconds).  A tiny limit makes a call time out on purpose;
+ * its outputs are then not valid.  Returns PIVOT_OK.
+ */
+int pivot_set_wait_limit(unsigned long long ns);
+
 /* Message of the last error on the calling thread ("" if none). */
 const char* pivot_last_error(void);
 

@@ -34,7 +34,7 @@ EXPORTED = (
     "pivot_workspace_size", "pivot_index_ws", "dense_workspace_size", "dense_index_ws",
     "pivot_decode_workspace_size", "pivot_decode_index_ws", "pivot_sync_status", "pivot_last_error",
     "pivot_trace_enable", "pivot_trace_collect", "pivot_decode_index_noalloc",
-    "pivot_index_ex", "pivot_decode_index_ex",
+    "pivot_index_ex", "pivot_decode_index_ex", "pivot_set_wait_limit",
 )
 
 
@@ -72,6 +72,7 @@ def load_library():
         "pivot_decode_index_noalloc": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P], I),
         "pivot_index_ex": ([P, P, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
         "pivot_decode_index_ex": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
+        "pivot_set_wait_limit": ([ctypes.c_ulonglong], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)

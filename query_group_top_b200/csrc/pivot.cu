@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -34,6 +35,13 @@ using namespace pivot;
 __device__ int g_status_word;  // per-device kernel status bits
 
 thread_local char g_err[512] = "";
+
+// Limit of the kernels' bounded waits (pivot_set_wait_limit); 0 = the default.
+std::atomic<unsigned long long> g_wait_ns{0};
+unsigned long long wait_limit_ns() {
+  const unsigned long long v = g_wait_ns.load();
+  return v ? v : kWaitNs;
+}
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -373,6 +381,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     sp.spill = reinterpret_cast<uint2*>(w + pl.off_spill);
     sp.cnt = reinterpret_cast<int4*>(w + pl.off_cnt);
     sp.status = dev->status;
+    sp.wait_ns = wait_limit_ns();
     int rc = (d == 128) ? launch_scan<128>(tmP, tmK, sp, nh, st) : launch_scan<64>(tmP, tmK, sp, nh, st);
     if (rc) return rc;
 
@@ -436,6 +445,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.d = d;
     rp.tmem_cols = tmem_cols_for(Kc);
     rp.status = dev->status;
+    rp.wait_ns = wait_limit_ns();
     if (out_cand) {
       cand_export_kernel<<<static_cast<unsigned>(H * pl.G), 256, 0, st>>>(rp.cand, out_cand, pl.G, H, Kc, g, L,
                                                                           nullptr, 0);
@@ -548,6 +558,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     rp.d = d;
     rp.tmem_cols = tmem_cols_for(Kc);
     rp.status = dev->status;
+    rp.wait_ns = wait_limit_ns();
     if (out_cand) {
       cand_export_kernel<<<static_cast<unsigned>(H * B), 256, 0, st>>>(cand, out_cand, B, H, Kc, g, 0, cu, max_seqlen);
       CUDA_TRY(cudaGetLastError());
@@ -744,6 +755,11 @@ int pivot_sync_status(void* stream, int* flags) {
 }
 
 const char* pivot_last_error(void) { return g_err; }
+
+int pivot_set_wait_limit(unsigned long long ns) {
+  g_wait_ns.store(ns);
+  return PIVOT_OK;
+}
 
 int pivot_trace_enable(int on) {
   g_trace_on = on != 0;

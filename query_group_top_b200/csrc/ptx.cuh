@@ -18,7 +18,7 @@ enum : int {
   kStNoConverge = 8,  // a selection exceeded its round limit (cannot happen on finite scores)
 };
 
-constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s: the default limit of a wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -76,17 +76,19 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 constexpr uint32_t kSuspendNs = 20000;
 
 // Waits until the phase with the given parity of `bar` has completed.
-// Returns false (and sets *abort, raising kStTimeout) after kWaitNs, or
+// Returns false (and sets *abort, raising kStTimeout) after limit_ns, or
 // returns false at once when another role has already set *abort.  Between
 // polls the warp is suspended on the barrier itself (mbar_try_wait_suspend),
 // so waiting warps leave the issue slots to the warps they wait for.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                          unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
+    if (mbar_try_wait_suspend(bar, parity, min(kSuspendNs, static_cast<uint32_t>(min(limit_ns, 0xFFFFFFFFull)))))
+      return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort = 1;
       atomicOr(status, kStTimeout);
       return false;
@@ -94,7 +96,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Bounded wait used on the clean-up path (no abort flag, shorter limit).
+// Bounded wait used on the clean-up path (no abort flag, a fixed limit that
+// the test knob of the other waits does not shorten: what was issued drains).
 __device__ __forceinline__ void mbar_wait_cleanup(uint32_t bar, uint32_t parity) {
   const unsigned long long t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {

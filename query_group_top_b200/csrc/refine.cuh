@@ -74,6 +74,7 @@ struct RefineParams {
   int* miss_count;        // zeroed before the launch
   int miss_cap;
   int* status;
+  unsigned long long wait_ns;   // limit of every bounded wait
 };
 
 // member selection modes
@@ -359,14 +360,14 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       // the list and B buffers of this parity are free once the select warps
       // are done with the item two back
       if (kk >= 2 && ok && warp == 0)
-        ok = mbar_wait(smem_u32(&M->cfree[buf]), ((kk >> 1) - 1) & 1, abort_flag, p.status);
+        ok = mbar_wait(smem_u32(&M->cfree[buf]), ((kk >> 1) - 1) & 1, abort_flag, p.status, p.wait_ns);
       ok = !named_barrier_or(1, C::NPROD, !ok);
       if (ok && pt == 0) {
         const uint32_t bytes = static_cast<uint32_t>(it.nch) * 128u * 4u;
         mbar_arrive_expect_tx(cbar, bytes);
         if (bytes) bulk_copy_g2s(smem_u32(cx), p.cand + (static_cast<long long>(it.h) * p.G + it.u) * CW, bytes, cbar);
       }
-      if (ok) ok = mbar_wait(cbar, (kk >> 1) & 1, abort_flag, p.status);
+      if (ok) ok = mbar_wait(cbar, (kk >> 1) & 1, abort_flag, p.status, p.wait_ns);
       const uint16_t* kbase = p.keys + (it.key_row0 * p.H + it.h) * static_cast<long long>(D) + p8 * 8;
       const uint32_t bB = sB + buf * C::B_BYTES;
       for (int ci = 0; ci < it.nch; ++ci) {
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         const int s = sseq % C::NS;
         // one warp watches the stage; the others sleep on the named barrier
         if (sseq >= C::NS && ok && warp == 0)
-          ok = mbar_wait(smem_u32(&M->empty[s]), ((sseq / C::NS) - 1) & 1, abort_flag, p.status);
+          ok = mbar_wait(smem_u32(&M->empty[s]), ((sseq / C::NS) - 1) & 1, abort_flag, p.status, p.wait_ns);
         ok = !named_barrier_or(1, C::NPROD, !ok);
         if (ok) {
           const uint32_t dst0 = sA + s * C::STAGE;
@@ -424,11 +425,11 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       for (int ci = 0; ci < NCH && ok; ++ci) {
         const int c = chunk_at(ci, it.nch);
         // the previous item's select warps are done with these columns
-        if (kk >= 1) ok = mbar_wait(smem_u32(&M->tfree[c]), (kk - 1) & 1, abort_flag, p.status);
+        if (kk >= 1) ok = mbar_wait(smem_u32(&M->tfree[c]), (kk - 1) & 1, abort_flag, p.status, p.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (ok && c < it.nch) {
           const int s = sseq % C::NS;
-          ok = mbar_wait(smem_u32(&M->full[s]), (sseq / C::NS) & 1, abort_flag, p.status);
+          ok = mbar_wait(smem_u32(&M->full[s]), (sseq / C::NS) & 1, abort_flag, p.status, p.wait_ns);
           ok = __all_sync(0xffffffffu, ok);
           if (ok && lane == 0) {
             tc_fence_after();
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       const int buf = kk & 1;
       const int nch = it.nch, nb = it.nb;
       const int32_t* cx = cidx0 + buf * CW;
-      if (ok) ok = mbar_wait(smem_u32(&M->cready[buf]), (kk >> 1) & 1, abort_flag, p.status);
+      if (ok) ok = mbar_wait(smem_u32(&M->cready[buf]), (kk >> 1) & 1, abort_flag, p.status, p.wait_ns);
       // ---- per-member usable counts (the candidate set is ascending) and modes
       if (stid < 16 && ok) {
         MemberSel& S = M->ms[stid];
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       if (anyb) {
         // ---- chunk 0's score range sets each member's histogram bins
         if (st == 0) {
-          if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status);
+          if (ok) ok = mbar_wait(smem_u32(&M->tready[0]), kk & 1, abort_flag, p.status, p.wait_ns);
           ok = __all_sync(0xffffffffu, ok);
           if (ok) {
             tc_fence_after();
@@ -577,7 +578,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         const uint32_t sh0 = smem_u32(shist);
         for (int i = st; i < nch; i += 4) {
           const int c = chunk_at(i, nch);
-          if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
+          if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, p.wait_ns);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
@@ -641,7 +642,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
 #pragma unroll 1
       for (int i = st; i < nch; i += 4) {
         const int c = chunk_at(i, nch);
-        if (ok && !anyb) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
+        if (ok && !anyb) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, p.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (!anyb) {   // nothing to classify
@@ -950,7 +951,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       // release then answers a commit of this item, and the MMA warp can never
       // find a chunk's "free" barrier two phases ahead of its wait.
       for (int c = nch + ((st - nch) & 3); c < NCH; c += 4) {
-        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status);
+        if (ok) ok = mbar_wait(smem_u32(&M->tready[c]), kk & 1, abort_flag, p.status, p.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) release(c);
       }

@@ -59,6 +59,7 @@ struct ScanParams {
                    // downward from its last; a region whose two runs sum to
                    // more than cap/2 has overflowed
   int* status;     // device status word
+  unsigned long long wait_ns;   // limit of every bounded wait
 };
 
 __device__ __forceinline__ int row_bound(const ScanParams& p, int i) {
@@ -179,7 +180,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
         if (!ok) return;
         const int s = step % C::NST;
         const int use = step / C::NST;
-        if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status)) {
+        if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_ns)) {
           ok = false;
           return;
         }
@@ -198,18 +199,18 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
       constexpr uint32_t idesc = umma_idesc_bf16(C::BM, C::BN);
       int use[C::NACC] = {0, 0, 0, 0};
       int step = 0;
-      bool ok = mbar_wait(a_full, 0, abort_flag, p.status);
+      bool ok = mbar_wait(a_full, 0, abort_flag, p.status, p.wait_ns);
       for_each_step(ns, p.S, nkt, [&](int q, int, int) {
         if (!ok) return;
         const int s = step % C::NST;
-        if (!mbar_wait(full_bar(s), (step / C::NST) & 1, abort_flag, p.status)) {
+        if (!mbar_wait(full_bar(s), (step / C::NST) & 1, abort_flag, p.status, p.wait_ns)) {
           ok = false;
           return;
         }
         int uq = 0;
 #pragma unroll
         for (int x = 0; x < C::NACC; ++x) uq = (x == q) ? use[x] : uq;
-        if (uq > 0 && !mbar_wait(tempty_bar(q), (uq - 1) & 1, abort_flag, p.status)) {
+        if (uq > 0 && !mbar_wait(tempty_bar(q), (uq - 1) & 1, abort_flag, p.status, p.wait_ns)) {
           ok = false;
           return;
         }
@@ -419,7 +420,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
       if (q != e) return;
       advance(phase);
       // the whole warp decides together: tcgen05.ld below is warp-collective
-      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(e), use & 1, abort_flag, p.status));
+      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(tfull_bar(e), use & 1, abort_flag, p.status, p.wait_ns));
       ++use;
       if (!alive) return;
       tc_fence_after();

@@ -79,7 +79,8 @@ def header_declarations():
             prm = prm.strip()
             if not prm or prm == "void":
                 continue
-            kinds.append("p" if "*" in prm else ("z" if "size_t" in prm else "i"))
+            # size_t and unsigned long long are the same 64-bit unsigned kind here
+            kinds.append("p" if "*" in prm else ("z" if ("size_t" in prm or "long long" in prm) else "i"))
         decls[name] = ("p" if "*" in ret else ("z" if ret == "size_t" else "i"), kinds)
     return decls
 

@@ -406,3 +406,67 @@ def test_refine_select_ties_and_misses():
     assert res["exempt"] == 0
     res, _ = check_full(qi, ki, 8, 300, 2000, oracle.REFINE)
     assert res["exempt"] == 0
+
+
+def test_bounded_waits_time_out_and_the_next_call_is_exact():
+    """Every kernel wait on another role gives up after a limit.  With the
+    limit set to 1 ns a call's waits run out: the kernels drain what they
+    issued, return, and pivot_sync_status reports PIVOT_ERR_TIMEOUT; with the
+    default limit restored the next call is exact."""
+    import ctypes
+    lib = qg.load_library()
+    L, H, d, g, top_k, Kc = 300, 1, 64, 4, 8, 16
+    q, k = synthetic.gen_prefill(L, H, d, seed=5, rho=0.9)
+    qd, kd = to_dev(q), to_dev(k)
+    qg.sync_status()
+    stream = torch.cuda.current_stream().cuda_stream
+    try:
+        lib.pivot_set_wait_limit(1)
+        qg.pivot_index(qd, kd, g, top_k, Kc, qg.REFINE)
+        flags = ctypes.c_int(0)
+        rc = lib.pivot_sync_status(stream, ctypes.byref(flags))
+        assert rc == 4 and flags.value & qg.FLAG_TIMEOUT, (rc, flags.value)
+    finally:
+        lib.pivot_set_wait_limit(0)
+    assert qg.sync_status() == 0
+    check_full(q, k, g, top_k, Kc, oracle.REFINE)
+
+
+def test_bare_entry_points_allocate_their_own_workspace():
+    """pivot_index, dense_index and pivot_decode_index take their scratch with
+    cudaMallocAsync on the stream; their rows equal the oracle's."""
+    lib = qg.load_library()
+    stream = torch.cuda.current_stream().cuda_stream
+    L, H, d, g, top_k, Kc = 700, 2, 128, 8, 30, 64
+    q, k = synthetic.gen_prefill(L, H, d, seed=41, rho=0.9)
+    qd, kd = to_dev(q), to_dev(k)
+    pos = np.broadcast_to(np.arange(L)[:, None], (L, H))
+    for mode in (oracle.REFINE, oracle.REUSE):
+        out = torch.full((L, H, top_k), -7, dtype=torch.int32, device="cuda")
+        assert lib.pivot_index(qd.data_ptr(), kd.data_ptr(), L, H, d, g, top_k, Kc, mode, out.data_ptr(), stream) == 0
+        qg.sync_status()
+        ref = oracle.prefill(q, k, g, top_k, Kc, mode)
+        cedge = ref["cand_edge"][np.arange(L) // g] if mode == oracle.REFINE else None
+        assert_parity(compare(out.cpu().numpy(), ref["out"], ref["edge"], pos, cedge), f"bare pivot_index {mode}")
+    out = torch.full((L, H, top_k), -7, dtype=torch.int32, device="cuda")
+    assert lib.dense_index(qd.data_ptr(), kd.data_ptr(), L, H, d, top_k, out.data_ptr(), stream) == 0
+    qg.sync_status()
+    ref = oracle.dense(q, k, top_k)
+    assert_parity(compare(out.cpu().numpy(), ref["out"], ref["edge"], pos), "bare dense_index")
+    dec = synthetic.gen_decode(3, H, d, 2, seed=43, lo=100, hi=3000)
+    dq, dk, cu = to_dev(dec.q), to_dev(dec.kcache), torch.from_numpy(dec.cu_seqlens).cuda()
+    max_seqlen = int(np.diff(dec.cu_seqlens).max())
+    bi, hh = np.meshgrid(np.arange(3), np.arange(H), indexing="ij")
+    for mode in (oracle.REFINE, oracle.REUSE):
+        out = torch.full((3, 2, H, top_k), -7, dtype=torch.int32, device="cuda")
+        assert lib.pivot_decode_index(dq.data_ptr(), dk.data_ptr(), cu.data_ptr(), 3, H, d, 2, top_k, Kc, mode,
+                                      max_seqlen, out.data_ptr(), stream) == 0
+        qg.sync_status()
+        r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, 2, top_k, Kc, mode, bi.ravel(), hh.ravel())
+        want = r["out"].reshape(3, H, 2, top_k).transpose(0, 2, 1, 3)
+        edge = r["edge"].reshape(3, H, 2, 2).transpose(0, 2, 1, 3)
+        cedge = None
+        if mode == oracle.REFINE:
+            cedge = np.broadcast_to(r["cand_edge"].reshape(3, H, 1, 2).transpose(0, 2, 1, 3), (3, 2, H, 2))
+        dpos = np.broadcast_to((dec.n_ctx[:, None] + np.arange(2)[None, :])[:, :, None], (3, 2, H))
+        assert_parity(compare(out.cpu().numpy(), want, edge, dpos, cedge), f"bare pivot_decode_index {mode}")
