@@ -356,6 +356,32 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_only(args, qg, torch):
+    """The MTP decode step alone on a few sequences of its workload (a small
+    case for profiling the decode kernels); prints ms per step."""
+    dc = synthetic.CONFIGS["C4"]
+    B = min(args.decode_only, dc["B"])
+    dq, dk, dcu, n_ctx = synthetic.gen_decode_device(B, dc["H"], dc["d"], dc["g"], dc["seed"], dc["lo"], dc["hi"],
+                                                     dc["rho"], dc["heavy_frac"], dc["heavy_scale"])
+    max_seqlen = int((n_ctx + dc["g"]).max())
+    dout = torch.empty((B, dc["g"], dc["H"], dc["top_k"]), dtype=torch.int32, device="cuda")
+    step = lambda: qg.pivot_decode_index(dq, dk, dcu, dc["g"], dc["top_k"], dc["Kc"], qg.REFINE, max_seqlen=max_seqlen,
+                                         out=dout)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    qg.sync_status()
+    key_bytes = float(n_ctx.astype(np.int64).sum() + B * (dc["g"] - 1)) * dc["H"] * dc["d"] * 2
+    print(json.dumps({"decode_only_sequences": B, "ms_per_step": e0.elapsed_time(e1) / args.steps,
+                      "key_bytes": key_bytes}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,6 +392,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2, help="0 skips the end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--no-configs", action="store_true", help="skip the records of the smaller prefill workloads")
+    ap.add_argument("--decode-only", type=int, default=0, metavar="B",
+                    help="profiling aid: run only the MTP decode step on the first B sequences of its workload")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: index only this many heads of the workload (0 = all)")
     args = ap.parse_args()
@@ -387,6 +415,10 @@ def main():
     torch.cuda.set_device(local)
     ranks = RankGroup("nccl", torch.device("cuda", local))
     barrier, max_over_ranks = ranks.barrier, ranks.max
+
+    if args.decode_only > 0:
+        decode_only(args, qg, torch)
+        return
 
     c = dict(synthetic.CONFIGS[WORKLOAD])
     if args.heads > 0:
