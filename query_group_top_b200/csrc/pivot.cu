@@ -179,7 +179,7 @@ struct Plan {
 void filter_shape(int K_sel, int L, int* cap, int* S) {
   const int BN = 128;  // keys per scan tile
   int c = std::max(2 * K_sel, 4 * BN);
-  int s = std::max(1, std::min(32, c / BN));
+  int s = std::max(1, std::min(16, c / BN));
   // at most 511 sampled tiles per row, so a row's sample fits 16-bit bin counts
   const int min_s = (L + BN * 511 - 1) / (BN * 511);
   s = std::max(s, min_s);

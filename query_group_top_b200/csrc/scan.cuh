@@ -28,7 +28,7 @@
 // The threshold comes from a sample of the row's prefix: every S-th key tile is
 // scanned twice before the main pass (two MSB radix histogram passes over the
 // sample in shared memory), and tau is set at a sample rank a few standard
-// deviations (three) above K * (sample size / prefix), so that nearly always
+// deviations (four) above K * (sample size / prefix), so that nearly always
 // at least K scores pass it.  Rows whose prefix fits half the
 // spill capacity take every key (tau = -inf).  Rows where the guess is wrong
 // (fewer than K survivors, or more than a spill region holds) are detected by
@@ -281,7 +281,7 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
           const int total = nsamp[r];
           if (row_samples && total > 0) {
             const float expect = static_cast<float>(p.K_sel) * static_cast<float>(total) / static_cast<float>(bound);
-            const int target_rank = static_cast<int>(ceilf(expect + 3.0f * sqrtf(expect) + 4.0f));
+            const int target_rank = static_cast<int>(ceilf(expect + 4.0f * sqrtf(expect) + 4.0f));
             if (target_rank <= total) {
               int cum = 0;
               for (int b = 255; b >= 0; --b) {
