@@ -5,9 +5,11 @@ One step = one PIVOT-Refine call (proxy build, tcgen05 prefix scan with fused
 filter, exact candidate select, per-member refine) over the long-context
 prefill workload: L=131072, H=16, d=128, g=16, top_k=2048, Kc=4096, bf16,
 seeded synthetic inputs (heavy-tailed keys, AR(1) queries).  The metric is
-indexed query-heads per second (L*H per step), aggregated over all GPUs; each
-GPU indexes its own independent layer (weak scaling, no collective on the
-data path).
+indexed query-heads per second (L*H per step), aggregated over all GPUs.  On N
+GPUs the heads of the one layer are split: rank r indexes heads
+[r*H/N, (r+1)*H/N) (strong scaling; heads are independent, so there is no
+collective on the data path, only the barriers and the max over ranks of the
+timing).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,6 +38,7 @@ import synthetic  # noqa: E402
 METRIC = "PIVOT-Refine indexed queries/s at L=131072; fraction of tensor/HBM roofline"
 UNIT = "query-heads/s"
 WORKLOAD = "C3"
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal
 
 
 def peaks():
@@ -48,13 +51,14 @@ def peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
 
 
-def workload_config(c):
+def workload_config(c, world=1):
     return {"workload": f"{WORKLOAD} long-context prefill L={c['L']} H={c['H']} d={c['d']} g={c['g']} "
                         f"top_k={c['top_k']} Kc={c['Kc']} PIVOT-Refine",
             "generator": f"keys N(0,1) with {c['heavy_frac']*100:g}% positions x{c['heavy_scale']:g}; "
                          f"queries AR(1) rho={c['rho']}; seed {c['seed']} (+rank)",
             "l2": "inputs 1.07 GB and outputs 17.2 GB per step exceed the 126 MB L2; no flush needed",
-            "parallelism": "one independent layer per GPU (weak scaling), no collective"}
+            "parallelism": (f"heads split across {world} GPUs (rank r: heads [r*H/N, (r+1)*H/N)), "
+                            "no collective on the data path")}
 
 
 def algorithmic(c):
@@ -205,15 +209,16 @@ class RankGroup:
             self.dist.destroy_process_group()
 
 
-def weak_value(world, L, H, ms_max):
-    """Whole-job throughput: every rank indexes its own L x H problem (weak
-    scaling), and the job takes as long as its slowest rank."""
-    return world * L * H / (ms_max / 1000.0)
+def job_value(L, H, ms_max):
+    """Whole-job throughput: the ranks together index the layer's L x H
+    query-heads, and the job takes as long as its slowest rank."""
+    return L * H / (ms_max / 1000.0)
 
 
-def rank_seed(base, rank):
-    """Each rank draws its own independent layer of the workload."""
-    return base + rank
+def split(n, rank, world):
+    """Items [a, b) of n (the decode batch's sequences) that rank `rank` of
+    `world` takes: contiguous, in rank order, sizes differing by at most one."""
+    return rank * n // world, (rank + 1) * n // world
 
 
 class ClockSampler:
@@ -347,7 +352,7 @@ def run_reference(args, rank):
     value = tot_q / tot_t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(c),
             "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": cores,
                              "sample": f"{tot_u} random (group, head) units of {WORKLOAD} over {args.steps} steps "
@@ -361,8 +366,8 @@ def decode_only(args, qg, torch):
     case for profiling the decode kernels); prints ms per step."""
     dc = synthetic.CONFIGS["C4"]
     B = min(args.decode_only, dc["B"])
-    dq, dk, dcu, n_ctx = synthetic.gen_decode_device(B, dc["H"], dc["d"], dc["g"], dc["seed"], dc["lo"], dc["hi"],
-                                                     dc["rho"], dc["heavy_frac"], dc["heavy_scale"])
+    dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], dc["seed"], dc["lo"], dc["hi"],
+                                                     dc["rho"], dc["heavy_frac"], dc["heavy_scale"], first=0, count=B)
     max_seqlen = int((n_ctx + dc["g"]).max())
     dout = torch.empty((B, dc["g"], dc["H"], dc["top_k"]), dtype=torch.int32, device="cuda")
     step = lambda: qg.pivot_decode_index(dq, dk, dcu, dc["g"], dc["top_k"], dc["Kc"], qg.REFINE, max_seqlen=max_seqlen,
@@ -424,10 +429,20 @@ def main():
     if args.heads > 0:
         c["H"] = min(args.heads, c["H"])
     L, H, d, g, top_k, Kc = c["L"], c["H"], c["d"], c["g"], c["top_k"], c["Kc"]
-    q_np, k_np = synthetic.gen_prefill(L, H, d, rank_seed(c["seed"], rank), c["rho"], c["heavy_frac"], c["heavy_scale"])
+    if world > H:
+        raise SystemExit(f"bench: {world} ranks but only {H} heads to split")
+    # every rank draws the same layer and keeps its own heads, as a contiguous
+    # [L, nh, d] layer (the layout a head-parallel model holds per GPU)
+    h0, h1 = qg.head_range(H, rank, world)
+    nh = h1 - h0
+    q_all, k_all = synthetic.gen_prefill(L, H, d, c["seed"], c["rho"], c["heavy_frac"], c["heavy_scale"])
+    q_np = np.ascontiguousarray(q_all[:, h0:h1])
+    k_np = np.ascontiguousarray(k_all[:, h0:h1])
+    del q_all, k_all
+    cl = dict(c, H=nh)   # this rank's share of the layer
     q = torch.from_numpy(q_np.view(np.int16)).cuda().view(torch.bfloat16)
     k = torch.from_numpy(k_np.view(np.int16)).cuda().view(torch.bfloat16)
-    out = torch.empty((L, H, top_k), dtype=torch.int32, device="cuda")
+    out = torch.empty((L, nh, top_k), dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
@@ -457,11 +472,11 @@ def main():
     clk = clocks.stop()
     flags = qg.sync_status()
     ms_max = max_over_ranks(ms)
-    value = weak_value(world, L, H, ms_max)
+    value = job_value(L, H, ms_max)
 
-    # roofline of the dominant kernel
+    # roofline of the dominant kernel (per launch on this rank's heads)
     pk = peaks()
-    alg = algorithmic(c)
+    alg = algorithmic(cl)
     kern = {name: {"ms_per_launch": tot / max(n, 1), "launches": n, "share": tot / (ms * args.steps)}
             for name, (tot, n) in trace.items()}
     dom = max(trace, key=lambda n: trace[n][0])
@@ -475,10 +490,23 @@ def main():
     else:
         achieved = work / t_launch / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": measured_traffic(dom, H), "kernel": dom,
+                "frac": achieved / pk["hbm"], "traffic": measured_traffic(dom, nh), "kernel": dom,
                 "peak_note": f"{pk['src']} HBM copy bandwidth"}
     scan_t = trace.get("scan_filter", (0, 1))
-    scan_tf = alg["scan_filter"][1] / (scan_t[0] / scan_t[1] / 1000.0) / 1e12 if scan_t[0] else None
+    scan_rec = None
+    if scan_t[0]:
+        scan_tf = alg["scan_filter"][1] / (scan_t[0] / scan_t[1] / 1000.0) / 1e12
+        # the fp32 proxy is scanned exactly as three bf16 terms: three bf16
+        # MMAs per key tile carry each algorithmic multiply-add
+        scan_rec = {"ms_per_launch": scan_t[0] / scan_t[1], "tflops": scan_tf,
+                    "frac_of_bf16_sustained": scan_tf / pk["bf16_sust"],
+                    "frac_of_bf16_burst": scan_tf / pk["bf16"],
+                    "bf16_mma_terms": 3, "bf16_mma_tflops": 3 * scan_tf,
+                    "bf16_mma_frac_of_sustained": 3 * scan_tf / pk["bf16_sust"]}
+        # the exact top-Kc select that follows the scan's fused filter
+        sel_ms = sum(trace[n][0] / trace[n][1] for n in ("finalize", "fallback") if n in trace)
+        scan_rec["select_ms_per_call"] = sel_ms
+        scan_rec["select_share_of_scan_and_select"] = sel_ms / (sel_ms + scan_rec["ms_per_launch"])
     gpu_launches = sum(n for _, n in trace.values())
 
     # end to end through the public API: pinned host inputs -> device -> indexer -> host result
@@ -489,10 +517,10 @@ def main():
         q_h = torch.from_numpy(q_np.view(np.int16)).view(torch.bfloat16).pin_memory()
         k_h = torch.from_numpy(k_np.view(np.int16)).view(torch.bfloat16).pin_memory()
         try:
-            out_h = torch.empty((L, H, top_k), dtype=torch.int32, pin_memory=True)
+            out_h = torch.empty((L, nh, top_k), dtype=torch.int32, pin_memory=True)
             pinned = True
         except Exception:
-            out_h = torch.empty((L, H, top_k), dtype=torch.int32)
+            out_h = torch.empty((L, nh, top_k), dtype=torch.int32)
             pinned = False
         q_d = torch.empty_like(q)
         k_d = torch.empty_like(k)
@@ -515,7 +543,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps)
-        e2e = {"value": weak_value(world, L, H, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e = {"value": job_value(L, H, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(q.numel() * 2 + k.numel() * 2),
                "d2h_bytes_per_step": int(out.numel() * 4), "pinned_output": pinned}
         del q_h, k_h, out_h, q_d, k_d
@@ -540,10 +568,11 @@ def main():
         out_dense = torch.empty_like(out)
         dense_ms = timed(lambda: qg.dense_index(q, k, top_k, out=out_dense), 1)
         qg.sync_status()
+        reuse_ms, dense_ms = max_over_ranks(reuse_ms), max_over_ranks(dense_ms)
         # Recall@k against the dense indexer on a seeded 1% of rows
         rng = np.random.default_rng(7)
-        rows = torch.from_numpy(rng.integers(1, L, size=L * H // 100)).cuda()
-        heads = torch.from_numpy(rng.integers(0, H, size=rows.numel())).cuda()
+        rows = torch.from_numpy(rng.integers(1, L, size=L * nh // 100)).cuda()
+        heads = torch.from_numpy(rng.integers(0, nh, size=rows.numel())).cuda()
         dn = out_dense[rows, heads].cpu().numpy()
         rec = {}
         for name, o in (("refine", out), ("reuse", out_reuse)):
@@ -551,13 +580,16 @@ def main():
             hit = [np.intersect1d(a[a >= 0], b[b >= 0]).size / max(1, (b >= 0).sum()) for a, b in zip(pv, dn)]
             rec[name] = float(np.mean(hit))
         del out_dense
-        # MTP decode workload: one step over 64 sequences (keys drawn on the device)
+        # MTP decode workload: one step over 64 sequences (keys drawn on the
+        # device), the sequences split across the ranks
         dc = synthetic.CONFIGS["C4"]
-        dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], rank_seed(dc["seed"], rank),
+        b0, b1 = split(dc["B"], rank, world)
+        dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], dc["seed"],
                                                          dc["lo"], dc["hi"], dc["rho"], dc["heavy_frac"],
-                                                         dc["heavy_scale"])
+                                                         dc["heavy_scale"], first=b0, count=b1 - b0)
+        nb = b1 - b0
         max_seqlen = int((n_ctx + dc["g"]).max())
-        dout = torch.empty((dc["B"], dc["g"], dc["H"], dc["top_k"]), dtype=torch.int32, device="cuda")
+        dout = torch.empty((nb, dc["g"], dc["H"], dc["top_k"]), dtype=torch.int32, device="cuda")
         dstep = lambda: qg.pivot_decode_index(dq, dk, dcu, dc["g"], dc["top_k"], dc["Kc"], qg.REFINE,
                                               max_seqlen=max_seqlen, out=dout)
         for _ in range(2):
@@ -568,29 +600,36 @@ def main():
         qg.trace_enable(False)
         dtr = qg.trace_collect()
         qg.sync_status()
-        key_bytes = float(n_ctx.astype(np.int64).sum() + dc["B"] * (dc["g"] - 1)) * dc["H"] * dc["d"] * 2
+        key_bytes = float(n_ctx.astype(np.int64).sum() + nb * (dc["g"] - 1)) * dc["H"] * dc["d"] * 2
         dscan = dtr.get("decode_scan", (0.0, 1))
         dscan_ms = dscan[0] / max(dscan[1], 1)
+        dscan_gbs = key_bytes / (dscan_ms / 1000.0) / 1e9 if dscan_ms else None
+        dec_ms_max = max_over_ranks(dec_ms)
         decode = {"workload": f"C4 MTP decode B={dc['B']} n_b~U[{dc['lo']},{dc['hi']}] H={dc['H']} d={dc['d']} "
                               f"g={dc['g']} top_k={dc['top_k']} Kc={dc['Kc']} PIVOT-Refine",
-                  "ms_per_step": dec_ms, "query_heads_per_s": dc["B"] * dc["g"] * dc["H"] / (dec_ms / 1000.0),
+                  "sequences_per_rank": nb, "ms_per_step": dec_ms_max,
+                  "query_heads_per_s": dc["B"] * dc["g"] * dc["H"] / (dec_ms_max / 1000.0),
                   "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in dtr.items()},
-                  "decode_scan_hbm_gbs": key_bytes / (dscan_ms / 1000.0) / 1e9 if dscan_ms else None,
-                  "decode_scan_hbm_frac": (key_bytes / (dscan_ms / 1000.0) / 1e9 / pk["hbm"]) if dscan_ms else None,
+                  "decode_scan_hbm_gbs": dscan_gbs,
+                  # a read-only stream against the nominal HBM3e bandwidth, and
+                  # against the measured copy (read + write) bandwidth
+                  "decode_scan_hbm_frac": dscan_gbs / NOMINAL_HBM_GBS if dscan_gbs else None,
+                  "decode_scan_frac_of_measured_copy": dscan_gbs / pk["hbm"] if dscan_gbs else None,
+                  "decode_step_hbm_frac": (key_bytes / (dec_ms / 1000.0) / 1e9) / NOMINAL_HBM_GBS,
                   "key_bytes": key_bytes}
         del dq, dk, dcu, dout
         torch.cuda.empty_cache()
-        w3 = config_work(c)
-        extras = {"refine_ms": ms, "reuse_ms": reuse_ms, "dense_ms": dense_ms, "decode": decode,
-                  "speedup_refine_vs_dense": dense_ms / ms, "speedup_reuse_vs_dense": dense_ms / reuse_ms,
+        w3 = config_work(cl)
+        extras = {"refine_ms": ms_max, "reuse_ms": reuse_ms, "dense_ms": dense_ms, "decode": decode,
+                  "speedup_refine_vs_dense": dense_ms / ms_max, "speedup_reuse_vs_dense": dense_ms / reuse_ms,
                   "recall_at_k_vs_dense": rec, "recall_rows": int(rows.numel()),
                   "roofline_ms": {"refine": roofline_ms(w3["refine"], pk), "reuse": roofline_ms(w3["reuse"], pk),
                                   "dense": roofline_ms(w3["dense"], pk)},
-                  "roofline_frac": {"refine": roofline_ms(w3["refine"], pk) / ms,
+                  "roofline_frac": {"refine": roofline_ms(w3["refine"], pk) / ms_max,
                                     "reuse": roofline_ms(w3["reuse"], pk) / reuse_ms,
                                     "dense": roofline_ms(w3["dense"], pk) / dense_ms}}
         del out_reuse
-        if not args.no_configs:
+        if not args.no_configs and world == 1:
             del out
             torch.cuda.empty_cache()
             extras["configs"] = config_records(qg, torch, stream, pk, max(3, args.steps))
@@ -600,9 +639,9 @@ def main():
         oracle.build()
         cpu = cpu_baseline(c, q_np, k_np) if (world == 1 and not args.no_cpu_baseline) else None
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(c),
-                "roofline": roof, "scan_tflops": scan_tf, "kernels": kern, "gpu_launches": gpu_launches,
+                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(c, world),
+                "roofline": roof, "scan": scan_rec, "kernels": kern, "gpu_launches": gpu_launches,
                 "status_flags": flags, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "extras": extras}
         print(json.dumps(line), flush=True)
     ranks.close()

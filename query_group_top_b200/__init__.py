@@ -18,7 +18,8 @@ import os
 import torch
 
 __all__ = ["REFINE", "REUSE", "PivotError", "pivot_index", "dense_index", "pivot_decode_index",
-           "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED"]
+           "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED",
+           "head_range"]
 
 REFINE, REUSE = 0, 1
 PROXY_BF16 = 0x100          # option bit of `mode`: scan with the bf16-rounded mean
@@ -255,3 +256,16 @@ def sync_status(stream=None) -> int:
     rc = lib.pivot_sync_status(_stream_ptr(stream), ctypes.byref(flags))
     _err(lib, rc)
     return flags.value
+
+
+def head_range(H: int, rank: int, world: int) -> tuple:
+    """Heads [h0, h1) of an H-head layer that rank `rank` of `world` indexes
+    when the indexer is split across GPUs by head.  Every head's proxy, scan,
+    candidate set and refine read only that head's queries and keys ("PIVOT
+    explained", "Show Me The Code": the loop over heads), so the ranks exchange
+    nothing; each indexes its heads as an [L, h1-h0, d] layer of its own.  The
+    ranges are contiguous, in rank order, cover every head once and differ in
+    size by at most one head."""
+    if H < 1 or world < 1 or not 0 <= rank < world:
+        raise ValueError(f"head_range: need H >= 1 and 0 <= rank < world (H={H}, rank={rank}, world={world})")
+    return rank * H // world, (rank + 1) * H // world

@@ -158,7 +158,7 @@ def make_prefill(name: str):
 
 def gen_decode_device(B: int, H: int, d: int, g: int, seed: int, lo: int, hi: int,
                       rho: float = 0.95, heavy_frac: float = 0.01, heavy_scale: float = 4.0,
-                      device="cuda"):
+                      device="cuda", first: int = 0, count=None):
     """Large decode batches drawn on the GPU (same recipe as ``gen_decode``).
 
     Context lengths, heavy-key positions and the step queries come from numpy
@@ -167,30 +167,37 @@ def gen_decode_device(B: int, H: int, d: int, g: int, seed: int, lo: int, hi: in
     then rounded to bf16 (round to nearest even).  Returns torch tensors
     (q [B,g,H,d] bf16, kcache [rows,H,d] bf16, cu_seqlens [B+1] int32) on the
     device and the numpy context lengths.  Use ``kcache[cu[b]:cu[b+1]]`` to
-    read a sequence back for a CPU check.
+    read a sequence back for a CPU check.  ``first`` and ``count`` draw only
+    sequences [first, first+count) of the B-sequence batch (the same values
+    as in the whole batch), packed from cache row 0.
     """
     import torch
     rng = np.random.default_rng(seed)
-    n_ctx = rng.integers(lo, hi, size=B, endpoint=True).astype(np.int32)
+    n_all = rng.integers(lo, hi, size=B, endpoint=True).astype(np.int32)
+    count = B - first if count is None else count
+    if not 0 <= first <= first + count <= B:
+        raise ValueError("gen_decode_device: sequences out of range")
+    n_ctx = n_all[first:first + count]
+    seqs = range(first, first + count)
     lens = n_ctx.astype(np.int64) + g
-    cu = np.zeros(B + 1, dtype=np.int64)
+    cu = np.zeros(count + 1, dtype=np.int64)
     cu[1:] = np.cumsum(lens)
     if cu[-1] >= 2**31:
         raise ValueError("decode cache too large for int32 offsets")
     kc = torch.empty((int(cu[-1]), H, d), dtype=torch.bfloat16, device=device)
-    q = np.empty((B, g, H, d), dtype=np.uint16)
+    q = np.empty((count, g, H, d), dtype=np.uint16)
     a = np.float32(rho)
     b_ = np.float32(math.sqrt(1.0 - rho * rho))
     gen = torch.Generator(device=device)
-    for b in range(B):
-        n = int(lens[b])
+    for i_b, b in enumerate(seqs):
+        n = int(lens[i_b])
         gen.manual_seed(seed * 1000003 + b)
         kb = torch.randn((n, H, d), generator=gen, device=device, dtype=torch.float32)
         n_heavy = int(round(heavy_frac * n))
         if n_heavy > 0:
             pos = np.random.default_rng([seed, b]).choice(n, size=n_heavy, replace=False)
             kb[torch.from_numpy(pos).to(device)] *= heavy_scale
-        kc[int(cu[b]):int(cu[b + 1])] = kb.to(torch.bfloat16)
+        kc[int(cu[i_b]):int(cu[i_b + 1])] = kb.to(torch.bfloat16)
         del kb
         rq = np.random.default_rng([seed, b, 1])
         eps = rq.standard_normal((g, H, d), dtype=np.float32)
@@ -198,7 +205,7 @@ def gen_decode_device(B: int, H: int, d: int, g: int, seed: int, lo: int, hi: in
         qq[0] = eps[0]
         for i in range(1, g):
             qq[i] = a * qq[i - 1] + b_ * eps[i]
-        q[b] = bf16_from_f32(qq)
+        q[i_b] = bf16_from_f32(qq)
     qd = torch.from_numpy(q.view(np.int16)).to(device).view(torch.bfloat16)
     cud = torch.from_numpy(cu.astype(np.int32)).to(device)
     return qd, kc, cud, n_ctx

@@ -5,7 +5,7 @@
   rows, candidate rows and one read of q and k);
 * DRAM traffic is taken from the committed one-head capture only while the
   refine source is the one that was captured, and scaled by the heads;
-* the weak-scaling throughput and the clock-sample summary.
+* the job throughput of a head-split layer and the clock-sample summary.
 """
 import hashlib
 import os
@@ -54,10 +54,10 @@ def test_traffic_follows_the_captured_source(tmp_path, monkeypatch):
     assert bench.measured_traffic("refine", 16) is None
 
 
-def test_weak_scaling_value():
-    # every rank indexes its own L x H layer; the job takes its slowest rank's time
-    assert bench.weak_value(1, 131072, 16, 50.0) == 131072 * 16 / 0.05
-    assert bench.weak_value(4, 1024, 8, 2.0) == 4 * 1024 * 8 / 0.002
+def test_job_value_of_a_head_split_layer():
+    # the ranks together index one L x H layer; the job takes its slowest rank's time
+    assert bench.job_value(131072, 16, 50.0) == 131072 * 16 / 0.05
+    assert bench.job_value(1024, 8, 2.0) == 1024 * 8 / 0.002
 
 
 def test_clock_summary_flags_throttle_reasons():
