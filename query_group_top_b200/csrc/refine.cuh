@@ -216,19 +216,33 @@ __device__ __forceinline__ int warp_rank_bin(const uint32_t* h, int r, int lane,
   }
   const unsigned hit = __ballot_sync(0xffffffffu, incl >= r);
   const int L = hit ? __ffs(hit) - 1 : 31;
-  int cum = __shfl_sync(0xffffffffu, incl - s, L);
-  int bin = NBINS - PER * L - PER;  // (the counts always reach r)
+  const int cum = __shfl_sync(0xffffffffu, incl - s, L);   // counts above group L
   const int bL = NBINS - PER * (L + 1);
-  for (int i = PER - 1; i >= 0; --i) {
-    const int c = static_cast<int>(h[bL + i]);
-    if (cum + c >= r) {
-      bin = bL + i;
-      break;
-    }
-    cum += c;
+  // group L's bins, one per lane, summed from the top bin down: the answer is
+  // the highest bin whose suffix (plus the counts above the group) reaches r
+  const int c = lane < PER ? static_cast<int>(h[bL + lane]) : 0;
+  int suf = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
   }
-  *above = cum;
-  return bin;
+  const unsigned ok = __ballot_sync(0xffffffffu, lane < PER && cum + suf >= r);
+  const int i = ok ? 31 - __clz(ok) : 0;   // (the counts always reach r)
+  *above = cum + __shfl_sync(0xffffffffu, suf - c, i);
+  return bL + i;
+}
+
+// v[j] for a lane-varying j in [0, 16), by a tree of selects (no local memory).
+__device__ __forceinline__ uint32_t pick16(const uint32_t (&v)[16], int j) {
+  uint32_t w8[8], w4[4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w8[i] = (j & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w4[i] = (j & 2) ? w8[2 * i + 1] : w8[2 * i];
+  const uint32_t w0 = (j & 4) ? w4[1] : w4[0];
+  const uint32_t w1 = (j & 4) ? w4[3] : w4[2];
+  return (j & 8) ? w1 : w0;
 }
 
 // One work item: a unit's batch of up to 16 members.
@@ -657,41 +671,44 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         for (int j = 0; j < 16; ++j) reg_fence(v[j]);
         if (!keep_tmem) release(c);
         const int base_t = c * 128 + q * 32;
-        const bool partial = base_t + 32 > nvmin;   // some classified member cannot use every lane
-        uint32_t lm[16];
-        uint32_t my_above = 0u, my_n = 0u;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float f = __uint_as_float(v[j]);
-          uint32_t a = __ballot_sync(0xffffffffu, f >= th[j]);
-          uint32_t b = __ballot_sync(0xffffffffu, f >= tl[j]);
-          if (partial) {
-            const int u = M->ms[j].nv - base_t;
-            const uint32_t um = u >= 32 ? 0xFFFFFFFFu : (u <= 0 ? 0u : ((1u << u) - 1u));
-            a &= um;
-            b &= um;
-          }
-          lm[j] = b & ~a;
-          my_above = lane == j ? a : my_above;
-          my_n = lane == j ? static_cast<uint32_t>(__popc(lm[j])) : my_n;
-        }
-        // lane j < 16: member j's bitmap word and list reservation
-        if (lane < 16) bmp[(c * 4 + q) * 16 + lane] = my_above;
-        if (__any_sync(0xffffffffu, my_n != 0u)) {
-          uint32_t base = 0u;
-          if (lane < 16 && my_n != 0u) base = atom_shared_add(smem_u32(&M->ms[lane].nlist), my_n);
-          const uint16_t slot = static_cast<uint16_t>(base_t + lane);
+        const int t = base_t + lane;
+        // member j: the ">= hi" lanes by one vote (its bitmap word), the lanes
+        // in [lo, hi) as bit j of this lane's band mask
+        uint32_t a[16];
+        uint32_t bm = 0u;
+        if (base_t + 32 <= nvmin) {   // every classified member can use every lane
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (lm[j] != 0u) {   // the same for every lane: boundary keys are few
-              const uint32_t at = min(__shfl_sync(0xffffffffu, base, j) + static_cast<uint32_t>(__popc(lm[j] & ltmask)),
-                                      static_cast<uint32_t>(kCap - 1));
-              if ((lm[j] >> lane) & 1u) {
-                st_shared_u32_nb(lk_s + 4u * (j * kCap + at), v[j]);
-                st_shared_u16_nb(ls_s + 2u * (j * kCap + at), slot);
-              }
-            }
+            const float f = __uint_as_float(v[j]);
+            const bool above = f >= th[j];
+            a[j] = __ballot_sync(0xffffffffu, above);
+            bm |= (!above && f >= tl[j]) ? (1u << j) : 0u;
           }
+        } else {                      // a member's usable prefix ends in this slice
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float f = __uint_as_float(v[j]);
+            const bool use = t < M->ms[j].nv;
+            const bool above = use && f >= th[j];
+            a[j] = __ballot_sync(0xffffffffu, above);
+            bm |= (use && !above && f >= tl[j]) ? (1u << j) : 0u;
+          }
+        }
+        if (lane == 0) {
+          uint4* w = reinterpret_cast<uint4*>(bmp + (c * 4 + q) * 16);
+          w[0] = make_uint4(a[0], a[1], a[2], a[3]);
+          w[1] = make_uint4(a[4], a[5], a[6], a[7]);
+          w[2] = make_uint4(a[8], a[9], a[10], a[11]);
+          w[3] = make_uint4(a[12], a[13], a[14], a[15]);
+        }
+        // this lane's boundary keys onto their members' lists (a boundary bin
+        // holds a few keys of the member's candidates, so few lanes loop)
+        while (bm != 0u) {
+          const int j = __ffs(bm) - 1;
+          bm &= bm - 1u;
+          const uint32_t at = min(atom_shared_add(smem_u32(&M->ms[j].nlist), 1u), static_cast<uint32_t>(kCap - 1));
+          st_shared_u32_nb(lk_s + 4u * (j * kCap + at), pick16(v, j));
+          st_shared_u16_nb(ls_s + 2u * (j * kCap + at), static_cast<uint16_t>(t));
         }
       }
       if (named_barrier_or(2, C::NSEL, !ok)) break;
@@ -864,6 +881,39 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         int32_t* out_row = p.out + orow * p.top_k;
         if (mode == kMAll) {
           for (int t = lane; t < K; t += 32) out_row[t] = cx[t];
+        } else if (mode == kMBand && (p.top_k & 3) == 0) {
+          // The row gathers in a 256-entry ring in this warp's own list space
+          // (free once its list is ranked) and leaves 128 indices (512 bytes)
+          // per 16-byte-per-lane store: far fewer global stores than one per
+          // bitmap word.  Rows start 16-byte aligned (out is, top_k % 4 == 0).
+          int32_t* ring = reinterpret_cast<int32_t*>(lkeys + sw * kCap);
+          int staged = 0, flushed = 0;   // uniform across the warp
+#pragma unroll 1
+          for (int w0 = 0; w0 < nch * 4; w0 += 4) {
+            uint32_t wd[4];
+            int32_t val[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              wd[x] = mb[16 * (w0 + x)];
+              val[x] = cx[(w0 + x) * 32 + lane];
+            }
+            // at most 128 new entries on fewer than 128 pending: the ring
+            // never overwrites an entry that has not left
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              if ((wd[x] >> lane) & 1u) ring[(staged + __popc(wd[x] & ltmask)) & 255] = val[x];
+              staged += __popc(wd[x]);
+            }
+            if (staged - flushed >= 128) {
+              __syncwarp();
+              const int4 v4 = reinterpret_cast<const int4*>(ring + (flushed & 255))[lane];
+              reinterpret_cast<int4*>(out_row + flushed)[lane] = v4;
+              flushed += 128;
+              __syncwarp();
+            }
+          }
+          __syncwarp();
+          for (int t = flushed + lane; t < staged; t += 32) out_row[t] = ring[t & 255];
         } else if (mode == kMBand) {
           int base = 0;
 #pragma unroll 1
