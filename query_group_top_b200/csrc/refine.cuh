@@ -200,12 +200,14 @@ __device__ __forceinline__ uint32_t warp_first_key_of_bin(int b, float scale, fl
 template <int NBINS>
 __device__ __forceinline__ int warp_rank_bin(const uint32_t* h, int r, int lane, int* above) {
   constexpr int PER = NBINS / 32;
-  static_assert(PER % 4 == 0, "bins are read four at a time");
+  static_assert(PER % 4 == 0 && ((PER / 4) & (PER / 4 - 1)) == 0, "bins are read four at a time, 2^n reads per lane");
   const int b0 = NBINS - PER * (lane + 1);
   int s = 0;
+  // lane l starts its 16-byte reads at a rotated offset: the lanes' groups lie
+  // PER words apart, so unrotated reads would all hit the same banks
 #pragma unroll
   for (int i = 0; i < PER / 4; ++i) {
-    const uint4 x = reinterpret_cast<const uint4*>(h + b0)[i];
+    const uint4 x = reinterpret_cast<const uint4*>(h + b0)[(i + lane) & (PER / 4 - 1)];
     s += static_cast<int>(x.x + x.y + x.z + x.w);
   }
   int incl = s;
@@ -881,39 +883,6 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         int32_t* out_row = p.out + orow * p.top_k;
         if (mode == kMAll) {
           for (int t = lane; t < K; t += 32) out_row[t] = cx[t];
-        } else if (mode == kMBand && (p.top_k & 3) == 0) {
-          // The row gathers in a 256-entry ring in this warp's own list space
-          // (free once its list is ranked) and leaves 128 indices (512 bytes)
-          // per 16-byte-per-lane store: far fewer global stores than one per
-          // bitmap word.  Rows start 16-byte aligned (out is, top_k % 4 == 0).
-          int32_t* ring = reinterpret_cast<int32_t*>(lkeys + sw * kCap);
-          int staged = 0, flushed = 0;   // uniform across the warp
-#pragma unroll 1
-          for (int w0 = 0; w0 < nch * 4; w0 += 4) {
-            uint32_t wd[4];
-            int32_t val[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              wd[x] = mb[16 * (w0 + x)];
-              val[x] = cx[(w0 + x) * 32 + lane];
-            }
-            // at most 128 new entries on fewer than 128 pending: the ring
-            // never overwrites an entry that has not left
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              if ((wd[x] >> lane) & 1u) ring[(staged + __popc(wd[x] & ltmask)) & 255] = val[x];
-              staged += __popc(wd[x]);
-            }
-            if (staged - flushed >= 128) {
-              __syncwarp();
-              const int4 v4 = reinterpret_cast<const int4*>(ring + (flushed & 255))[lane];
-              reinterpret_cast<int4*>(out_row + flushed)[lane] = v4;
-              flushed += 128;
-              __syncwarp();
-            }
-          }
-          __syncwarp();
-          for (int t = flushed + lane; t < staged; t += 32) out_row[t] = ring[t & 255];
         } else if (mode == kMBand) {
           int base = 0;
 #pragma unroll 1
