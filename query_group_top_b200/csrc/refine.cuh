@@ -499,12 +499,26 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
       const int nch = it.nch, nb = it.nb;
       const int32_t* cx = cidx0 + buf * CW;
       if (ok) ok = mbar_wait(smem_u32(&M->cready[buf]), (kk >> 1) & 1, abort_flag, p.status, p.wait_ns);
+      ok = __all_sync(0xffffffffu, ok);
       // ---- per-member usable counts (the candidate set is ascending) and modes
-      if (stid < 16 && ok) {
-        MemberSel& S = M->ms[stid];
+      if (sw == 0 && ok) {
+        // member m (lane m) uses the candidates below its position.  The row
+        // is ascending and its entries at or past member 0's position are the
+        // group's own keys at its end, so when the last 32 entries hold them
+        // all, one vote per member counts them; else a binary search does
+        const int first = it.pos0 + it.mb;
+        const int e = it.nc - 32 + lane;
+        const int ce = e >= 0 ? cx[e] : -1;
+        const bool covered = it.nc <= 32 || __shfl_sync(0xffffffffu, ce, 0) < first;
         int nv = 0;
-        if (stid < nb) {
-          const int pos = it.pos0 + it.mb + stid;
+        if (covered) {
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const int past = __popc(__ballot_sync(0xffffffffu, ce >= first + m));
+            if (lane == m) nv = it.nc - past;
+          }
+        } else if (lane < 16) {
+          const int pos = first + lane;
           int lo = 0, hi = it.nc;
           while (lo < hi) {
             const int mid = (lo + hi) >> 1;
@@ -513,29 +527,36 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
           }
           nv = lo;
         }
-        const int K = min(p.top_k, nv);
-        S.nv = nv;
-        S.K = K;
-        S.mode = K == 0 ? kMNone : (K == nv ? kMAll : kMBand);
-        S.nlist = 0;
-        S.need = 0;
-        S.lo = kInf;   // None and All take no list; Band is set below
-        S.hi = kInf;
-        S.kmin = 0xFFFFFFFFu;
-        S.kmax = 0u;
+        if (lane < 16) {
+          if (lane >= nb) nv = 0;
+          MemberSel& S = M->ms[lane];
+          const int K = min(p.top_k, nv);
+          S.nv = nv;
+          S.K = K;
+          S.mode = K == 0 ? kMNone : (K == nv ? kMAll : kMBand);
+          S.nlist = 0;
+          S.need = 0;
+          S.lo = kInf;   // None and All take no list; Band is set below
+          S.hi = kInf;
+          S.kmin = 0xFFFFFFFFu;
+          S.kmax = 0u;
+        }
       }
       // bitmaps and histograms start at zero
       for (int i = stid; i < (C::BMP_BYTES + 16 * kBins * 4) / 16; i += C::NSEL)
         reinterpret_cast<uint4*>(bmp)[i] = make_uint4(0, 0, 0, 0);
       if (named_barrier_or(2, C::NSEL, !ok)) break;
-      bool anyb = false;       // a member that needs a selection (uniform)
-      int nvmin = 0x7FFFFFFF;  // fewest usable candidates of such a member (uniform)
-      for (int m = 0; m < 16; ++m) {
-        if (M->ms[m].mode == kMBand) {
-          anyb = true;
-          nvmin = min(nvmin, M->ms[m].nv);
-        }
+      // the members that need a selection (bit m), and the fewest usable
+      // candidates among them: one read per lane, one vote (uniform values)
+      uint32_t bandm;
+      int nvmin;
+      {
+        const MemberSel& S = M->ms[lane & 15];
+        const bool band = S.mode == kMBand;
+        bandm = __ballot_sync(0xffffffffu, band) & 0xFFFFu;
+        nvmin = static_cast<int>(__reduce_min_sync(0xffffffffu, band ? static_cast<uint32_t>(S.nv) : 0x7FFFFFFFu));
       }
+      const bool anyb = bandm != 0u;
 
       if (anyb) {
         // ---- chunk 0's score range sets each member's histogram bins
@@ -548,11 +569,12 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             tmem_ld_32x32b_x16(tq, v);
             tmem_ld_wait();
             const int t = q * 32 + lane;
+            const bool all_use = 128 <= nvmin;   // chunk 0 lies inside every member's usable prefix
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               reg_fence(v[j]);
-              if (M->ms[j].mode == kMBand) {
-                const bool use = t < M->ms[j].nv;
+              if ((bandm >> j) & 1u) {
+                const bool use = all_use || t < M->ms[j].nv;
                 const uint32_t key = score_key(__uint_as_float(v[j]));
                 const uint32_t mn = __reduce_min_sync(0xffffffffu, use ? key : 0xFFFFFFFFu);
                 const uint32_t mx = __reduce_max_sync(0xffffffffu, use ? key : 0u);
@@ -884,18 +906,22 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
         if (mode == kMAll) {
           for (int t = lane; t < K; t += 32) out_row[t] = cx[t];
         } else if (mode == kMBand) {
+          // eight 32-candidate words per round: their shared-memory reads go
+          // out together, so a round waits for one read latency, not eight
+          const int nw = nch * 4;
           int base = 0;
 #pragma unroll 1
-          for (int w0 = 0; w0 < nch * 4; w0 += 4) {
-            uint32_t wd[4];
-            int32_t val[4];
+          for (int w0 = 0; w0 < nw; w0 += 8) {
+            uint32_t wd[8];
+            int32_t val[8];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              wd[x] = mb[16 * (w0 + x)];
-              val[x] = cx[(w0 + x) * 32 + lane];
+            for (int x = 0; x < 8; ++x) {
+              const bool inw = w0 + x < nw;
+              wd[x] = inw ? mb[16 * (w0 + x)] : 0u;
+              val[x] = inw ? cx[(w0 + x) * 32 + lane] : 0;
             }
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
+            for (int x = 0; x < 8; ++x) {
               if ((wd[x] >> lane) & 1u) out_row[base + __popc(wd[x] & ltmask)] = val[x];
               base += __popc(wd[x]);
             }
