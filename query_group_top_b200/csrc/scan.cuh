@@ -113,7 +113,10 @@ scan_filter_kernel(const __grid_constant__ CUtensorMap tm_proxy, const __grid_co
                    ScanParams p) {
   using C = ScanCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte alignment by an offset from the shared array itself, so that
+  // every pointer derived from it stays a shared-space pointer (plain shared
+  // loads and stores rather than generic ones)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sA = sbase + C::OFF_A;
   const uint32_t sB = sbase + C::OFF_B;
