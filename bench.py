@@ -105,10 +105,13 @@ def roofline_ms(work, pk):
     return max(work["bytes"] / (pk["hbm"] * 1e9), work["flops"] / (pk["bf16"] * 1e12)) * 1e3
 
 
-def config_records(qg, torch, stream, pk, steps, names=("C0", "C1", "C2")):
+def config_records(qg, torch, stream, pk, steps, names=("C0", "C1", "C2"), member_names=("C0", "C1")):
     """Refine, Reuse and dense on the smaller prefill workloads: ms per call,
     query-heads/s, the fraction of each call's roofline, PIVOT's speedup over
-    the dense indexer and Recall@k against it (on a seeded sample of rows)."""
+    the dense indexer and Recall@k against it (on a seeded sample of rows).
+    On `member_names` also the per-member-scan variant of Refine (each member's
+    own top-Kc candidates over its prefix), whose recall change is the point
+    of that variant."""
     recs = {}
     for name in names:
         c = synthetic.CONFIGS[name]
@@ -120,6 +123,9 @@ def config_records(qg, torch, stream, pk, steps, names=("C0", "C1", "C2")):
         calls = {"refine": lambda o: qg.pivot_index(q, k, g, top_k, Kc, qg.REFINE, out=o),
                  "reuse": lambda o: qg.pivot_index(q, k, g, top_k, Kc, qg.REUSE, out=o),
                  "dense": lambda o: qg.dense_index(q, k, top_k, out=o)}
+        if name in member_names:
+            calls["refine_member_scan"] = lambda o: qg.pivot_index(q, k, g, top_k, Kc, qg.REFINE, out=o,
+                                                                   scan="member")
         for mode, fn in calls.items():
             o = torch.empty((L, H, top_k), dtype=torch.int32, device="cuda")
             for _ in range(2):
@@ -140,7 +146,7 @@ def config_records(qg, torch, stream, pk, steps, names=("C0", "C1", "C2")):
         heads = torch.from_numpy(rng.integers(0, H, size=n)).cuda()
         dn = outs["dense"][rows, heads].cpu().numpy()
         rec = {}
-        for mode in ("refine", "reuse"):
+        for mode in [m for m in outs if m != "dense"]:
             pv = outs[mode][rows, heads].cpu().numpy()
             rec[mode] = float(np.mean([np.intersect1d(a[a >= 0], b[b >= 0]).size / max(1, (b >= 0).sum())
                                        for a, b in zip(pv, dn)]))
@@ -149,9 +155,9 @@ def config_records(qg, torch, stream, pk, steps, names=("C0", "C1", "C2")):
             "shape": f"L={L} H={H} d={d} g={g} top_k={top_k} Kc={Kc}",
             "ms": ms,
             "query_heads_per_s": {m: L * H / (v / 1000.0) for m, v in ms.items()},
-            "roofline_ms": {m: roofline_ms(work[m], pk) for m in ms},
-            "roofline_frac": {m: roofline_ms(work[m], pk) / ms[m] for m in ms},
-            "speedup_vs_dense": {"refine": ms["dense"] / ms["refine"], "reuse": ms["dense"] / ms["reuse"]},
+            "roofline_ms": {m: roofline_ms(work[m], pk) for m in ms if m in work},
+            "roofline_frac": {m: roofline_ms(work[m], pk) / ms[m] for m in ms if m in work},
+            "speedup_vs_dense": {m: ms["dense"] / v for m, v in ms.items() if m != "dense"},
             "recall_at_k_vs_dense": rec, "recall_rows": int(n)}
         del outs, q, k
         torch.cuda.empty_cache()

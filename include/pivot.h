@@ -52,6 +52,19 @@ typedef enum { PIVOT_REFINE = 0, PIVOT_REUSE = 1 } pivot_mode_t;
  */
 enum { PIVOT_PROXY_BF16 = 0x100 };
 
+/*
+ * Option bit OR-ed into PIVOT_REFINE (prefill entry points only): the
+ * listing's reading of Refine ("Show Me The Code", pivot_refine, which scans
+ * k[:pos] for each member): member pos takes its candidate set from the group
+ * proxy's scores over its own prefix j < pos, instead of one set per group
+ * over j < last.  A fidelity variant, not the method's one shared scan: the
+ * scan runs once per member (rows = positions) and every member gathers its
+ * own candidates.  Its candidate rows hold L*H*ceil(Kc/128)*128 int32 of the
+ * workspace; out_cand (when given) is then [L,H,Kc].  Decode entry points and
+ * PIVOT_REUSE return PIVOT_ERR_INVALID_ARG with this bit.
+ */
+enum { PIVOT_PER_MEMBER_SCAN = 0x200 };
+
 typedef enum {
   PIVOT_OK = 0,
   PIVOT_ERR_INVALID_ARG = 1,

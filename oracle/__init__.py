@@ -52,7 +52,7 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         P = ctypes.c_void_p
         i = ctypes.c_int
-        lib.oracle_prefill_units.argtypes = [P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P]
+        lib.oracle_prefill_units.argtypes = [P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_dense_units.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P]
         lib.oracle_decode_units.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P]
         for f in (lib.oracle_prefill_units, lib.oracle_dense_units, lib.oracle_decode_units):
@@ -83,8 +83,9 @@ def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False, prox
     listed (group, head) units; `proxy` is the scan operand's precision.
 
     Returns dict: out [n,g,top_k] int32, score [n,g,top_k] f64, edge [n,g,2] f64,
-    cand [n,Kc] int32 and cand_edge [n,2] (Refine), proxy [n,d] float32 (the
-    fp32 mean) and proxy_bf16 [n,d] uint16 (its bf16 rounding).
+    cand [n,Kc] int32 and cand_edge [n,2] (Refine), member_cand_edge [n,g,2]
+    (mode 2: each member's own Kc-th and (Kc+1)-th proxy scores), proxy [n,d]
+    float32 (the fp32 mean) and proxy_bf16 [n,d] uint16 (its bf16 rounding).
     """
     lib = _load()
     pb = _proxy_flag(proxy)
@@ -101,11 +102,13 @@ def prefill_units(q, k, g, top_k, Kc, mode, groups, heads, want_cand=False, prox
     cedge = np.empty((n, 2), np.float64)
     p32 = np.empty((n, d), np.float32)
     p16 = np.empty((n, d), np.uint16)
+    medge = np.empty((n, g, 2), np.float64)
     rc = lib.oracle_prefill_units(_p(q), _p(k), L, H, d, g, top_k, Kc, mode, pb, n, _p(groups), _p(heads),
-                                  _p(out), _p(sc), _p(edge), _p(cand), _p(cedge), _p(p32), _p(p16))
+                                  _p(out), _p(sc), _p(edge), _p(cand), _p(cedge), _p(p32), _p(p16), _p(medge))
     if rc != 0:
         raise ValueError("oracle_prefill_units rejected its arguments")
-    return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, proxy=p32, proxy_bf16=p16)
+    return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, member_cand_edge=medge, proxy=p32,
+                proxy_bf16=p16)
 
 
 def prefill(q, k, g, top_k, Kc, mode, want_cand=False, proxy="fp32"):
@@ -120,6 +123,7 @@ def prefill(q, k, g, top_k, Kc, mode, want_cand=False, proxy="fp32"):
         a = np.swapaxes(a, 1, 2).reshape(G * g, H, *a.shape[3:])
         return np.ascontiguousarray(a[:L])
     res = dict(out=fold(r["out"]), score=fold(r["score"]), edge=fold(r["edge"]),
+               member_cand_edge=fold(r["member_cand_edge"]),
                cand_edge=r["cand_edge"].reshape(G, H, 2), proxy=r["proxy"].reshape(G, H, -1),
                proxy_bf16=r["proxy_bf16"].reshape(G, H, -1))
     if want_cand:

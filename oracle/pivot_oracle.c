@@ -156,7 +156,8 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
                      const uint16_t *kbase, long kstride, int d, int s, int last,
                      int top_k, int Kc, int mode, int proxy_bf16,
                      int32_t *out, double *out_sc, double *edge,
-                     int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb)
+                     int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb,
+                     double *mcand_edge)
 {
     double *p = (double *)malloc(sizeof(double) * (size_t)d);
     int bound = (mode == 1) ? s : last;
@@ -179,6 +180,7 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
     }
     if (cand) for (int t = 0; t < Kc; ++t) cand[t] = -1;
     if (cand_edge) { cand_edge[0] = NAN; cand_edge[1] = NAN; }
+    if (mcand_edge) for (int m = 0; m < 2 * g; ++m) mcand_edge[m] = NAN;
 
     if (mode == 1) {
         /* Reuse: the proxy's top-k over j < s, shared by every member. */
@@ -199,7 +201,7 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
         for (int m = 0; m < nm; ++m) {
             int pos = mpos[m];
             memcpy(own, sig, sizeof(scored_t) * (size_t)pos);
-            int nC = select_top(own, pos, Kc, Kc, C, NULL, NULL);
+            int nC = select_top(own, pos, Kc, Kc, C, NULL, mcand_edge ? mcand_edge + 2 * m : NULL);
             for (int t = 0; t < nC; ++t) {
                 v[t].j = C[t];
                 v[t].s = dot(mq[m], kbase + (long)C[t] * kstride, d);
@@ -240,13 +242,16 @@ static int one_group(const uint16_t *const *mq, const int32_t *mpos, int nm, int
  * Per unit u: out [g, top_k] (member m = position i*g + m), out_sc [g, top_k]
  * (nullable), edge [g, 2] (nullable), cand [Kc] (nullable), cand_edge [2]
  * (nullable), proxy32 [d] fp32 mean (nullable), proxyb [d] its bf16 rounding
- * (nullable).  Returns 0, or -1 on bad arguments.
+ * (nullable), mcand_edge [g, 2] (nullable; mode 2 only): each member's own
+ * Kc-th and (Kc+1)-th proxy scores over its prefix.  Returns 0, or -1 on bad
+ * arguments.
  */
 int oracle_prefill_units(const uint16_t *q, const uint16_t *k, int L, int H, int d,
                          int g, int top_k, int Kc, int mode, int proxy_bf16,
                          int n_units, const int32_t *unit_group, const int32_t *unit_head,
                          int32_t *out, double *out_sc, double *edge,
-                         int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb)
+                         int32_t *cand, double *cand_edge, float *proxy32, uint16_t *proxyb,
+                         double *mcand_edge)
 {
     if (L < 1 || H < 1 || d < 1 || g < 1 || top_k < 1 || Kc < top_k || mode < 0 || mode > 2 ||
         proxy_bf16 < 0 || proxy_bf16 > 1)
@@ -271,7 +276,8 @@ int oracle_prefill_units(const uint16_t *q, const uint16_t *k, int L, int H, int
                        cand ? cand + (long)u * Kc : NULL,
                        cand_edge ? cand_edge + (long)u * 2 : NULL,
                        proxy32 ? proxy32 + (long)u * d : NULL,
-                       proxyb ? proxyb + (long)u * d : NULL);
+                       proxyb ? proxyb + (long)u * d : NULL,
+                       mcand_edge ? mcand_edge + (long)u * g * 2 : NULL);
     }
     free(mq); free(mpos);
     return rc;
@@ -340,7 +346,7 @@ int oracle_decode_units(const uint16_t *q, const uint16_t *kcache, const int32_t
                        cand ? cand + (long)u * Kc : NULL,
                        cand_edge ? cand_edge + (long)u * 2 : NULL,
                        proxy32 ? proxy32 + (long)u * d : NULL,
-                       proxyb ? proxyb + (long)u * d : NULL);
+                       proxyb ? proxyb + (long)u * d : NULL, NULL);
     }
     free(mq); free(mpos);
     return rc;

@@ -17,12 +17,13 @@ import os
 
 import torch
 
-__all__ = ["REFINE", "REUSE", "PivotError", "pivot_index", "dense_index", "pivot_decode_index",
+__all__ = ["REFINE", "REUSE", "PROXY_BF16", "PER_MEMBER_SCAN", "PivotError", "pivot_index", "dense_index", "pivot_decode_index",
            "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED",
            "head_range"]
 
 REFINE, REUSE = 0, 1
 PROXY_BF16 = 0x100          # option bit of `mode`: scan with the bf16-rounded mean
+PER_MEMBER_SCAN = 0x200     # option bit of REFINE: each member's own-prefix candidate set
 FLAG_TIMEOUT, FLAG_BADLEN, FLAG_FALLBACK, FLAG_NOCONVERGE = 1, 2, 4, 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -124,12 +125,14 @@ def _out(out, shape, dtype, device, name):
     return out
 
 
-def _mode_bits(mode, proxy):
+def _mode_bits(mode, proxy, scan="group"):
     if mode not in (REFINE, REUSE):
         raise PivotError("mode must be REFINE or REUSE")
     if proxy not in ("fp32", "bf16"):
         raise PivotError('proxy must be "fp32" (the method) or "bf16" (the variant)')
-    return mode | (PROXY_BF16 if proxy == "bf16" else 0)
+    if scan not in ("group", "member") or (scan == "member" and mode != REFINE):
+        raise PivotError('scan must be "group" (the method) or, with REFINE, "member" (the listing\'s variant)')
+    return mode | (PROXY_BF16 if proxy == "bf16" else 0) | (PER_MEMBER_SCAN if scan == "member" else 0)
 
 
 def _ptr(t):
@@ -137,16 +140,18 @@ def _ptr(t):
 
 
 def pivot_index(q, k, g, top_k, Kc, mode=REFINE, out=None, out_scores=None, stream=None, proxy="fp32",
-                out_proxy=None, out_cand=None):
+                out_proxy=None, out_cand=None, scan="group"):
     """PIVOT prefill indexer: q, k bf16 [L, H, d] -> int32 [L, H, top_k] (ascending, -1 padded).
 
     proxy: "fp32" scans with the fp32 group mean (the method), "bf16" with its
-    bf16 rounding (a variant).  out_proxy (float32 [G, H, d]) and out_cand
-    (int32 [G, H, Kc], Refine only) receive the groups' proxies and candidate
-    sets when given (G = ceil(L / g)).
+    bf16 rounding (a variant).  scan: "group" takes one candidate set per
+    group (the method), "member" (Refine only) each member's own top-Kc over
+    its prefix (the listing's variant).  out_proxy (float32 [G, H, d]) and
+    out_cand (int32 [G, H, Kc], Refine only; [L, H, Kc] with scan="member")
+    receive the groups' proxies and candidate sets when given (G = ceil(L / g)).
     """
     lib = load_library()
-    bits = _mode_bits(mode, proxy)
+    bits = _mode_bits(mode, proxy, scan)
     _check_bf16("q", q, 3)
     _check_bf16("k", k, 3)
     if q.shape != k.shape:
@@ -159,7 +164,7 @@ def pivot_index(q, k, g, top_k, Kc, mode=REFINE, out=None, out_scores=None, stre
     if out_proxy is not None:
         out_proxy = _out(out_proxy, (G, H, d), torch.float32, q.device, "out_proxy")
     if out_cand is not None:
-        out_cand = _out(out_cand, (G, H, Kc), torch.int32, q.device, "out_cand")
+        out_cand = _out(out_cand, (L if scan == "member" else G, H, Kc), torch.int32, q.device, "out_cand")
     sp = _stream_ptr(stream)
     n = lib.pivot_workspace_size(L, H, d, g, top_k, Kc, bits)
     ws = _workspace(n, q.device, sp)

@@ -4,6 +4,7 @@
 // Prefill (pivot_index / dense_index), per head pass:
 //   proxy_kernel        group means -> fp32 proxies and their three bf16
 //                       terms                                 (skipped for dense)
+//   proxy_expand_kernel the proxies copied to every position  (per-member scan only)
 //   scan_filter_kernel  tcgen05 prefix scan + threshold filter -> spill lists
 //   finalize_kernel     exact top-K per row from the spill list
 //   fallback_kernel     exact recompute for rows the filter could not settle
@@ -168,10 +169,11 @@ constexpr size_t kSpillBudget = size_t(8) << 30;  // spill bytes per head pass
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Plan {
-  // sizes
-  int G, cap, S, K_sel, heads_per_pass, nfb;
+  // sizes: G = scan rows per head (groups; positions for dense and the
+  // per-member scan), Gg = groups (proxy rows)
+  int G, Gg, cap, S, K_sel, heads_per_pass, nfb;
   // offsets
-  size_t off_proxy, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, off_miss, total;
+  size_t off_proxy, off_proxy_e, off_spill, off_cnt, off_fb, off_fblist, off_fbscratch, off_cand, off_miss, total;
 };
 
 // Sample stride and spill capacity for a select of K_sel keys per row over
@@ -193,9 +195,18 @@ void filter_shape(int K_sel, int L, int* cap, int* S) {
 size_t miss_cap(size_t units, int g) { return units * static_cast<size_t>((g + 15) / 16) * 16; }
 size_t miss_bytes(size_t units, int g) { return up(sizeof(int)) + up(miss_cap(units, g) * sizeof(int2)); }
 
-Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool dense, int sms) {
+// The mode argument: PIVOT_REFINE or PIVOT_REUSE, optionally OR-ed with
+// PIVOT_PROXY_BF16 and (Refine) PIVOT_PER_MEMBER_SCAN.
+int base_mode(int mode) { return mode & ~static_cast<int>(PIVOT_PROXY_BF16 | PIVOT_PER_MEMBER_SCAN); }
+bool proxy_bf16(int mode) { return (mode & PIVOT_PROXY_BF16) != 0; }
+bool per_member_scan(int mode) { return (mode & PIVOT_PER_MEMBER_SCAN) != 0; }
+
+Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode_bits, bool dense, int sms) {
+  const int mode = base_mode(mode_bits);
+  const bool pm = !dense && mode == PIVOT_REFINE && per_member_scan(mode_bits);
   Plan p{};
-  p.G = dense ? L : (L + g - 1) / g;
+  p.Gg = dense ? L : (L + g - 1) / g;
+  p.G = pm ? L : p.Gg;
   p.K_sel = (dense || mode == PIVOT_REUSE) ? top_k : Kc;
   filter_shape(p.K_sel, L, &p.cap, &p.S);
   const size_t per_head_spill = static_cast<size_t>(p.G) * p.cap * sizeof(uint2);
@@ -203,9 +214,12 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   p.nfb = 2 * std::max(1, sms);
   const size_t rows_pass = static_cast<size_t>(p.heads_per_pass) * p.G;
   size_t o = 0;
-  // fp32 proxies [G][H][d], then their bf16 terms [3][G][H][d]
+  // fp32 proxies [Gg][H][d], then their bf16 terms [3][Gg][H][d]; for the
+  // per-member scan the same per position, [L][H][d] and [3][L][H][d]
   p.off_proxy = o;
-  o += dense ? 0 : up(static_cast<size_t>(p.G) * H * d * 4) + up(static_cast<size_t>(3) * p.G * H * d * 2);
+  o += dense ? 0 : up(static_cast<size_t>(p.Gg) * H * d * 4) + up(static_cast<size_t>(3) * p.Gg * H * d * 2);
+  p.off_proxy_e = o;
+  o += pm ? up(static_cast<size_t>(L) * H * d * 4) + up(static_cast<size_t>(3) * L * H * d * 2) : 0;
   p.off_spill = o;
   o += up(rows_pass * p.cap * sizeof(uint2));
   p.off_cnt = o;
@@ -219,7 +233,7 @@ Plan plan_prefill(int L, int H, int d, int g, int top_k, int Kc, int mode, bool 
   p.off_cand = o;
   o += (!dense && mode == PIVOT_REFINE) ? up(static_cast<size_t>(H) * p.G * cand_row_words(Kc) * sizeof(int32_t)) : 0;
   p.off_miss = o;
-  o += (!dense && mode == PIVOT_REFINE) ? miss_bytes(static_cast<size_t>(H) * p.G, g) : 0;
+  o += (!dense && mode == PIVOT_REFINE) ? miss_bytes(static_cast<size_t>(H) * p.G, pm ? 1 : g) : 0;
   p.total = o;
   return p;
 }
@@ -233,9 +247,6 @@ uint32_t tmem_cols_for(int Kc) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// The mode argument: PIVOT_REFINE or PIVOT_REUSE, optionally OR-ed with PIVOT_PROXY_BF16.
-int base_mode(int mode) { return mode & ~static_cast<int>(PIVOT_PROXY_BF16); }
-bool proxy_bf16(int mode) { return (mode & PIVOT_PROXY_BF16) != 0; }
 
 int check_common(const void* q, const void* k, int H, int d, int top_k, int Kc, int mode, const void* out) {
   if (!q || !k || !out) return fail(PIVOT_ERR_INVALID_ARG, "null tensor pointer");
@@ -246,7 +257,10 @@ int check_common(const void* q, const void* k, int H, int d, int top_k, int Kc, 
   if (top_k < 1 || Kc < top_k || Kc > 4096)
     return fail(PIVOT_ERR_INVALID_ARG, "need 1 <= top_k <= Kc <= 4096 (top_k=%d, Kc=%d)", top_k, Kc);
   if (base_mode(mode) != PIVOT_REFINE && base_mode(mode) != PIVOT_REUSE)
-    return fail(PIVOT_ERR_INVALID_ARG, "mode must be PIVOT_REFINE or PIVOT_REUSE, optionally | PIVOT_PROXY_BF16");
+    return fail(PIVOT_ERR_INVALID_ARG,
+                "mode must be PIVOT_REFINE or PIVOT_REUSE, optionally | PIVOT_PROXY_BF16 (| PIVOT_PER_MEMBER_SCAN)");
+  if (per_member_scan(mode) && base_mode(mode) != PIVOT_REFINE)
+    return fail(PIVOT_ERR_INVALID_ARG, "PIVOT_PER_MEMBER_SCAN applies to PIVOT_REFINE only");
   return PIVOT_OK;
 }
 
@@ -329,33 +343,46 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
   if (out_proxy && !aligned16(out_proxy)) return fail(PIVOT_ERR_INVALID_ARG, "out_proxy must be 16-byte aligned");
   if (out_cand && mode != PIVOT_REFINE)
     return fail(PIVOT_ERR_INVALID_ARG, "out_cand is only produced in PIVOT_REFINE mode");
+  if (per_member_scan(mode_bits) && (dense || mode != PIVOT_REFINE))
+    return fail(PIVOT_ERR_INVALID_ARG, "PIVOT_PER_MEMBER_SCAN applies to PIVOT_REFINE only");
+  const bool pm = per_member_scan(mode_bits);
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
-  const Plan pl = plan_prefill(L, H, d, dense ? 1 : g, top_k, Kc, mode, dense, dev->sms);
+  const Plan pl = plan_prefill(L, H, d, dense ? 1 : g, top_k, Kc, mode_bits, dense, dev->sms);
   if (!ws || ws_bytes < pl.total)
     return fail(PIVOT_ERR_WORKSPACE, "workspace too small: need %zu bytes, got %zu", pl.total, ws_bytes);
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return fail(PIVOT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   uint8_t* w = static_cast<uint8_t*>(ws);
-  // scan operand: the queries themselves (dense), else the proxies' bf16 terms
-  float* P32 = dense ? nullptr : reinterpret_cast<float*>(w + pl.off_proxy);
-  const uint16_t* P = dense ? static_cast<const uint16_t*>(q)
-                            : reinterpret_cast<const uint16_t*>(w + pl.off_proxy +
-                                                                up(static_cast<size_t>(pl.G) * H * d * 4));
+  // scan operand: the queries themselves (dense), else the proxies' bf16
+  // terms (per group; for the per-member scan copied to every position)
+  float* P32g = dense ? nullptr : reinterpret_cast<float*>(w + pl.off_proxy);
+  uint16_t* P3g = dense ? nullptr : reinterpret_cast<uint16_t*>(w + pl.off_proxy + up(static_cast<size_t>(pl.Gg) * H * d * 4));
+  float* P32e = pm ? reinterpret_cast<float*>(w + pl.off_proxy_e) : nullptr;
+  uint16_t* P3e = pm ? reinterpret_cast<uint16_t*>(w + pl.off_proxy_e + up(static_cast<size_t>(L) * H * d * 4)) : nullptr;
+  const float* P32 = pm ? P32e : P32g;
+  const uint16_t* P = dense ? static_cast<const uint16_t*>(q) : (pm ? P3e : P3g);
   const int gg = dense ? 1 : g;
+  const int g_scan = pm ? 1 : gg;   // members per scan row
   const bool refine = !dense && mode == PIVOT_REFINE;
   // a proxy of one member is that member's bf16 query: its mid and lo terms are zero
   const int nterms = (dense || gg == 1 || proxy_bf16(mode_bits)) ? 1 : 3;
 
   if (!dense) {
-    const long long n = static_cast<long long>(pl.G) * H * (d / 8);
+    const long long n = static_cast<long long>(pl.Gg) * H * (d / 8);
     TraceScope tr("proxy", st);
     proxy_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-        static_cast<const uint16_t*>(q), P32, const_cast<uint16_t*>(P), pl.G, H, d, gg, L, 0,
-        proxy_bf16(mode_bits) ? 1 : 0);
+        static_cast<const uint16_t*>(q), P32g, P3g, pl.Gg, H, d, gg, L, 0, proxy_bf16(mode_bits) ? 1 : 0);
     CUDA_TRY(cudaGetLastError());
     if (out_proxy)
-      CUDA_TRY(cudaMemcpyAsync(out_proxy, P32, static_cast<size_t>(pl.G) * H * d * 4, cudaMemcpyDeviceToDevice, st));
+      CUDA_TRY(cudaMemcpyAsync(out_proxy, P32g, static_cast<size_t>(pl.Gg) * H * d * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  if (pm) {
+    const long long n = static_cast<long long>(L) * H * (d / 8);
+    TraceScope tr("proxy_expand", st);
+    proxy_expand_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(P32g, P3g, P32e, P3e, pl.Gg, L, H,
+                                                                                   d, g);
+    CUDA_TRY(cudaGetLastError());
   }
 
   for (int h0 = 0; h0 < H; h0 += pl.heads_per_pass) {
@@ -371,8 +398,10 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     sp.G = pl.G;
     sp.L = L;
     sp.H = H;
-    sp.g = gg;
-    sp.bound_kind = refine ? 0 : 1;
+    sp.g = g_scan;
+    // Refine: row i sees j < last(i); Reuse and dense: j < i*g; the
+    // per-member scan: position i sees j < i
+    sp.bound_kind = (refine && !pm) ? 0 : 1;
     sp.K_sel = pl.K_sel;
     sp.cap = pl.cap;
     sp.S = pl.S;
@@ -389,7 +418,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     fp.G = pl.G;
     fp.L = L;
     fp.H = H;
-    fp.g = gg;
+    fp.g = g_scan;
     fp.bound_kind = sp.bound_kind;
     fp.K_sel = pl.K_sel;
     fp.cap = pl.cap;
@@ -439,7 +468,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.G = pl.G;
     rp.L = L;
     rp.H = H;
-    rp.g = g;
+    rp.g = g_scan;   // the per-member scan: one member per unit, its own candidate row
     rp.top_k = top_k;
     rp.Kc = Kc;
     rp.d = d;
@@ -447,8 +476,8 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.status = dev->status;
     rp.wait_ns = wait_limit_ns();
     if (out_cand) {
-      cand_export_kernel<<<static_cast<unsigned>(H * pl.G), 256, 0, st>>>(rp.cand, out_cand, pl.G, H, Kc, g, L,
-                                                                          nullptr, 0);
+      cand_export_kernel<<<static_cast<unsigned>(H * pl.G), 256, 0, st>>>(rp.cand, out_cand, pl.G, H, Kc, g_scan,
+                                                                          L, nullptr, 0);
       CUDA_TRY(cudaGetLastError());
     }
     uint8_t* miss = w + pl.off_miss;
@@ -472,6 +501,7 @@ int check_decode(const void* q, const void* kc, const int32_t* cu, int B, int H,
                  int mode, int max_seqlen, const void* out, const void* out_scores) {
   if (int rc = check_common(q, kc, H, d, top_k, Kc, mode, out)) return rc;
   if (!cu) return fail(PIVOT_ERR_INVALID_ARG, "null cu_seqlens");
+  if (per_member_scan(mode)) return fail(PIVOT_ERR_INVALID_ARG, "PIVOT_PER_MEMBER_SCAN applies to the prefill entry points only");
   if (B < 1 || g < 1 || max_seqlen < g) return fail(PIVOT_ERR_INVALID_ARG, "need B >= 1, g >= 1, max_seqlen >= g");
   if (max_seqlen >= (1 << 30)) return fail(PIVOT_ERR_INVALID_ARG, "max_seqlen too large");
   if (out_scores && !aligned16(out_scores)) return fail(PIVOT_ERR_INVALID_ARG, "out_scores must be 16-byte aligned");
@@ -648,7 +678,7 @@ int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t*
 
 size_t pivot_workspace_size(int L, int H, int d, int g, int top_k, int Kc, int mode) {
   if (L < 1 || H < 1 || g < 1 || top_k < 1 || Kc < top_k) return 0;
-  return plan_prefill(L, H, d, g, top_k, Kc, base_mode(mode), false, device_sms()).total;
+  return plan_prefill(L, H, d, g, top_k, Kc, mode, false, device_sms()).total;
 }
 
 size_t dense_workspace_size(int L, int H, int d, int top_k) {
@@ -684,7 +714,7 @@ int pivot_index(const void* q, const void* k, int L, int H, int d, int g, int to
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = plan_prefill(L, H, d, g, top_k, Kc, base_mode(mode), false, dev->sms).total;
+  const size_t bytes = plan_prefill(L, H, d, g, top_k, Kc, mode, false, dev->sms).total;
   return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
     return run_prefill(q, k, L, H, d, g, top_k, Kc, mode, false, out_idx, nullptr, nullptr, nullptr, ws, n, st);
   });

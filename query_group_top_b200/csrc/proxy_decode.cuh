@@ -86,6 +86,32 @@ __global__ void proxy_kernel(const uint16_t* __restrict__ q, float* __restrict__
   }
 }
 
+// The listing's per-member Refine scans each member's own prefix with its
+// group's proxy ("Show Me The Code", pivot_refine: k[:pos] per member).  The
+// scan then treats positions as its rows, so every position gets a copy of
+// its group's proxy: P32e [L][H][d] fp32 and the bf16 terms P3e [3][L][H][d]
+// from P32 [G][H][d] and P3 [3][G][H][d].  One thread per (position, head,
+// 8 channels): 32-byte and three 16-byte copies.
+__global__ void proxy_expand_kernel(const float* __restrict__ P32, const uint16_t* __restrict__ P3,
+                                    float* __restrict__ P32e, uint16_t* __restrict__ P3e, int G, int L, int H,
+                                    int d, int g) {
+  const long long total = static_cast<long long>(L) * H * (d / 8);
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  const int c8 = static_cast<int>(t % (d / 8));
+  const long long ph = t / (d / 8);
+  const int h = static_cast<int>(ph % H);
+  const long long pos = ph / H;
+  const long long src = ((pos / g) * H + h) * d + c8 * 8;
+  const long long dst = (pos * H + h) * d + c8 * 8;
+  reinterpret_cast<float4*>(P32e + dst)[0] = reinterpret_cast<const float4*>(P32 + src)[0];
+  reinterpret_cast<float4*>(P32e + dst)[1] = reinterpret_cast<const float4*>(P32 + src)[1];
+  const long long tg = static_cast<long long>(G) * H * d, te = static_cast<long long>(L) * H * d;
+#pragma unroll
+  for (int term = 0; term < 3; ++term)
+    *reinterpret_cast<uint4*>(P3e + term * te + dst) = *reinterpret_cast<const uint4*>(P3 + term * tg + src);
+}
+
 struct DecodeParams {
   const uint16_t* kcache;   // [rows][H][d]
   const float* P;           // [B][H][d] fp32 proxies

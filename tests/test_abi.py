@@ -54,6 +54,11 @@ def test_argument_errors_before_device_work(lib):
     assert lib.pivot_index(p + 2, p, 16, 1, 64, 4, 2, 4, 0, p, None) == 1      # misaligned
     assert lib.dense_index(p, p, 16, 1, 64, 0, p, None) == 1
     assert lib.pivot_decode_index(p, p, None, 1, 1, 64, 2, 2, 4, 0, 16, p, None) == 1
+    # the per-member scan is a Refine variant of the prefill entry points
+    assert lib.pivot_index(p, p, 16, 1, 64, 4, 2, 4, 1 | 0x200, p, None) == 1   # with Reuse
+    cu = (ctypes.c_int32 * 2)(0, 16)
+    assert lib.pivot_decode_index_ws(p, p, ctypes.addressof(cu), 1, 1, 64, 2, 2, 4, 0x200, 16, p, None, p, 1 << 20,
+                                     None) == 1
 
 
 def test_no_device_means_unsupported(lib):

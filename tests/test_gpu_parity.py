@@ -110,6 +110,72 @@ def test_proxies_bit_exact_and_candidate_sets(shape, proxy):
     assert eq.mean() > 0.99
 
 
+PER_MEMBER_SHAPES = [
+    # L, H, d, g, top_k, Kc
+    (5, 2, 64, 3, 2, 4),
+    (300, 3, 128, 16, 24, 48),
+    (1000, 2, 64, 8, 37, 80),
+    (2049, 2, 128, 4, 100, 300),
+    (1500, 1, 128, 1, 40, 80),
+]
+
+
+@pytest.mark.parametrize("shape", PER_MEMBER_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_per_member_scan_refine(shape):
+    """The listing's reading of Refine ("Show Me The Code", pivot_refine: a
+    proxy scan over k[:pos] for each member): every member's candidate set is
+    the group proxy's top-Kc over its own prefix.  Checked in full against the
+    oracle's per-member mode; a row is exempt when its final select or its own
+    candidate select is a near tie."""
+    L, H, d, g, top_k, Kc = shape
+    q, k = synthetic.gen_prefill(L, H, d, seed=5 * L + g, rho=0.9)
+    qd, kd = to_dev(q), to_dev(k)
+    sc = torch.empty((L, H, top_k), dtype=torch.float32, device="cuda")
+    C = torch.empty((L, H, Kc), dtype=torch.int32, device="cuda")
+    out = qg.pivot_index(qd, kd, g, top_k, Kc, qg.REFINE, out_scores=sc, out_cand=C, scan="member")
+    assert qg.sync_status() & ~qg.FLAG_FALLBACK == 0
+    ref = oracle.prefill(q, k, g, top_k, Kc, oracle.REFINE_PER_MEMBER)
+    pos = np.broadcast_to(np.arange(L)[:, None], (L, H))
+    res = compare(out.cpu().numpy(), ref["out"], ref["edge"], pos, ref["member_cand_edge"], sc.cpu().numpy(),
+                  ref["score"])
+    assert_parity(res, f"per-member L={L} H={H} d={d} g={g} k={top_k} Kc={Kc}")
+    # every member's candidate row: min(Kc, pos) ascending indices below pos
+    device_rows_valid(C, 0, lambda p: torch.clamp(p, max=Kc))
+    # a group's last member scans the shared prefix j < last: same rows as the method
+    shared = qg.pivot_index(qd, kd, g, top_k, Kc, qg.REFINE)
+    last = torch.from_numpy(np.minimum(np.arange(0, L, g) + g, L) - 1).cuda()
+    ref_shared = oracle.prefill(q, k, g, top_k, Kc, oracle.REFINE)
+    lc = last.cpu().numpy()
+    ok = np.all(out[last].cpu().numpy() == shared[last].cpu().numpy(), axis=-1)
+    assert np.all(ok | near_tie(ref_shared["cand_edge"]) | near_tie(ref["edge"][lc]) |
+                  near_tie(ref_shared["edge"][lc]))
+
+
+def test_per_member_scan_c1_sampled():
+    """The per-member scan on the C1 workload (L=8192, H=16, g=8, k=256,
+    Kc=512): the whole layer on the GPU, 96 sampled groups by the oracle."""
+    c = synthetic.CONFIGS["C1"]
+    q, k = synthetic.make_prefill("C1")
+    L, H, _ = q.shape
+    g, top_k, Kc = c["g"], c["top_k"], c["Kc"]
+    G = (L + g - 1) // g
+    qd, kd = to_dev(q), to_dev(k)
+    sc = torch.empty((L, H, top_k), dtype=torch.float32, device="cuda")
+    out = qg.pivot_index(qd, kd, g, top_k, Kc, qg.REFINE, out_scores=sc, scan="member")
+    qg.sync_status()
+    device_rows_valid(out, 0, lambda p: torch.clamp(p, max=top_k))
+    gi, hi = sampled_units(G, H, 96, seed=L + 17)
+    r = oracle_threads(oracle.prefill_units, q, k, g, top_k, Kc, oracle.REFINE_PER_MEMBER, gi, hi)
+    for u, (i, h) in enumerate(zip(gi, hi)):
+        rows = np.arange(i * g, min(i * g + g, L))
+        nm = len(rows)
+        o = out[rows[0]:rows[-1] + 1, h].cpu().numpy()
+        s = sc[rows[0]:rows[-1] + 1, h].cpu().numpy()
+        res = compare(o, r["out"][u, :nm], r["edge"][u, :nm], rows, r["member_cand_edge"][u, :nm], s,
+                      r["score"][u, :nm])
+        assert_parity(res, f"C1 per-member group={i} head={h}")
+
+
 def test_exact_ties_and_fallback_rows():
     """Constant keys: every score of a row ties, the lowest indices win; the
     sampled threshold cannot separate them, so long rows go to the exact

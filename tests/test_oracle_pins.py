@@ -332,3 +332,23 @@ def test_threaded_oracle_runs_equal_serial_runs():
         b = oracle_threads(oracle.prefill_units, q, k, 8, 5, 11, mode, gi, hi, threads=3, want_cand=True)
         for key in a:
             np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+
+
+def test_member_candidate_edges_are_each_members_own_boundary():
+    """In the listing's Refine each member's candidate set is the top-Kc of the
+    group proxy's scores over its own prefix; the oracle reports that select's
+    Kc-th and (Kc+1)-th scores per member (the near-tie test of the CUDA
+    comparison).  Brute force: sort the member's prefix scores."""
+    import tests.brute as brute
+    L, H, d, g, top_k, Kc = 90, 2, 16, 4, 3, 10
+    q, k = synthetic.gen_prefill(L, H, d, seed=21, rho=0.9)
+    r = oracle.prefill(q, k, g, top_k, Kc, oracle.REFINE_PER_MEMBER)
+    qd, kd = brute.decode_bf16(q), brute.decode_bf16(k)
+    for h in range(H):
+        for pos in range(L):
+            s = pos // g * g
+            proxy = qd[s:min(s + g, L), h].mean(axis=0).astype(np.float32).astype(np.float64)
+            sc = np.sort(kd[:pos, h] @ proxy)[::-1]
+            K = min(Kc, pos)
+            exp = [sc[K - 1] if K >= 1 else np.nan, sc[K] if pos > K and K >= 1 else np.nan]
+            np.testing.assert_allclose(r["member_cand_edge"][pos, h], exp, rtol=1e-12, atol=0)
