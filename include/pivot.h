@@ -147,6 +147,25 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * MTP decode over a paged key cache (the layout of paged-attention serving
+ * engines).  kpages: bf16 [num_pages][page_size][H][d].  block_table: int32
+ * [B][max_pages] (device) maps sequence b's logical page p -- its keys
+ * p*page_size .. p*page_size + page_size - 1 -- to a page of kpages.
+ * seqlens: int32 [B] (device), the cache rows n_b + g that sequence b holds.
+ * page_size must be a power of two and max_pages * page_size >= max_seqlen
+ * (else PIVOT_ERR_INVALID_ARG).  Every page id that a sequence's first
+ * seqlens[b] keys use must index a page of kpages: the tables live on the
+ * device and are not checked.  Everything else -- q, the outputs, the
+ * workspace (pivot_decode_workspace_size), sequences longer than max_seqlen
+ * -- is as in pivot_decode_index_ws, and the results equal those of the same
+ * sequences packed contiguously.
+ */
+int pivot_decode_index_paged(const void* q, const void* kpages, const int32_t* block_table, const int32_t* seqlens,
+                             int B, int H, int d, int g, int page_size, int max_pages, int top_k, int Kc, int mode,
+                             int max_seqlen, int32_t* out_idx, float* out_scores, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * As the _ws variants, with two more nullable outputs that expose the
  * method's intermediate results ("How It Works": the proxy of each group and
  * its candidate set C = top-Kc of the proxy scores):

@@ -18,6 +18,7 @@ import os
 import torch
 
 __all__ = ["REFINE", "REUSE", "PROXY_BF16", "PER_MEMBER_SCAN", "PivotError", "pivot_index", "dense_index", "pivot_decode_index",
+           "pivot_decode_index_paged",
            "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED",
            "head_range"]
 
@@ -36,7 +37,7 @@ EXPORTED = (
     "pivot_workspace_size", "pivot_index_ws", "dense_workspace_size", "dense_index_ws",
     "pivot_decode_workspace_size", "pivot_decode_index_ws", "pivot_sync_status", "pivot_last_error",
     "pivot_trace_enable", "pivot_trace_collect", "pivot_decode_index_noalloc",
-    "pivot_index_ex", "pivot_decode_index_ex", "pivot_set_wait_limit",
+    "pivot_index_ex", "pivot_decode_index_ex", "pivot_set_wait_limit", "pivot_decode_index_paged",
 )
 
 
@@ -74,6 +75,7 @@ def load_library():
         "pivot_decode_index_noalloc": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P], I),
         "pivot_index_ex": ([P, P, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
         "pivot_decode_index_ex": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
+        "pivot_decode_index_paged": ([P, P, P, P, I, I, I, I, I, I, I, I, I, I, P, P, P, Z, P], I),
         "pivot_set_wait_limit": ([ctypes.c_ulonglong], I),
     }
     for name, (args, res) in sig.items():
@@ -232,6 +234,44 @@ def pivot_decode_index(q, kcache, cu_seqlens, g, top_k, Kc, mode=REFINE, max_seq
         rc = lib.pivot_decode_index_ex(q.data_ptr(), kcache.data_ptr(), cu_seqlens.data_ptr(), B, H, d, g, top_k,
                                        Kc, bits, int(max_seqlen), out.data_ptr(), _ptr(out_scores),
                                        _ptr(out_proxy), _ptr(out_cand), ws.data_ptr(), ws.numel(), sp)
+    _err(lib, rc)
+    return out
+
+
+def pivot_decode_index_paged(q, kpages, block_table, seqlens, g, top_k, Kc, mode=REFINE, max_seqlen=None,
+                             out=None, out_scores=None, stream=None, proxy="fp32"):
+    """PIVOT decode over a paged key cache: q bf16 [B, g, H, d], kpages bf16
+    [num_pages, page_size, H, d] (page_size a power of two), block_table int32
+    [B, max_pages] and seqlens int32 [B] on the device (sequence b's key j is
+    row j % page_size of page block_table[b, j // page_size]; it holds
+    seqlens[b] = n_b + g keys) -> int32 [B, g, H, top_k], as pivot_decode_index."""
+    lib = load_library()
+    bits = _mode_bits(mode, proxy)
+    _check_bf16("q", q, 4)
+    _check_bf16("kpages", kpages, 4)
+    B, gq, H, d = q.shape
+    if gq != g:
+        raise PivotError("q's second axis must equal g")
+    _, page_size, Hk, dk = kpages.shape
+    if (Hk, dk) != (H, d):
+        raise PivotError("kpages must be [num_pages, page_size, H, d] with q's H and d")
+    if (block_table.dtype != torch.int32 or not block_table.is_cuda or block_table.dim() != 2
+            or block_table.shape[0] != B or not block_table.is_contiguous()):
+        raise PivotError("block_table must be a contiguous int32 CUDA tensor [B, max_pages]")
+    if seqlens.dtype != torch.int32 or not seqlens.is_cuda or seqlens.numel() != B:
+        raise PivotError("seqlens must be an int32 CUDA tensor of B lengths")
+    if max_seqlen is None:
+        raise PivotError("max_seqlen (an upper bound on cache rows per sequence) is required")
+    out = _out(out, (B, g, H, top_k), torch.int32, q.device, "out")
+    if out_scores is not None:
+        out_scores = _out(out_scores, (B, g, H, top_k), torch.float32, q.device, "out_scores")
+    sp = _stream_ptr(stream)
+    n = lib.pivot_decode_workspace_size(B, H, d, g, top_k, Kc, bits, int(max_seqlen))
+    ws = _workspace(n, q.device, sp)
+    rc = lib.pivot_decode_index_paged(q.data_ptr(), kpages.data_ptr(), block_table.data_ptr(), seqlens.data_ptr(), B,
+                                      H, d, g, int(page_size), int(block_table.shape[1]), top_k, Kc, bits,
+                                      int(max_seqlen), out.data_ptr(), _ptr(out_scores), ws.data_ptr(), ws.numel(),
+                                      sp)
     _err(lib, rc)
     return out
 

@@ -285,7 +285,10 @@ int launch_scan(const CUtensorMap& tmP, const CUtensorMap& tmK, const ScanParams
 template <int D>
 int launch_refine(RefineParams rp, int units, int sms, uint8_t* miss, cudaStream_t st) {
   const int smem = RefineCfg<D>::smem_bytes(rp.Kc);
-  CUDA_TRY(cudaFuncSetAttribute(refine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  // a paged decode cache looks each candidate's key row up in the block table
+  const bool paged = rp.ci.block_table != nullptr;
+  auto kern = paged ? refine_kernel<D, true> : refine_kernel<D, false>;
+  CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   rp.nbatch = (rp.g + 15) / 16;
   rp.n_items = units * rp.nbatch;
   rp.miss_count = reinterpret_cast<int*>(miss);
@@ -296,7 +299,7 @@ int launch_refine(RefineParams rp, int units, int sms, uint8_t* miss, cudaStream
   const int grid = std::max(1, std::min(rp.n_items, sms));
   {
     TraceScope tr("refine", st);
-    refine_kernel<D><<<grid, RefineCfg<D>::NT, smem, st>>>(rp);
+    kern<<<grid, RefineCfg<D>::NT, smem, st>>>(rp);
   }
   CUDA_TRY(cudaGetLastError());
   const int fsmem = (2 * cand_row_words(rp.Kc) + 2 * rp.top_k) * 4;
@@ -316,13 +319,13 @@ int launch_refine(RefineParams rp, int units, int sms, uint8_t* miss, cudaStream
 // (prefill: the group's last position; decode: n_b + g - 1, or no candidates
 // for a sequence the decode scan skipped).
 __global__ void cand_export_kernel(const int32_t* __restrict__ cand, int32_t* __restrict__ out, int G, int H,
-                                   int Kc, int g, int L, const int32_t* __restrict__ cu, int max_seqlen) {
+                                   int Kc, int g, int L, CacheIndex ci, int max_seqlen) {
   const int h = blockIdx.x / G, u = blockIdx.x % G;
   int bound;
-  if (cu == nullptr) {
+  if (!ci.decode()) {
     bound = min(u * g + g, L) - 1;
   } else {
-    const int len = cu[u + 1] - cu[u];
+    const int len = ci.len(u);
     bound = (len > max_seqlen || len < g) ? 0 : len - 1;
   }
   const int n = min(Kc, max(bound, 0));
@@ -464,7 +467,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.cand = reinterpret_cast<const int32_t*>(w + pl.off_cand);
     rp.out = out;
     rp.out_scores = out_scores;
-    rp.cu = nullptr;
+    rp.ci = CacheIndex{};
     rp.G = pl.G;
     rp.L = L;
     rp.H = H;
@@ -477,7 +480,7 @@ int run_prefill(const void* q, const void* k, int L, int H, int d, int g, int to
     rp.wait_ns = wait_limit_ns();
     if (out_cand) {
       cand_export_kernel<<<static_cast<unsigned>(H * pl.G), 256, 0, st>>>(rp.cand, out_cand, pl.G, H, Kc, g_scan,
-                                                                          L, nullptr, 0);
+                                                                          L, CacheIndex{}, 0);
       CUDA_TRY(cudaGetLastError());
     }
     uint8_t* miss = w + pl.off_miss;
@@ -497,10 +500,20 @@ size_t decode_ws_size(int B, int H, int d, int g, int Kc, int mode, int max_seql
   return o;
 }
 
-int check_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, int d, int g, int top_k, int Kc,
+// The packed decode cache of the cu_seqlens entry points.
+CacheIndex packed(const int32_t* cu) { return CacheIndex{cu, nullptr, nullptr, 0, 0}; }
+
+int check_decode(const void* q, const void* kc, const CacheIndex& ci, int B, int H, int d, int g, int top_k, int Kc,
                  int mode, int max_seqlen, const void* out, const void* out_scores) {
   if (int rc = check_common(q, kc, H, d, top_k, Kc, mode, out)) return rc;
-  if (!cu) return fail(PIVOT_ERR_INVALID_ARG, "null cu_seqlens");
+  if (!ci.cu && !(ci.seqlens && ci.block_table))
+    return fail(PIVOT_ERR_INVALID_ARG, "null cu_seqlens (packed cache) or seqlens / block_table (paged cache)");
+  if (!ci.cu) {
+    if (ci.max_pages < 1 || ci.log2_page < 0 || ci.log2_page > 20)
+      return fail(PIVOT_ERR_INVALID_ARG, "need max_pages >= 1 and a page size that is a power of two <= 2^20");
+    if ((static_cast<long long>(ci.max_pages) << ci.log2_page) < max_seqlen)
+      return fail(PIVOT_ERR_INVALID_ARG, "max_seqlen exceeds max_pages * page_size");
+  }
   if (per_member_scan(mode)) return fail(PIVOT_ERR_INVALID_ARG, "PIVOT_PER_MEMBER_SCAN applies to the prefill entry points only");
   if (B < 1 || g < 1 || max_seqlen < g) return fail(PIVOT_ERR_INVALID_ARG, "need B >= 1, g >= 1, max_seqlen >= g");
   if (max_seqlen >= (1 << 30)) return fail(PIVOT_ERR_INVALID_ARG, "max_seqlen too large");
@@ -508,10 +521,10 @@ int check_decode(const void* q, const void* kc, const int32_t* cu, int B, int H,
   return PIVOT_OK;
 }
 
-int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, int d, int g, int top_k, int Kc,
+int run_decode(const void* q, const void* kc, const CacheIndex& ci, int B, int H, int d, int g, int top_k, int Kc,
                int mode_bits, int max_seqlen, int32_t* out, float* out_scores, float* out_proxy, int32_t* out_cand,
                void* ws, size_t ws_bytes, cudaStream_t st) {
-  if (int rc = check_decode(q, kc, cu, B, H, d, g, top_k, Kc, mode_bits, max_seqlen, out, out_scores)) return rc;
+  if (int rc = check_decode(q, kc, ci, B, H, d, g, top_k, Kc, mode_bits, max_seqlen, out, out_scores)) return rc;
   const int mode = base_mode(mode_bits);
   if (out_proxy && !aligned16(out_proxy)) return fail(PIVOT_ERR_INVALID_ARG, "out_proxy must be 16-byte aligned");
   if (out_cand && mode != PIVOT_REFINE)
@@ -540,7 +553,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
   DecodeParams dp{};
   dp.kcache = static_cast<const uint16_t*>(kc);
   dp.P = P;
-  dp.cu = cu;
+  dp.ci = ci;
   dp.scores = scores;
   dp.cand = mode == PIVOT_REFINE ? cand : nullptr;
   dp.out = out;
@@ -557,10 +570,11 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
   dim3 grid((max_seqlen + kDecChunk - 1) / kDecChunk, H, B);
   {
   TraceScope tr("decode_scan", st);
+  const bool paged = ci.cu == nullptr;
   if (d == 128)
-    decode_scan_kernel<128><<<grid, kDecNT, 0, st>>>(dp);
+    (paged ? decode_scan_kernel<128, true> : decode_scan_kernel<128, false>)<<<grid, kDecNT, 0, st>>>(dp);
   else
-    decode_scan_kernel<64><<<grid, kDecNT, 0, st>>>(dp);
+    (paged ? decode_scan_kernel<64, true> : decode_scan_kernel<64, false>)<<<grid, kDecNT, 0, st>>>(dp);
   }
   CUDA_TRY(cudaGetLastError());
   const int sel_smem = dp.K_sel * 8;
@@ -577,7 +591,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     rp.cand = cand;
     rp.out = out;
     rp.out_scores = out_scores;
-    rp.cu = cu;
+    rp.ci = ci;
     rp.max_seqlen = max_seqlen;
     rp.G = B;
     rp.L = 0;
@@ -590,7 +604,7 @@ int run_decode(const void* q, const void* kc, const int32_t* cu, int B, int H, i
     rp.status = dev->status;
     rp.wait_ns = wait_limit_ns();
     if (out_cand) {
-      cand_export_kernel<<<static_cast<unsigned>(H * B), 256, 0, st>>>(cand, out_cand, B, H, Kc, g, 0, cu, max_seqlen);
+      cand_export_kernel<<<static_cast<unsigned>(H * B), 256, 0, st>>>(cand, out_cand, B, H, Kc, g, 0, ci, max_seqlen);
       CUDA_TRY(cudaGetLastError());
     }
     uint8_t* miss = reinterpret_cast<uint8_t*>(cand) + up(static_cast<size_t>(H) * B * cand_row_words(Kc) * sizeof(int32_t));
@@ -657,7 +671,7 @@ extern "C" {
 int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
                                int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
                                float* out_scores, void* stream) {
-  if (int rc = check_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores))
+  if (int rc = check_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores))
     return rc;
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
@@ -671,7 +685,7 @@ int pivot_decode_index_noalloc(const void* q, const void* kcache, const int32_t*
   if (int rc = noalloc_scratch(&scratch)) return rc;
   // Nothing in the decode scratch has to start at zero: every word is written
   // before it is read within the call.
-  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
+  return run_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
                     nullptr, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -743,28 +757,41 @@ int dense_index(const void* q, const void* k, int L, int H, int d, int top_k, in
 int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d,
                           int g, int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx,
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
-  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
+  return run_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
                     nullptr, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pivot_decode_index_paged(const void* q, const void* kpages, const int32_t* block_table, const int32_t* seqlens,
+                             int B, int H, int d, int g, int page_size, int max_pages, int top_k, int Kc, int mode,
+                             int max_seqlen, int32_t* out_idx, float* out_scores, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (page_size < 1 || (page_size & (page_size - 1)) != 0)
+    return fail(PIVOT_ERR_INVALID_ARG, "page_size must be a power of two (got %d)", page_size);
+  int log2_page = 0;
+  while ((1 << log2_page) < page_size) ++log2_page;
+  const CacheIndex ci{nullptr, seqlens, block_table, max_pages, log2_page};
+  return run_decode(q, kpages, ci, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr, nullptr,
+                    workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int pivot_decode_index_ex(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d, int g,
                           int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx, float* out_scores,
                           float* out_proxy, int32_t* out_cand, void* workspace, size_t workspace_bytes,
                           void* stream) {
-  return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, out_proxy,
+  return run_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, out_proxy,
                     out_cand, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int pivot_decode_index(const void* q, const void* kcache, const int32_t* cu_seqlens, int B, int H, int d, int g,
                        int top_k, int Kc, int mode, int max_seqlen, int32_t* out_idx, void* stream) {
-  if (int rc = check_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr))
+  if (int rc = check_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr))
     return rc;
   DeviceInfo* dev = nullptr;
   if (int rc = device_info(&dev)) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = decode_ws_size(B, H, d, g, Kc, mode, max_seqlen);
   return with_temp_workspace(bytes, st, [&](void* ws, size_t n) {
-    return run_decode(q, kcache, cu_seqlens, B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr, nullptr,
+    return run_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, nullptr, nullptr,
                       nullptr, ws, n, st);
   });
 }

@@ -25,6 +25,7 @@
 
 #include <cuda_bf16.h>
 
+#include "decode_cache.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
 
@@ -113,9 +114,9 @@ __global__ void proxy_expand_kernel(const float* __restrict__ P32, const uint16_
 }
 
 struct DecodeParams {
-  const uint16_t* kcache;   // [rows][H][d]
+  const uint16_t* kcache;   // packed [rows][H][d] or paged [pages][page_size][H][d]
   const float* P;           // [B][H][d] fp32 proxies
-  const int32_t* cu;        // [B+1]
+  CacheIndex ci;            // where each sequence's keys live
   uint32_t* scores;         // [H*B][max_seqlen] order keys
   int32_t* cand;            // [H][B][cand_row_words(K_sel)] candidate rows (Refine)
   int32_t* out;             // [B][g][H][width] (Reuse)
@@ -130,13 +131,15 @@ constexpr int kDecChunk = 2048;   // keys per scan CTA
 constexpr int kDecNT = 256;
 
 __device__ __forceinline__ bool decode_unit(const DecodeParams& p, int b, int& n_b, int& bound) {
-  const int len = p.cu[b + 1] - p.cu[b];
+  const int len = p.ci.len(b);
   n_b = len - p.g;
   bound = p.mode == 0 ? n_b + p.g - 1 : n_b;
   return len <= p.max_seqlen && n_b >= 0;
 }
 
-template <int D>
+// PAGED selects the cache layout at compile time, so the packed layout's
+// loop carries no page lookups.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kDecNT) decode_scan_kernel(DecodeParams p) {
   constexpr int LPK = D / 8;          // lanes per key row (16 bytes each)
   constexpr int KPW = 32 / LPK;       // key rows per warp step
@@ -159,7 +162,10 @@ __global__ void __launch_bounds__(kDecNT) decode_scan_kernel(DecodeParams p) {
     pf[0] = a.x; pf[1] = a.y; pf[2] = a.z; pf[3] = a.w;
     pf[4] = c.x; pf[5] = c.y; pf[6] = c.z; pf[7] = c.w;
   }
-  const uint16_t* kb = p.kcache + (static_cast<long long>(p.cu[b]) * p.H + h) * D + part * 8;
+  // packed: rows from the sequence's first cache row; paged: rows from the
+  // cache start, found through the block table
+  const long long r0 = PAGED ? 0 : static_cast<long long>(p.ci.cu[b]);
+  const uint16_t* kb = p.kcache + (r0 * p.H + h) * D + part * 8;
   const long long kstride = static_cast<long long>(p.H) * D;
   uint32_t* srow = p.scores + (static_cast<long long>(h) * p.B + b) * p.max_seqlen;
   constexpr int UNROLL = 4;
@@ -168,7 +174,11 @@ __global__ void __launch_bounds__(kDecNT) decode_scan_kernel(DecodeParams p) {
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
       const int j = base + u * NW * KPW + sub;
-      kv[u] = (j < j_end) ? __ldg(reinterpret_cast<const uint4*>(kb + j * kstride)) : make_uint4(0, 0, 0, 0);
+      if constexpr (PAGED)
+        kv[u] = (j < j_end) ? __ldg(reinterpret_cast<const uint4*>(kb + p.ci.row(b, 0, j) * kstride))
+                            : make_uint4(0, 0, 0, 0);
+      else
+        kv[u] = (j < j_end) ? __ldg(reinterpret_cast<const uint4*>(kb + j * kstride)) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {

@@ -53,6 +53,7 @@
 // refine_fallback_kernel redoes it exactly afterwards.
 #pragma once
 
+#include "decode_cache.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
 
@@ -64,7 +65,7 @@ struct RefineParams {
   const int32_t* cand;    // [H][G][cand_row_words(Kc)] candidate rows in read order (ptx.cuh)
   int32_t* out;           // prefill [L][H][top_k]; decode [B][g][H][top_k]
   float* out_scores;      // same shape as out, or null
-  const int32_t* cu;      // decode: [B+1] cache row offsets; null for prefill
+  CacheIndex ci;          // decode: where each sequence's keys live; all null for prefill
   int G, L, H, g, top_k, Kc, d;
   int max_seqlen;         // decode: sequences with more cache rows (or fewer than g) are skipped
   int n_items;            // H * G units x member batches
@@ -251,7 +252,7 @@ __device__ __forceinline__ uint32_t pick16(const uint32_t (&v)[16], int j) {
 struct RefineItem {
   int h, u, mb, nb, pos0, nc, nch;
   int jlim;             // candidate key indices lie in [0, jlim): the scan's bound
-  long long key_row0;   // cache row of key index 0
+  long long key_row0;   // cache row of key index 0 (packed layouts)
   long long qrow0;      // row (before *H) of member 0's query and output
 };
 
@@ -262,7 +263,7 @@ __device__ __forceinline__ RefineItem refine_item(const RefineParams& p, int ite
   it.h = ui / p.G;
   it.u = ui - it.h * p.G;
   int nm;
-  if (p.cu == nullptr) {
+  if (!p.ci.decode()) {
     const int s = it.u * p.g;
     nm = min(s + p.g, p.L) - s;
     it.pos0 = s;
@@ -270,8 +271,8 @@ __device__ __forceinline__ RefineItem refine_item(const RefineParams& p, int ite
     it.qrow0 = s;
   } else {
     nm = p.g;
-    it.key_row0 = p.cu[it.u];
-    const int len = p.cu[it.u + 1] - p.cu[it.u];
+    it.key_row0 = p.ci.row0(it.u);
+    const int len = p.ci.len(it.u);
     it.pos0 = len - p.g;
     it.qrow0 = static_cast<long long>(it.u) * p.g;
     if (len > p.max_seqlen || it.pos0 < 0) {
@@ -306,7 +307,9 @@ __device__ __forceinline__ int chunk_pos(int c, int nch) {
   return c < nch ? ((c & 1) ? ne + (c >> 1) : (c >> 1)) : c;
 }
 
-template <int D>
+// PAGED: decode keys behind a block table (the key row of each candidate is
+// looked up); else the rows of a sequence (or of the prefill) are contiguous.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
   using C = RefineCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -404,7 +407,8 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(RefineParams p) {
             // a missing candidate (-1 padding) reads as zeros; so would an
             // index outside the scan's bound, which no candidate row holds
             const bool in = j >= 0 && j < it.jlim;
-            const uint16_t* src = kbase + (in ? j : 0) * rowstride;
+            const long long row = PAGED ? p.ci.row(it.u, 0, in ? j : 0) : (in ? j : 0);
+            const uint16_t* src = kbase + row * rowstride;
             const uint32_t dst = dst0 + rr * 128 + ((p8 ^ (rr & 7)) << 4);
             const uint32_t nbytes = in ? 16u : 0u;
 #pragma unroll
@@ -1067,7 +1071,7 @@ __global__ void __launch_bounds__(kRfbNT) refine_fallback_kernel(RefineParams p)
       const int j = cl[t];
       float acc = 0.f;
       if (j >= 0 && j < it.jlim) {
-        const uint4* kr = reinterpret_cast<const uint4*>(kb + j * rowstride);
+        const uint4* kr = reinterpret_cast<const uint4*>(kb + p.ci.row(it.u, 0, j) * rowstride);
 #pragma unroll 4
         for (int c8 = 0; c8 < D / 8; ++c8) {
           const uint4 u = kr[c8];

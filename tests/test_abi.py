@@ -59,6 +59,10 @@ def test_argument_errors_before_device_work(lib):
     cu = (ctypes.c_int32 * 2)(0, 16)
     assert lib.pivot_decode_index_ws(p, p, ctypes.addressof(cu), 1, 1, 64, 2, 2, 4, 0x200, 16, p, None, p, 1 << 20,
                                      None) == 1
+    # paged cache: the page size must be a power of two, and the pages must cover max_seqlen
+    assert lib.pivot_decode_index_paged(p, p, p, p, 1, 1, 64, 2, 24, 4, 2, 4, 0, 16, p, None, p, 1 << 20, None) == 1
+    assert lib.pivot_decode_index_paged(p, p, p, p, 1, 1, 64, 2, 16, 1, 2, 4, 0, 17, p, None, p, 1 << 20, None) == 1
+    assert lib.pivot_decode_index_paged(p, p, None, p, 1, 1, 64, 2, 16, 4, 2, 4, 0, 16, p, None, p, 1 << 20, None) == 1
 
 
 def test_no_device_means_unsupported(lib):

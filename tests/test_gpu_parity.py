@@ -354,6 +354,62 @@ def test_decode_small(case, proxy):
         assert_parity(res, f"decode {case} mode={mode}")
 
 
+def paged_cache(dec, page_size, seed):
+    """The packed cache of `dec` laid out in pages: every sequence's rows cut
+    into pages of page_size rows, the pages placed in a random order (with a
+    few unused pages between them) and reached through a block table."""
+    rng = np.random.default_rng(seed)
+    cu = dec.cu_seqlens.astype(np.int64)
+    B = len(cu) - 1
+    lens = np.diff(cu)
+    npages = (lens + page_size - 1) // page_size
+    total = int(npages.sum()) + 5
+    order = rng.permutation(total)
+    _, H, d = dec.kcache.shape
+    kpages = np.zeros((total, page_size, H, d), np.uint16)
+    table = np.zeros((B, int(npages.max())), np.int32)
+    at = 0
+    for b in range(B):
+        for pg in range(int(npages[b])):
+            phys = int(order[at])
+            at += 1
+            rows = dec.kcache[cu[b] + pg * page_size:min(cu[b] + (pg + 1) * page_size, cu[b + 1])]
+            kpages[phys, :len(rows)] = rows
+            table[b, pg] = phys
+    return kpages, table, lens.astype(np.int32)
+
+
+@pytest.mark.parametrize("page_size", [16, 128])
+def test_paged_decode_equals_packed_and_oracle(page_size):
+    """A paged key cache (the serving layout): the keys of a packed cache cut
+    into pages in a random order behind a block table.  Refine and Reuse must
+    give the packed cache's rows and scores bit for bit, and match the oracle."""
+    B, H, d, g, top_k, Kc = 5, 2, 128, 3, 48, 96
+    dec = synthetic.gen_decode(B, H, d, g, seed=page_size + 3, lo=20, hi=2600)
+    max_seqlen = int(np.diff(dec.cu_seqlens).max())
+    kpages, table, lens = paged_cache(dec, page_size, seed=page_size)
+    qd, kp = to_dev(dec.q), to_dev(kpages)
+    bt, sl = torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda()
+    bi, hh = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+    for mode in (oracle.REFINE, oracle.REUSE):
+        want_rows, want_sc = run_decode(dec, g, top_k, Kc, mode, max_seqlen)
+        sc = torch.empty((B, g, H, top_k), dtype=torch.float32, device="cuda")
+        out = qg.pivot_decode_index_paged(qd, kp, bt, sl, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sc)
+        assert qg.sync_status() & ~qg.FLAG_FALLBACK == 0
+        got, gs = out.cpu().numpy(), sc.cpu().numpy()
+        np.testing.assert_array_equal(got, want_rows)
+        np.testing.assert_array_equal(gs.view(np.uint32), want_sc.view(np.uint32))
+        r = oracle.decode_units(dec.q, dec.kcache, dec.cu_seqlens, g, top_k, Kc, mode, bi.ravel(), hh.ravel())
+        want = r["out"].reshape(B, H, g, top_k).transpose(0, 2, 1, 3)
+        edge = r["edge"].reshape(B, H, g, 2).transpose(0, 2, 1, 3)
+        wsc = r["score"].reshape(B, H, g, top_k).transpose(0, 2, 1, 3)
+        cedge = None
+        if mode == oracle.REFINE:
+            cedge = np.broadcast_to(r["cand_edge"].reshape(B, H, 1, 2).transpose(0, 2, 1, 3), (B, g, H, 2))
+        pos = np.broadcast_to((dec.n_ctx[:, None] + np.arange(g)[None, :])[:, :, None], (B, g, H))
+        assert_parity(compare(got, want, edge, pos, cedge, gs, wsc), f"paged decode ps={page_size} mode={mode}")
+
+
 def test_c4_decode_sampled():
     """The MTP decode workload at full size (64 sequences, contexts up to 131072,
     19 GB of keys) in the launch configuration the bench times; the oracle
