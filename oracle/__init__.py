@@ -55,7 +55,9 @@ def _load():
         lib.oracle_prefill_units.argtypes = [P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_dense_units.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P]
         lib.oracle_decode_units.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P]
-        for f in (lib.oracle_prefill_units, lib.oracle_dense_units, lib.oracle_decode_units):
+        lib.oracle_sparse_attention.argtypes = [P, P, P, P, P, i, i, i, i, i, P]
+        for f in (lib.oracle_prefill_units, lib.oracle_dense_units, lib.oracle_decode_units,
+                  lib.oracle_sparse_attention):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -185,3 +187,28 @@ def decode_units(q, kcache, cu_seqlens, g, top_k, Kc, mode, seqs, heads, want_ca
     if rc != 0:
         raise ValueError("oracle_decode_units rejected its arguments")
     return dict(out=out, score=sc, edge=edge, cand=cand, cand_edge=cedge, proxy=p32, proxy_bf16=p16)
+
+
+def sparse_attention(q, k, v, idx, cu_seqlens=None, g=1):
+    """The attention that consumes the index rows: out[r, h] = softmax over the
+    row's valid indices of (q . k_j) * d^-1/2, applied to v_j (fp64); rows
+    without a valid index give zeros.  Prefill: q, k, v bf16 bits [R, H, d].
+    Decode: q [B, g, H, d] or [B*g, H, d], k and v the packed cache, index j of
+    sequence b at cache row cu_seqlens[b] + j.  idx int32 [..., H, top_k].
+    Returns float64 [R, H, d] (R = query rows)."""
+    lib = _load()
+    q = _u16(q)
+    k = _u16(k)
+    v = _u16(v)
+    H, d = q.shape[-2], q.shape[-1]
+    R = q.size // (H * d)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    top_k = idx.shape[-1]
+    if idx.size != R * H * top_k or k.shape != v.shape:
+        raise ValueError("sparse_attention: shapes do not agree")
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    out = np.empty((R, H, d), np.float64)
+    rc = lib.oracle_sparse_attention(_p(q), _p(k), _p(v), _p(idx), _p(cu), R, H, d, g, top_k, _p(out))
+    if rc != 0:
+        raise ValueError("oracle_sparse_attention rejected its arguments")
+    return out

@@ -351,3 +351,54 @@ int oracle_decode_units(const uint16_t *q, const uint16_t *kcache, const int32_t
     free(mq); free(mpos);
     return rc;
 }
+
+/*
+ * The sparse attention that consumes the index rows ("Show Me The Code", the
+ * demo after pivot_refine): for query row r and head h, with the valid
+ * indices J of its row (entries >= 0; -1 is padding),
+ *     s_j = (q . k_j) * d^-1/2,   w = softmax(s) over J,   out = sum_j w_j v_j,
+ * all in fp64 on the bf16 inputs.  A row without a valid index (position 0)
+ * gets zeros, as the demo leaves out[0].  Prefill (cu == NULL): q, k, v are
+ * [R, H, d] and index j is key row j.  Decode (cu != NULL): q is [R, H, d]
+ * with R = B*g (row r is member r % g of sequence r / g), k and v are the
+ * packed cache [rows, H, d] and index j of sequence b is cache row cu[b] + j.
+ * idx [R, H, top_k] int32; out [R, H, d] fp64.  Returns 0, or -1 on bad
+ * arguments.
+ */
+int oracle_sparse_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *idx,
+                            const int32_t *cu, int R, int H, int d, int g, int top_k, double *out)
+{
+    if (R < 1 || H < 1 || d < 1 || top_k < 1 || (cu && g < 1)) return -1;
+    double *s = (double *)malloc(sizeof(double) * (size_t)top_k);
+    if (!s) return -1;
+    const double scale = 1.0 / sqrt((double)d);
+    for (int r = 0; r < R; ++r) {
+        long base = cu ? (long)cu[r / g] : 0;
+        for (int h = 0; h < H; ++h) {
+            const int32_t *row = idx + ((long)r * H + h) * top_k;
+            const uint16_t *qr = q + ((long)r * H + h) * d;
+            double *o = out + ((long)r * H + h) * d;
+            double m = -INFINITY;
+            int any = 0;
+            for (int t = 0; t < top_k; ++t) {
+                if (row[t] < 0) continue;
+                s[t] = dot(qr, k + ((base + row[t]) * H + h) * (long)d, d) * scale;
+                if (s[t] > m) m = s[t];
+                any = 1;
+            }
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            if (!any) continue;
+            double z = 0.0;
+            for (int t = 0; t < top_k; ++t) {
+                if (row[t] < 0) continue;
+                double w = exp(s[t] - m);
+                z += w;
+                const uint16_t *vr = v + ((base + row[t]) * H + h) * (long)d;
+                for (int c = 0; c < d; ++c) o[c] += w * bf16_val(vr[c]);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= z;
+        }
+    }
+    free(s);
+    return 0;
+}

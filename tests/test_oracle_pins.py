@@ -352,3 +352,73 @@ def test_member_candidate_edges_are_each_members_own_boundary():
             K = min(Kc, pos)
             exp = [sc[K - 1] if K >= 1 else np.nan, sc[K] if pos > K and K >= 1 else np.nan]
             np.testing.assert_allclose(r["member_cand_edge"][pos, h], exp, rtol=1e-12, atol=0)
+
+
+# ------------------------------------------------- the sparse-attention consumer
+def _attend_brute(q, k, v, idx, base=None):
+    """numpy restatement: softmax over each row's valid indices of
+    (q . k_j) / sqrt(d), times v_j; zeros for a row without indices."""
+    import tests.brute as brute
+    qd, kd, vd = brute.decode_bf16(q), brute.decode_bf16(k), brute.decode_bf16(v)
+    R, H, d = qd.shape
+    out = np.zeros((R, H, d))
+    for r in range(R):
+        b0 = 0 if base is None else base[r]
+        for h in range(H):
+            sel = idx[r, h][idx[r, h] >= 0] + b0
+            if sel.size == 0:
+                continue
+            s = kd[sel, h] @ qd[r, h] / np.sqrt(d)
+            w = np.exp(s - s.max())
+            out[r, h] = (w / w.sum()) @ vd[sel, h]
+    return out
+
+
+def test_sparse_attention_matches_brute_force():
+    rng = np.random.default_rng(40)
+    L, H, d, top_k = 40, 3, 16, 6
+    q, k = synthetic.gen_iid(L, H, d, seed=41)
+    v, _ = synthetic.gen_iid(L, H, d, seed=42)
+    idx = -np.ones((L, H, top_k), np.int32)
+    for pos in range(L):
+        for h in range(H):
+            n = min(top_k, pos) - int(rng.integers(0, 2))
+            if n > 0:
+                idx[pos, h, :n] = np.sort(rng.choice(pos, size=n, replace=False))
+    got = oracle.sparse_attention(q, k, v, idx)
+    np.testing.assert_allclose(got, _attend_brute(q, k, v, idx), rtol=1e-12, atol=1e-12)
+    # decode layout: rows of sequence b start at cu[b]
+    B, g = 4, 2
+    cu = np.array([0, 9, 20, 30, 40], np.int32)
+    qd, _ = synthetic.gen_iid(B * g, H, d, seed=43)
+    idx2 = -np.ones((B * g, H, top_k), np.int32)
+    for r in range(B * g):
+        n_b = int(cu[r // g + 1] - cu[r // g]) - g
+        pos = n_b + r % g
+        for h in range(H):
+            idx2[r, h, :min(top_k, pos)] = np.sort(rng.choice(pos, size=min(top_k, pos), replace=False))
+    got2 = oracle.sparse_attention(qd, k, v, idx2, cu_seqlens=cu, g=g)
+    want2 = _attend_brute(qd, k, v, idx2, base=np.repeat(cu[:-1], g))
+    np.testing.assert_allclose(got2, want2, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_attention_closed_forms():
+    """One index: the output is that value row exactly.  Equal keys: equal
+    weights, the mean of the selected value rows.  No index: zeros.  The
+    demo's shape ("Show Me The Code"): (1024, 8, 64)."""
+    L, H, d = 12, 2, 8
+    q, k = synthetic.gen_iid(L, H, d, seed=44)
+    v, _ = synthetic.gen_iid(L, H, d, seed=45)
+    import tests.brute as brute
+    vd = brute.decode_bf16(v)
+    idx = -np.ones((L, H, 4), np.int32)
+    idx[5, 0, 0] = 3
+    idx[7, 1, :3] = [0, 2, 6]
+    kc = synthetic.bf16_from_f32(np.ones((L, H, d), np.float32))
+    out = oracle.sparse_attention(q, kc, v, idx)
+    np.testing.assert_array_equal(out[5, 0], vd[3, 0])
+    np.testing.assert_allclose(out[7, 1], vd[[0, 2, 6], 1].mean(axis=0), rtol=1e-14, atol=1e-15)
+    assert np.all(out[0] == 0) and np.all(out[6] == 0)
+    q0, k0 = synthetic.make_prefill("C0")
+    idx0 = np.zeros((1024, 8, 64), np.int32)
+    assert oracle.sparse_attention(q0, k0, k0, idx0).shape == (1024, 8, 64)
