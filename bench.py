@@ -623,7 +623,28 @@ def main():
                   "decode_scan_frac_of_measured_copy": dscan_gbs / pk["hbm"] if dscan_gbs else None,
                   "decode_step_hbm_frac": (key_bytes / (dec_ms / 1000.0) / 1e9) / NOMINAL_HBM_GBS,
                   "key_bytes": key_bytes}
-        del dq, dk, dcu, dout
+        # the sparse attention that consumes the step's index rows, over a
+        # value cache of the key cache's shape (seeded normal values); its
+        # algorithmic bytes: every selected key and value row once per query
+        # head, plus q, the index rows and the fp32 output
+        gen_v = torch.Generator(device="cuda")
+        gen_v.manual_seed(dc["seed"] * 7 + 1)
+        dv = torch.randn(dk.shape, generator=gen_v, device="cuda", dtype=torch.bfloat16)
+        att_out = torch.empty((nb, dc["g"], dc["H"], dc["d"]), dtype=torch.float32, device="cuda")
+        att = lambda: qg.sparse_attention(dq, dk, dv, dout, cu_seqlens=dcu, g=dc["g"], out=att_out)
+        for _ in range(2):
+            att()
+        att_ms = timed(att, args.steps)
+        qg.sync_status()
+        n_valid = int((dout >= 0).sum().item())
+        att_bytes = (n_valid * 2 * dc["d"] * 2 + dout.numel() * 4 + dq.numel() * 2 + att_out.numel() * 4)
+        decode["sparse_attention"] = {
+            "ms": att_ms, "selected_keys": n_valid, "algorithmic_bytes": att_bytes,
+            "gbs": att_bytes / (att_ms / 1000.0) / 1e9,
+            "hbm_frac_nominal": att_bytes / (att_ms / 1000.0) / 1e9 / NOMINAL_HBM_GBS,
+            "note": "gathers of the selected key and value rows; the MTP step's g members select mostly the "
+                    "same rows, so part of the gathers hit L2 and the rate can exceed the DRAM bandwidth"}
+        del dq, dk, dv, dcu, dout, att_out
         torch.cuda.empty_cache()
         w3 = config_work(cl)
         extras = {"refine_ms": ms_max, "reuse_ms": reuse_ms, "dense_ms": dense_ms, "decode": decode,

@@ -147,6 +147,26 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The sparse attention that consumes the index rows ("Show Me The Code": the
+ * demo after pivot_refine): for query row r, head h and the valid entries J of
+ * idx[r][h] (>= 0; -1 is padding),
+ *     out[r][h] = sum_{j in J} softmax_j((q[r][h] . k_j) * d^-1/2) v_j,
+ * with fp32 arithmetic; a row without a valid index gets zeros.
+ *   q:   bf16 [R][H][d]; prefill R = L, decode R = B*g (q of pivot_decode_index).
+ *   k,v: bf16; prefill [L][H][d] (index j = key row j); decode the packed cache
+ *        [rows][H][d] with cu_seqlens (device [B+1], index j of sequence
+ *        r / g = cache row cu_seqlens[r / g] + j); cu_seqlens NULL = prefill.
+ *   idx: int32 [R][H][top_k] (the indexer's output rows); every valid index
+ *        must address a key of its sequence -- it is not checked.
+ *   out: float32 [R][H][d].
+ * Asynchronous on `stream`; no workspace.  Returns PIVOT_OK,
+ * PIVOT_ERR_INVALID_ARG or PIVOT_ERR_UNSUPPORTED (d not 64/128, no sm_100).
+ */
+int pivot_sparse_attention(const void* q, const void* k, const void* v, const int32_t* idx,
+                           const int32_t* cu_seqlens, int R, int H, int d, int g, int top_k, float* out,
+                           void* stream);
+
+/*
  * MTP decode over a paged key cache (the layout of paged-attention serving
  * engines).  kpages: bf16 [num_pages][page_size][H][d].  block_table: int32
  * [B][max_pages] (device) maps sequence b's logical page p -- its keys

@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = ["REFINE", "REUSE", "PROXY_BF16", "PER_MEMBER_SCAN", "PivotError", "pivot_index", "dense_index", "pivot_decode_index",
-           "pivot_decode_index_paged",
+           "pivot_decode_index_paged", "sparse_attention",
            "sync_status", "trace_enable", "trace_collect", "library_path", "load_library", "EXPORTED",
            "head_range"]
 
@@ -38,6 +38,7 @@ EXPORTED = (
     "pivot_decode_workspace_size", "pivot_decode_index_ws", "pivot_sync_status", "pivot_last_error",
     "pivot_trace_enable", "pivot_trace_collect", "pivot_decode_index_noalloc",
     "pivot_index_ex", "pivot_decode_index_ex", "pivot_set_wait_limit", "pivot_decode_index_paged",
+    "pivot_sparse_attention",
 )
 
 
@@ -76,6 +77,7 @@ def load_library():
         "pivot_index_ex": ([P, P, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
         "pivot_decode_index_ex": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, Z, P], I),
         "pivot_decode_index_paged": ([P, P, P, P, I, I, I, I, I, I, I, I, I, I, P, P, P, Z, P], I),
+        "pivot_sparse_attention": ([P, P, P, P, P, I, I, I, I, I, P, P], I),
         "pivot_set_wait_limit": ([ctypes.c_ulonglong], I),
     }
     for name, (args, res) in sig.items():
@@ -272,6 +274,40 @@ def pivot_decode_index_paged(q, kpages, block_table, seqlens, g, top_k, Kc, mode
                                       H, d, g, int(page_size), int(block_table.shape[1]), top_k, Kc, bits,
                                       int(max_seqlen), out.data_ptr(), _ptr(out_scores), ws.data_ptr(), ws.numel(),
                                       sp)
+    _err(lib, rc)
+    return out
+
+
+def sparse_attention(q, k, v, idx, cu_seqlens=None, g=1, out=None, stream=None):
+    """The attention that consumes the index rows: for each query row and head,
+    softmax over the row's valid indices of (q . k_j) * d^-1/2, applied to v_j
+    (fp32; rows without indices give zeros).  Prefill: q, k, v bf16 [L, H, d],
+    idx int32 [L, H, top_k].  Decode: q bf16 [B, g, H, d], k and v the packed
+    cache [rows, H, d] with cu_seqlens int32 [B+1] (device), idx [B, g, H,
+    top_k].  Returns float32 with q's shape."""
+    lib = load_library()
+    _check_bf16("q", q, q.dim())
+    _check_bf16("k", k, 3)
+    _check_bf16("v", v, 3)
+    if k.shape != v.shape or k.shape[1:] != q.shape[-2:]:
+        raise PivotError("k and v must be [rows, H, d] with q's H and d")
+    H, d = q.shape[-2], q.shape[-1]
+    R = q.numel() // (H * d)
+    if (idx.dtype != torch.int32 or not idx.is_cuda or not idx.is_contiguous() or tuple(idx.shape[:-1]) != tuple(q.shape[:-1])):
+        raise PivotError("idx must be a contiguous int32 CUDA tensor [..., H, top_k] matching q")
+    top_k = idx.shape[-1]
+    cu_ptr = None
+    if cu_seqlens is not None:
+        if q.dim() != 4 or q.shape[1] != g:
+            raise PivotError("with cu_seqlens, q must be [B, g, H, d]")
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.numel() != q.shape[0] + 1:
+            raise PivotError("cu_seqlens must be an int32 CUDA tensor of B+1 offsets")
+        cu_ptr = cu_seqlens.data_ptr()
+    elif q.dim() != 3:
+        raise PivotError("prefill q must be [L, H, d]")
+    out = _out(out, tuple(q.shape), torch.float32, q.device, "out")
+    rc = lib.pivot_sparse_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), cu_ptr, R, H, d, g,
+                                    top_k, out.data_ptr(), _stream_ptr(stream))
     _err(lib, rc)
     return out
 

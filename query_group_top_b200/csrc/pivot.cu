@@ -11,6 +11,7 @@
 // then refine_kernel (Refine only): per-member re-score of the candidate set.
 // Decode (pivot_decode_index): proxy_kernel -> decode_scan_kernel ->
 // decode_select_kernel -> refine_kernel.
+// Consumer (pivot_sparse_attention): sparse_attention_kernel over index rows.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -23,6 +24,7 @@
 #include <vector>
 
 #include "../../include/pivot.h"
+#include "attend.cuh"
 #include "finalize.cuh"
 #include "proxy_decode.cuh"
 #include "ptx.cuh"
@@ -759,6 +761,43 @@ int pivot_decode_index_ws(const void* q, const void* kcache, const int32_t* cu_s
                           float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
   return run_decode(q, kcache, packed(cu_seqlens), B, H, d, g, top_k, Kc, mode, max_seqlen, out_idx, out_scores, nullptr,
                     nullptr, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pivot_sparse_attention(const void* q, const void* k, const void* v, const int32_t* idx,
+                           const int32_t* cu_seqlens, int R, int H, int d, int g, int top_k, float* out,
+                           void* stream) {
+  if (!q || !k || !v || !idx || !out) return fail(PIVOT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out))
+    return fail(PIVOT_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (R < 1 || H < 1 || top_k < 1 || (cu_seqlens && g < 1))
+    return fail(PIVOT_ERR_INVALID_ARG, "need R >= 1, H >= 1, top_k >= 1 (and g >= 1 with cu_seqlens)");
+  if (static_cast<long long>(R) * H >= (1ll << 31)) return fail(PIVOT_ERR_INVALID_ARG, "R * H too large");
+  if (d != 64 && d != 128) return fail(PIVOT_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", d);
+  DeviceInfo* dev = nullptr;
+  if (int rc = device_info(&dev)) return rc;
+  AttendParams ap{};
+  ap.q = static_cast<const uint16_t*>(q);
+  ap.k = static_cast<const uint16_t*>(k);
+  ap.v = static_cast<const uint16_t*>(v);
+  ap.idx = idx;
+  ap.cu = cu_seqlens;
+  ap.out = out;
+  ap.R = R;
+  ap.H = H;
+  ap.g = cu_seqlens ? g : 1;
+  ap.top_k = top_k;
+  ap.scale = 1.0f / sqrtf(static_cast<float>(d));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    TraceScope tr("sparse_attention", st);
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(R) * H);
+    if (d == 128)
+      sparse_attention_kernel<128><<<grid, kAttNT, 0, st>>>(ap);
+    else
+      sparse_attention_kernel<64><<<grid, kAttNT, 0, st>>>(ap);
+  }
+  CUDA_TRY(cudaGetLastError());
+  return PIVOT_OK;
 }
 
 int pivot_decode_index_paged(const void* q, const void* kpages, const int32_t* block_table, const int32_t* seqlens,

@@ -592,3 +592,58 @@ def test_bare_entry_points_allocate_their_own_workspace():
             cedge = np.broadcast_to(r["cand_edge"].reshape(3, H, 1, 2).transpose(0, 2, 1, 3), (3, 2, H, 2))
         dpos = np.broadcast_to((dec.n_ctx[:, None] + np.arange(2)[None, :])[:, :, None], (3, 2, H))
         assert_parity(compare(out.cpu().numpy(), want, edge, dpos, cedge), f"bare pivot_decode_index {mode}")
+
+
+# ------------------------------------------------- the sparse-attention consumer
+ATT_TOL = 1e-4   # fp32 online softmax over <= 4096 terms against the fp64 oracle
+
+
+def assert_attention_close(got, want, what):
+    err = np.abs(got.astype(np.float64) - want) / np.maximum(1.0, np.abs(want))
+    assert err.max() <= ATT_TOL, f"{what}: max relative error {err.max():.3g} at {np.unravel_index(err.argmax(), err.shape)}"
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_sparse_attention_prefill(d):
+    """The demo's consumer ("Show Me The Code"): softmax(q . k[sel] / sqrt(d)) @ v[sel]
+    per position and head, over the rows that the Refine indexer wrote (and a
+    ragged random set of rows with padding), against the fp64 oracle; position 0
+    has no index and gets zeros."""
+    L, H, g, top_k, Kc = 1024, 4, 8, 64, 128
+    q, k = synthetic.gen_prefill(L, H, d, seed=d + 1, rho=0.9)
+    v, _ = synthetic.gen_iid(L, H, d, seed=d + 2)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    idx = qg.pivot_index(qd, kd, g, top_k, Kc, qg.REFINE)
+    out = qg.sparse_attention(qd, kd, vd, idx)
+    qg.sync_status()
+    want = oracle.sparse_attention(q, k, v, idx.cpu().numpy())
+    got = out.cpu().numpy()
+    assert_attention_close(got, want, f"prefill d={d}")
+    assert np.all(got[0] == 0)
+    # ragged rows: random valid prefixes of a width that no stream count divides
+    rng = np.random.default_rng(d)
+    tk = 37
+    ridx = -np.ones((L, H, tk), np.int32)
+    for pos in range(1, L):
+        n = int(rng.integers(0, min(tk, pos) + 1))
+        ridx[pos, :, :n] = np.sort(rng.choice(pos, size=n, replace=False))
+    out2 = qg.sparse_attention(qd, kd, vd, torch.from_numpy(ridx).cuda())
+    assert_attention_close(out2.cpu().numpy(), oracle.sparse_attention(q, k, v, ridx), f"ragged d={d}")
+
+
+def test_sparse_attention_decode():
+    """The consumer after an MTP decode step: q [B, g, H, d], the packed key and
+    value caches, the decode indexer's rows."""
+    B, H, d, g, top_k, Kc = 4, 2, 128, 2, 256, 512
+    dec = synthetic.gen_decode(B, H, d, g, seed=77, lo=100, hi=3000)
+    rows = dec.kcache.shape[0]
+    v, _ = synthetic.gen_iid(rows, H, d, seed=78)
+    max_seqlen = int(np.diff(dec.cu_seqlens).max())
+    qd, kd, vd = to_dev(dec.q), to_dev(dec.kcache), to_dev(v)
+    cu = torch.from_numpy(dec.cu_seqlens).cuda()
+    idx = qg.pivot_decode_index(qd, kd, cu, g, top_k, Kc, qg.REFINE, max_seqlen=max_seqlen)
+    out = qg.sparse_attention(qd, kd, vd, idx, cu_seqlens=cu, g=g)
+    qg.sync_status()
+    want = oracle.sparse_attention(dec.q, dec.kcache, v, idx.cpu().numpy().reshape(B * g, H, top_k),
+                                   cu_seqlens=dec.cu_seqlens, g=g)
+    assert_attention_close(out.cpu().numpy().reshape(B * g, H, d), want, "decode")
