@@ -368,8 +368,9 @@ def run_reference(args, rank):
 
 
 def decode_only(args, qg, torch):
-    """The MTP decode step alone on a few sequences of its workload (a small
-    case for profiling the decode kernels); prints ms per step."""
+    """The MTP decode step alone on a few sequences of its workload, then the
+    sparse attention over its index rows (a small case for profiling the decode
+    kernels and the consumer); prints ms per step of each."""
     dc = synthetic.CONFIGS["C4"]
     B = min(args.decode_only, dc["B"])
     dq, dk, dcu, n_ctx = synthetic.gen_decode_device(dc["B"], dc["H"], dc["d"], dc["g"], dc["seed"], dc["lo"], dc["hi"],
@@ -387,10 +388,27 @@ def decode_only(args, qg, torch):
         step()
     e1.record()
     torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / args.steps
     qg.sync_status()
     key_bytes = float(n_ctx.astype(np.int64).sum() + B * (dc["g"] - 1)) * dc["H"] * dc["d"] * 2
-    print(json.dumps({"decode_only_sequences": B, "ms_per_step": e0.elapsed_time(e1) / args.steps,
-                      "key_bytes": key_bytes}), flush=True)
+    # then the sparse attention over the step's index rows (a value cache of
+    # the key cache's shape)
+    gen_v = torch.Generator(device="cuda")
+    gen_v.manual_seed(dc["seed"] * 7 + 1)
+    dv = torch.randn(dk.shape, generator=gen_v, device="cuda", dtype=torch.bfloat16)
+    att_out = torch.empty((B, dc["g"], dc["H"], dc["d"]), dtype=torch.float32, device="cuda")
+    att = lambda: qg.sparse_attention(dq, dk, dv, dout, cu_seqlens=dcu, g=dc["g"], out=att_out)
+    for _ in range(args.warmup):
+        att()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        att()
+    e1.record()
+    torch.cuda.synchronize()
+    qg.sync_status()
+    print(json.dumps({"decode_only_sequences": B, "ms_per_step": step_ms, "key_bytes": key_bytes,
+                      "sparse_attention_ms": e0.elapsed_time(e1) / args.steps}), flush=True)
 
 
 def main():
