@@ -55,7 +55,7 @@ def workload_config(c, world=1):
     return {"workload": f"{WORKLOAD} long-context prefill L={c['L']} H={c['H']} d={c['d']} g={c['g']} "
                         f"top_k={c['top_k']} Kc={c['Kc']} PIVOT-Refine",
             "generator": f"keys N(0,1) with {c['heavy_frac']*100:g}% positions x{c['heavy_scale']:g}; "
-                         f"queries AR(1) rho={c['rho']}; seed {c['seed']} (+rank)",
+                         f"queries AR(1) rho={c['rho']}; seed {c['seed']}",
             "l2": "inputs 1.07 GB and outputs 17.2 GB per step exceed the 126 MB L2; no flush needed",
             "parallelism": (f"heads split across {world} GPUs (rank r: heads [r*H/N, (r+1)*H/N)), "
                             "no collective on the data path")}
