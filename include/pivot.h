@@ -87,7 +87,9 @@ typedef enum {
  *     top-min(top_k, that count).
  *   mode = PIVOT_REUSE (listing pivot_reuse): scan keys j < s (group start);
  *     every member gets the proxy's top-min(top_k, s).  Kc is not used.
- *   Either may be OR-ed with PIVOT_PROXY_BF16 (the bf16-proxy variant).
+ *   Either may be OR-ed with PIVOT_PROXY_BF16 (the bf16-proxy variant);
+ *   PIVOT_REFINE also with PIVOT_PER_MEMBER_SCAN (the listing's per-member
+ *   scan).
  * q, k:     bf16 [L][H][d].
  * out_idx:  int32 [L][H][top_k].
  * Temporary device memory is taken with cudaMallocAsync on `stream` and freed
