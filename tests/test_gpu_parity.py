@@ -647,3 +647,76 @@ def test_sparse_attention_decode():
     want = oracle.sparse_attention(dec.q, dec.kcache, v, idx.cpu().numpy().reshape(B * g, H, top_k),
                                    cu_seqlens=dec.cu_seqlens, g=g)
     assert_attention_close(out.cpu().numpy().reshape(B * g, H, d), want, "decode")
+
+
+def test_sparse_attention_c4_sampled():
+    """The consumer at the decode workload's full size, in the launch
+    configuration the bench times (64 sequences, 19 GB of keys and as many
+    values, the decode indexer's rows): whole sequences checked by the oracle,
+    the longest and the shortest included."""
+    c = synthetic.CONFIGS["C4"]
+    g, top_k, Kc, H, d = c["g"], c["top_k"], c["Kc"], c["H"], c["d"]
+    q, kc, cu, n_ctx = synthetic.gen_decode_device(c["B"], H, d, g, c["seed"], c["lo"], c["hi"],
+                                                   c["rho"], c["heavy_frac"], c["heavy_scale"])
+    max_seqlen = int((n_ctx + g).max())
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(c["seed"] * 7 + 1)
+    vc = torch.randn(kc.shape, generator=gen, device="cuda", dtype=torch.bfloat16)
+    idx = qg.pivot_decode_index(q, kc, cu, g, top_k, Kc, qg.REFINE, max_seqlen=max_seqlen)
+    out = qg.sparse_attention(q, kc, vc, idx, cu_seqlens=cu, g=g)
+    qg.sync_status()
+    cu_h = cu.cpu().numpy()
+    rng = np.random.default_rng(45)
+    for b in [int(np.argmax(n_ctx)), int(np.argmin(n_ctx))] + list(rng.integers(0, c["B"], size=1)):
+        rows = slice(int(cu_h[b]), int(cu_h[b + 1]))
+        kb = kc[rows].cpu().view(torch.int16).numpy().view(np.uint16)
+        vb = vc[rows].cpu().view(torch.int16).numpy().view(np.uint16)
+        qb = q[b].cpu().view(torch.int16).numpy().view(np.uint16)          # [g, H, d]
+        want = oracle.sparse_attention(qb, kb, vb, idx[b].cpu().numpy(), cu_seqlens=np.array([0, kb.shape[0]], np.int32),
+                                       g=g)
+        assert_attention_close(out[b].cpu().numpy(), want, f"C4 consumer seq={b} n_ctx={n_ctx[b]}")
+    del kc, vc, out, idx
+    torch.cuda.empty_cache()
+
+
+def test_paged_decode_c4_equals_packed():
+    """The paged cache at the decode workload's full size: the 64 sequences'
+    keys moved into 64-row pages in a random order on the device; every row
+    and score must equal the packed cache's (Refine and Reuse)."""
+    c = synthetic.CONFIGS["C4"]
+    g, top_k, Kc, H, d = c["g"], c["top_k"], c["Kc"], c["H"], c["d"]
+    q, kc, cu, n_ctx = synthetic.gen_decode_device(c["B"], H, d, g, c["seed"], c["lo"], c["hi"],
+                                                   c["rho"], c["heavy_frac"], c["heavy_scale"])
+    max_seqlen = int((n_ctx + g).max())
+    ps = 64
+    cu_h = cu.cpu().numpy().astype(np.int64)
+    lens = np.diff(cu_h)
+    npages = (lens + ps - 1) // ps
+    total = int(npages.sum())
+    order = np.random.default_rng(46).permutation(total)
+    table = np.zeros((c["B"], int(npages.max())), np.int32)
+    src, dst = [], []
+    at = 0
+    for b in range(c["B"]):
+        for pg in range(int(npages[b])):
+            table[b, pg] = order[at]
+            r0 = pg * ps
+            n = int(min(ps, lens[b] - r0))
+            src.append(np.arange(cu_h[b] + r0, cu_h[b] + r0 + n))
+            dst.append(order[at] * ps + np.arange(n))
+            at += 1
+    kp = torch.zeros((total * ps, H, d), dtype=torch.bfloat16, device="cuda")
+    kp[torch.from_numpy(np.concatenate(dst)).cuda()] = kc[torch.from_numpy(np.concatenate(src)).cuda()]
+    kp = kp.view(total, ps, H, d)
+    bt = torch.from_numpy(table).cuda()
+    sl = torch.from_numpy(lens.astype(np.int32)).cuda()
+    for mode in (qg.REFINE, qg.REUSE):
+        sa = torch.empty((c["B"], g, H, top_k), dtype=torch.float32, device="cuda")
+        sb = torch.empty_like(sa)
+        a = qg.pivot_decode_index(q, kc, cu, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sa)
+        b = qg.pivot_decode_index_paged(q, kp, bt, sl, g, top_k, Kc, mode, max_seqlen=max_seqlen, out_scores=sb)
+        qg.sync_status()
+        assert torch.equal(a, b), f"mode={mode}"
+        assert torch.equal(sa.view(torch.int32), sb.view(torch.int32)), f"mode={mode}"
+    del kc, kp
+    torch.cuda.empty_cache()
