@@ -40,6 +40,14 @@ def test_workspace_sizes_are_host_arithmetic(lib):
     # the Refine candidate set alone: H * G * Kc int32
     assert a - b >= 16 * 8192 * 4096 * 4
     assert lib.pivot_workspace_size(0, 16, 128, 16, 2048, 4096, 0) == 0
+    # the per-member scan holds one candidate row per position (H * L * Kc
+    # int32) and the proxies copied to every position (L * H * d * (4 + 6) B)
+    L, H, d, g, k, Kc = 8192, 16, 128, 8, 256, 512
+    e = lib.pivot_workspace_size(L, H, d, g, k, Kc, qg.REFINE | qg.PER_MEMBER_SCAN)
+    f = lib.pivot_workspace_size(L, H, d, g, k, Kc, qg.REFINE)
+    assert e - f >= H * L * Kc * 4 - H * (L // g) * Kc * 4 + L * H * d * 10
+    # the bf16-proxy option changes no buffer size
+    assert lib.pivot_workspace_size(L, H, d, g, k, Kc, qg.REFINE | qg.PROXY_BF16) == f
 
 
 def test_argument_errors_before_device_work(lib):
